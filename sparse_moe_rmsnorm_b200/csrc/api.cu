@@ -1,0 +1,435 @@
+// C ABI of the B200 MoE block: context and workspace management, argument
+// validation, TMA descriptor encoding and the five stage launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "moe_b200.h"
+#include "kernels.cuh"
+
+namespace moe {
+cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
+cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+cudaError_t launch_finalize(const float *y_acc, uint16_t *y, long long n, cudaStream_t s);
+cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
+cudaError_t launch_selftest_wait(unsigned int *err, unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// u8 codes [E][R][K/2]: box {128 bytes, box_rows, 1}, 128-byte swizzle, zero fill out of range.
+bool encode_codes(CUtensorMap *m, const void *codes, int E, int R, int K, int box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)R, (cuuint64_t)E};
+    const cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R * (K / 2)};
+    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 [rows][cols]: box {64, box_rows}, 128-byte swizzle.
+bool encode_f16_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct moe_ctx {
+    moe_shape_t shape;
+    int device;
+    int num_sms;
+    void *ws;
+    size_t ws_bytes;
+    __half *xn16;
+    float *rho;
+    int *topk_idx;
+    float *topk_w;
+    int *counts, *offsets, *tiles;
+    int *row_token;
+    float *row_w;
+    __half *h;
+    float *y_acc;
+    unsigned int *err;
+    unsigned long long wait_limit_ns;
+    CUtensorMap map_xn16;   // gather4 rows of the normalised tokens
+    CUtensorMap map_h;      // 16-row boxes of h
+    const void *w13_ptr;
+    CUtensorMap map_w13;
+    const void *w2_ptr;
+    CUtensorMap map_w2;
+};
+
+namespace {
+
+struct Buf {
+    void *ptr;
+    size_t bytes;
+};
+
+Buf ws_buffer(moe_ctx *c, int which) {
+    const moe_shape_t &s = c->shape;
+    const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
+    switch (which) {
+        case MOE_WS_XN16: return {c->xn16, T * s.d_model * 2};
+        case MOE_WS_RHO: return {c->rho, T * 4};
+        case MOE_WS_TOPK_IDX: return {c->topk_idx, P * 4};
+        case MOE_WS_TOPK_W: return {c->topk_w, P * 4};
+        case MOE_WS_COUNTS: return {c->counts, E * 4};
+        case MOE_WS_OFFSETS: return {c->offsets, (E + 1) * 4};
+        case MOE_WS_ROW_TOKEN: return {c->row_token, P * 4};
+        case MOE_WS_ROW_W: return {c->row_w, P * 4};
+        case MOE_WS_H: return {c->h, P * s.d_ff * 2};
+        case MOE_WS_YACC: return {c->y_acc, T * s.d_model * 4};
+        case MOE_WS_TILES: return {c->tiles, (E + 1) * 4};
+        default: return {nullptr, 0};
+    }
+}
+
+int check_call(moe_ctx *c, int T, int top_k) {
+    if (!c) return MOE_ERR_ARG;
+    if (T < 0 || T > c->shape.T_max) return MOE_ERR_ARG;
+    if (top_k < 1 || top_k > c->shape.top_k) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Token rows per GEMM work item: the smallest multiple of 16 that holds every
+// token (an expert receives each token at most once), capped at 256.
+int token_block_rows(int T) {
+    int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;
+    return nb < 256 ? nb : 256;
+}
+
+int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
+                const uint16_t *bias, cudaStream_t stream) {
+    const moe_shape_t &s = c->shape;
+    GemmParams p;
+    memset(&p, 0, sizeof p);
+    const int E = s.n_experts, d = s.d_model, F = s.d_ff;
+    if (mode == MODE_UP) {
+        if (codes != c->w13_ptr) {
+            if (!encode_codes(&c->map_w13, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
+            c->w13_ptr = codes;
+        }
+        p.map_codes = c->map_w13;
+        p.map_b = c->map_xn16;
+        p.K = d;
+        p.R = 2 * F;
+        p.MB = F / 64;
+        p.out = c->h;
+        p.out_ld = F;
+    } else {
+        if (codes != c->w2_ptr) {
+            if (!encode_codes(&c->map_w2, codes, E, d, F, 128)) return MOE_ERR_CUDA;
+            c->w2_ptr = codes;
+        }
+        p.map_codes = c->map_w2;
+        p.map_b = c->map_h;
+        p.K = F;
+        p.R = d;
+        p.MB = (d + GEMM_BM - 1) / GEMM_BM;
+        p.out = c->y_acc;
+        p.out_ld = d;
+    }
+    p.scales = scales;
+    p.bias = bias;
+    p.F = F;
+    p.E = E;
+    p.nb_rows = token_block_rows(T);
+    p.b_stage_bytes = p.nb_rows * 128;
+    p.n_d_bufs = p.nb_rows <= 128 ? 2 : 1;
+    // TMEM: A slots first, then the accumulator buffer(s)
+    p.n_a_slots = (512 - p.n_d_bufs * p.nb_rows) / 32;
+    if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
+    p.n_a_slots &= ~1;
+    // shared memory: as many code stages as fit (up to 8) next to a B ring of at
+    // least 3 stages (up to 16), then whatever is left goes to the code ring
+    const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, p.b_stage_bytes);
+    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 24);
+    int nbs = 16, sc = 8;
+    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && nbs > 3) --nbs;
+    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && sc > 4) --sc;
+    while ((sc + 1) * GEMM_CODE_STAGE + nbs * p.b_stage_bytes <= room && sc < GEMM_SC_MAX) ++sc;
+    if (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room) return MOE_ERR_ARG;
+    p.n_b_stages = nbs;
+    p.n_c_stages = sc;
+    p.counts = c->counts;
+    p.offsets = c->offsets;
+    p.tiles = c->tiles;
+    p.row_token = c->row_token;
+    p.row_w = c->row_w;
+    p.rho = c->rho;
+    p.err = c->err;
+    p.wait_limit_ns = c->wait_limit_ns;
+    const GemmSmem plan = gemm_smem_plan(p.K, E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
+    if (plan.total > GEMM_SMEM_LIMIT) return MOE_ERR_ARG;
+    const long long P = (long long)T * top_k;
+    const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
+    long long max_work = (long long)p.MB * max_blocks;
+    int grid = c->num_sms;
+    if (max_work < grid) grid = (int)(max_work > 0 ? max_work : 1);
+    return cuda_status(launch_expert_gemm(mode, p, grid, plan.total, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_strerror(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0)";
+        case MOE_ERR_NOMEM: return "out of device memory";
+        default: return "unknown error";
+    }
+}
+
+const char *moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
+    if (!shape || !out) return MOE_ERR_ARG;
+    *out = nullptr;
+    const moe_shape_t s = *shape;
+    if (s.T_max < 1 || s.T_max > (1 << 20)) return MOE_ERR_ARG;
+    if (s.d_model < 64 || s.d_model > 6144 || s.d_model % 64) return MOE_ERR_ARG;
+    if (s.d_ff < 64 || s.d_ff > 6144 || s.d_ff % 64) return MOE_ERR_ARG;
+    if (s.n_experts < 1 || s.n_experts > 256) return MOE_ERR_ARG;
+    if (s.top_k < 1 || s.top_k > 8 || s.top_k > s.n_experts) return MOE_ERR_ARG;
+    if (!(s.eps >= 0.0f)) return MOE_ERR_ARG;
+    if ((long long)s.T_max * s.top_k > (1LL << 30) / 1) return MOE_ERR_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED;
+    if (!encode_fn()) return MOE_ERR_CUDA;
+
+    moe_ctx *c = new (std::nothrow) moe_ctx;
+    if (!c) return MOE_ERR_NOMEM;
+    memset(c, 0, sizeof *c);
+    c->shape = s;
+    c->device = dev;
+    c->num_sms = prop.multiProcessorCount;
+    c->wait_limit_ns = 2000000000ull;
+
+    const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
+    const size_t sizes[] = {T * s.d_model * 2, T * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
+                            P * 4, P * 4, P * s.d_ff * 2, T * s.d_model * 4, 64};
+    size_t total = 0;
+    for (size_t v : sizes) total += round256(v);
+    if (cudaMalloc(&c->ws, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete c;
+        return MOE_ERR_NOMEM;
+    }
+    c->ws_bytes = total;
+    char *b = static_cast<char *>(c->ws);
+    void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
+                      (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
+                      (void **)&c->row_w, (void **)&c->h, (void **)&c->y_acc, (void **)&c->err};
+    for (size_t i = 0; i < sizeof(sizes) / sizeof(sizes[0]); ++i) {
+        *slots[i] = b;
+        b += round256(sizes[i]);
+    }
+    if (cudaMemset(c->ws, 0, total) != cudaSuccess ||
+        !encode_f16_rows(&c->map_xn16, c->xn16, s.T_max, s.d_model, 1) ||
+        !encode_f16_rows(&c->map_h, c->h, (int)P, s.d_ff, 16)) {
+        cudaFree(c->ws);
+        delete c;
+        return MOE_ERR_CUDA;
+    }
+    *out = c;
+    return MOE_OK;
+}
+
+int moe_destroy(moe_ctx_t *ctx) {
+    if (!ctx) return MOE_OK;
+    cudaDeviceSynchronize();
+    cudaFree(ctx->ws);
+    delete ctx;
+    return MOE_OK;
+}
+
+int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale, const uint16_t *router_w,
+              const float *router_b, int top_k, void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned16(x) || !aligned16(norm_scale) || !aligned16(router_w) || !aligned16(router_b)) return MOE_ERR_ARG;
+    RouteParams p;
+    p.x = x;
+    p.norm_scale = norm_scale;
+    p.router_w = router_w;
+    p.router_b = router_b;
+    p.T = T;
+    p.d = c->shape.d_model;
+    p.E = c->shape.n_experts;
+    p.k = top_k;
+    p.eps = c->shape.eps;
+    p.xn16 = c->xn16;
+    p.rho = c->rho;
+    p.topk_idx = c->topk_idx;
+    p.topk_w = c->topk_w;
+    p.y_acc = c->y_acc;
+    return cuda_status(launch_route(p, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    GroupParams p;
+    p.topk_idx = c->topk_idx;
+    p.topk_w = c->topk_w;
+    p.P = T * top_k;
+    p.k = top_k;
+    p.E = c->shape.n_experts;
+    p.nb_rows = token_block_rows(T);
+    p.counts = c->counts;
+    p.offsets = c->offsets;
+    p.tiles = c->tiles;
+    p.row_token = c->row_token;
+    p.row_w = c->row_w;
+    p.err = c->err;
+    return cuda_status(launch_group(p, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
+                  const uint16_t *b13, void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned16(w13_codes) || !aligned16(w13_scales) || !aligned16(b13)) return MOE_ERR_ARG;
+    return gemm_launch(c, MODE_UP, T, top_k, w13_codes, w13_scales, b13, static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, const uint8_t *w2_scales,
+                    const uint16_t *b2, void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned16(w2_codes) || !aligned16(w2_scales) || !aligned16(b2)) return MOE_ERR_ARG;
+    return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, static_cast<cudaStream_t>(stream));
+}
+
+int moe_finalize(moe_ctx_t *c, int T, int top_k, uint16_t *y, int32_t *topk_idx_out, float *topk_w_out,
+                 void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned16(y)) return MOE_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rc = cuda_status(launch_finalize(c->y_acc, y, (long long)T * c->shape.d_model, s));
+    if (rc) return rc;
+    const size_t pk = (size_t)T * top_k;
+    if (topk_idx_out && cudaMemcpyAsync(topk_idx_out, c->topk_idx, pk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (topk_w_out && cudaMemcpyAsync(topk_w_out, c->topk_w, pk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w, const float *router_b,
+                const uint8_t *w13_codes, const uint8_t *w13_scales, const uint16_t *b13,
+                const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+                const uint16_t *norm_scale, int top_k, uint16_t *y, int32_t *topk_idx_out, float *topk_w_out,
+                void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(router_b) || !aligned16(w13_codes) ||
+        !aligned16(w13_scales) || !aligned16(b13) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
+        !aligned16(b2) || !aligned16(norm_scale) || !aligned16(y))
+        return MOE_ERR_ARG;
+    if (y == x) return MOE_ERR_ARG;
+    if ((rc = moe_route(c, T, x, norm_scale, router_w, router_b, top_k, stream))) return rc;
+    if ((rc = moe_group(c, T, top_k, stream))) return rc;
+    if ((rc = moe_expert_up(c, T, top_k, w13_codes, w13_scales, b13, stream))) return rc;
+    if ((rc = moe_expert_down(c, T, top_k, w2_codes, w2_scales, b2, stream))) return rc;
+    return moe_finalize(c, T, top_k, y, topk_idx_out, topk_w_out, stream);
+}
+
+int moe_copy_workspace(moe_ctx_t *c, int which, void *dst, size_t bytes, void *stream) {
+    if (!c || !dst) return MOE_ERR_ARG;
+    const Buf b = ws_buffer(c, which);
+    if (!b.ptr || bytes > b.bytes) return MOE_ERR_ARG;
+    if (bytes == 0) return MOE_OK;
+    return cuda_status(cudaMemcpyAsync(dst, b.ptr, bytes, cudaMemcpyDefault, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_sync_status(moe_ctx_t *c, void *stream) {
+    if (!c) return MOE_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int err = 0;
+    if (cudaMemcpyAsync(&err, c->err, sizeof err, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (err) {
+        if (cudaMemsetAsync(c->err, 0, sizeof err, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_ERR_TIMEOUT;
+    }
+    return MOE_OK;
+}
+
+int moe_set_wait_limit_ns(moe_ctx_t *c, unsigned long long ns) {
+    if (!c || ns == 0) return MOE_ERR_ARG;
+    c->wait_limit_ns = ns;
+    return MOE_OK;
+}
+
+int moe_selftest_wait_timeout(moe_ctx_t *c, void *stream) {
+    if (!c) return MOE_ERR_ARG;
+    return cuda_status(launch_selftest_wait(c->err, c->wait_limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, void *stream) {
+    if (!codes || !scales || !out || R < 0 || K < 32 || K % 32) return MOE_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(codes) & 3u) || (K / 2) % 4) return MOE_ERR_ARG;
+    return cuda_status(launch_decode(codes, scales, R, K, out, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,531 @@
+// Grouped MXFP4-weight GEMMs of the MoE experts on sm_100a (tcgen05 + TMEM + TMA).
+//
+// One persistent CTA per SM walks the work items (expert e, 128-row weight
+// block, block of up to 256 tokens routed to e).  For each item:
+//   A (weights, M = 128 rows): packed E2M1 codes arrive by TMA (128-byte
+//     swizzle) into a shared-memory ring; the E8M0 scales of the 128 rows by
+//     one untiled bulk copy.  Decoder warps convert 64 K-elements per row at a
+//     time to fp16 (hardware e2m1x2 conversion times the block's power of
+//     two, relative to a per-row power of two that keeps every block of the
+//     row exact in fp16) and store them straight into tensor memory, where
+//     the MMA reads A ("A from TMEM" form).  The decoded weights never touch
+//     shared memory, so shared-memory bandwidth is left to the codes and B.
+//   B (activations, N = tokens, K-major fp16): TMA into a shared-memory ring
+//     in the 128-byte swizzled canonical layout -- gathered row by row
+//     (tile::gather4) from the normalised tokens for the gate/up GEMM,
+//     contiguous expert-sorted rows of h for the down GEMM.
+//   D (fp32, 128 lanes x N columns) accumulates in TMEM; epilogue warps read
+//     it back with tcgen05.ld.
+// Gate/up epilogue: z = D * 2^c * rho_token + b13, clamped SwiGLU
+//   h = min(g,7) * sigmoid(1.702 min(g,7)) * (clamp(u,-7,7) + 1)
+//   ("gpt-oss-20B" hub page, section 3.3); each 128-row block holds 64 gate
+//   rows and their 64 linear rows so the pair meets in one warp.
+// Down epilogue: y_acc[token] += w_token * (D * 2^c + b2) by fp32 atomics
+//   (weighted combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
+//
+// Warp roles (512 threads): 0 codes/scales TMA, 1 MMA issue, 2 B TMA,
+// 3 TMEM allocation, 4-7 and 12-15 two decoder groups (alternate sub-stages),
+// 8-11 epilogue.  The decoders hand each row's power-of-two shift to the
+// epilogue through shared memory.  Every mbarrier wait is
+// bounded (WaitCtl); when one runs out the CTA stops issuing work, drains its
+// copies and MMAs in flight, frees TMEM and returns with the error latched.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+struct Work {
+    int e, mb, p0, n_valid, n_mma;
+};
+
+__device__ __forceinline__ void work_of(int w, const int *tiles_s, const int *counts_s, const int *offsets_s, int E,
+                                        int MB, int nb_rows, Work &t) {
+    // the last expert e with MB * tiles[e] <= w has at least one token block
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (MB * tiles_s[mid] <= w) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int local = w - MB * tiles_s[e];
+    const int nblk = tiles_s[e + 1] - tiles_s[e];
+    t.e = e;
+    t.mb = local / nblk;
+    const int nb = local - t.mb * nblk;
+    t.p0 = offsets_s[e] + nb * nb_rows;
+    t.n_valid = min(nb_rows, counts_s[e] - nb * nb_rows);
+    t.n_mma = (t.n_valid + 15) & ~15;
+}
+
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+    const uint64_t start = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - start > limit_ns) return;
+    }
+}
+
+// Wait for the `n_issued` most recent fills of a ring of `n_slots` full
+// barriers (fill i went to slot i % n_slots with phase parity (i / n_slots) & 1).
+__device__ __forceinline__ void drain_ring(uint64_t *full, int n_slots, long long n_issued,
+                                           unsigned long long limit_ns) {
+    for (long long i = n_issued - 1; i >= 0 && i >= n_issued - n_slots; --i)
+        mbar_wait_drain(&full[i % n_slots], (uint32_t)((i / n_slots) & 1), limit_ns);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Largest E8M0 byte (other than 255) of a row's n scale bytes (n even, row
+// 2-byte aligned), read as 16-bit words so the loads pipeline.
+__device__ __forceinline__ int row_scale_max(const uint8_t *s, int n) {
+    const uint16_t *w = reinterpret_cast<const uint16_t *>(s);
+    int m = -1;
+#pragma unroll 8
+    for (int b = 0; b < n / 2; ++b) {
+        const uint32_t v = w[b];
+        const int lo = (int)(v & 0xFFu), hi = (int)(v >> 8);
+        m = max(m, lo == 255 ? -1 : lo);
+        m = max(m, hi == 255 ? -1 : hi);
+    }
+    return m;
+}
+
+__device__ __forceinline__ float select4(const float (&v)[16], int base, int i) {
+    const float a = v[base], b = v[base + 1], c = v[base + 2], d = v[base + 3];
+    return i == 0 ? a : (i == 1 ? b : (i == 2 ? c : d));
+}
+
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const GemmSmem plan = gemm_smem_plan(p.K, p.E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
+    const int SC = p.n_c_stages, NA = p.n_a_slots;
+    uint8_t *code_ring = smem + plan.code_off;
+    uint8_t *b_ring = smem + plan.b_off;
+    uint8_t *scale_buf = smem + plan.scale_off;
+    const int scale_bytes = align_up(GEMM_BM * (p.K / 32), 128);
+    int *meta_tok = reinterpret_cast<int *>(smem + plan.meta_off);                    // [4][NB_MAX]
+    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off + 4 * GEMM_NB_MAX * 4);  // [4][NB_MAX]
+    int *shift_s = reinterpret_cast<int *>(smem + plan.shift_off);                   // [2][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bar_off);
+    uint64_t *c_full = bars;
+    uint64_t *c_empty = c_full + SC;
+    uint64_t *s_full = c_empty + SC;
+    uint64_t *s_empty = s_full + 2;
+    uint64_t *a_full = s_empty + 2;
+    uint64_t *a_empty = a_full + NA;
+    uint64_t *b_full = a_empty + NA;
+    uint64_t *b_empty = b_full + p.n_b_stages;
+    uint64_t *d_full = b_empty + p.n_b_stages;
+    uint64_t *d_empty = d_full + 2;
+    uint64_t *h_full = d_empty + 2;
+    uint64_t *h_empty = h_full + 2;
+    uint64_t *drain_bar = h_empty + 2;
+    uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
+    volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
+    int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
+    int *offsets_s = counts_s + (p.E + 1);
+    int *tiles_s = offsets_s + (p.E + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB32 = p.K / 32;
+    const int n_sub_total = p.K / GEMM_KA;
+    const int n_cstages = (p.K + GEMM_KS - 1) / GEMM_KS;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < SC; ++i) {
+            mbar_init(&c_full[i], 1);
+            mbar_init(&c_empty[i], 8);     // both decoder groups
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 8);
+            mbar_init(&d_full[i], 1);
+            mbar_init(&d_empty[i], 4);
+            mbar_init(&h_full[i], 4);
+            mbar_init(&h_empty[i], 4);
+        }
+        for (int i = 0; i < NA; ++i) {
+            mbar_init(&a_full[i], 4);      // the four warps of the group that decoded the slot
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < p.n_b_stages; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_s = 0;
+        fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+        counts_s[i] = i < p.E ? p.counts[i] : 0;
+        offsets_s[i] = p.offsets[i];
+        tiles_s[i] = p.tiles[i];
+    }
+    if (warp == 3) {
+        tmem_alloc(tmem_base_s, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    const int total = p.MB * tiles_s[p.E];
+    const WaitCtl wc{abort_s, p.err, MODE == MODE_UP ? (unsigned)ERR_WAIT_UP : (unsigned)ERR_WAIT_DOWN,
+                     p.wait_limit_ns};
+    const int d_stride = p.n_d_bufs == 2 ? p.nb_rows : 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------ codes + scales producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.map_codes);
+            int cslot = 0, sb = 0;
+            uint32_t cph = 0, sph = 0;
+            long long c_issued = 0, s_issued = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                Work t;
+                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+                if (!mbar_wait(&s_empty[sb], sph ^ 1, wc)) { ok = false; break; }
+                uint8_t *sdst = scale_buf + sb * scale_bytes;
+                if (MODE == MODE_UP) {
+                    const int j0 = t.mb * 64;
+                    const uint32_t bytes = 64u * KB32;
+                    mbar_arrive_expect_tx(&s_full[sb], 2 * bytes);
+                    bulk_load(sdst, p.scales + ((size_t)t.e * p.R + j0) * KB32, bytes, &s_full[sb]);
+                    bulk_load(sdst + bytes, p.scales + ((size_t)t.e * p.R + p.F + j0) * KB32, bytes, &s_full[sb]);
+                } else {
+                    const int m0 = t.mb * GEMM_BM;
+                    const uint32_t bytes = (uint32_t)min(GEMM_BM, p.R - m0) * KB32;
+                    mbar_arrive_expect_tx(&s_full[sb], bytes);
+                    bulk_load(sdst, p.scales + ((size_t)t.e * p.R + m0) * KB32, bytes, &s_full[sb]);
+                }
+                ++s_issued;
+                if (++sb == 2) { sb = 0; sph ^= 1; }
+                for (int ks = 0; ks < n_cstages; ++ks) {
+                    if (!mbar_wait(&c_empty[cslot], cph ^ 1, wc)) { ok = false; break; }
+                    uint8_t *cdst = code_ring + cslot * GEMM_CODE_STAGE;
+                    mbar_arrive_expect_tx(&c_full[cslot], GEMM_CODE_STAGE);
+                    if (MODE == MODE_UP) {
+                        tma_load_3d(cdst, &p.map_codes, &c_full[cslot], ks * 128, t.mb * 64, t.e);
+                        tma_load_3d(cdst + 64 * 128, &p.map_codes, &c_full[cslot], ks * 128, p.F + t.mb * 64, t.e);
+                    } else {
+                        tma_load_3d(cdst, &p.map_codes, &c_full[cslot], ks * 128, t.mb * GEMM_BM, t.e);
+                    }
+                    ++c_issued;
+                    if (++cslot == SC) { cslot = 0; cph ^= 1; }
+                }
+            }
+            if (!ok) {
+                drain_ring(c_full, SC, c_issued, p.wait_limit_ns);
+                drain_ring(s_full, 2, s_issued, p.wait_limit_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            int aslot = 0, bslot = 0, db = 0;
+            uint32_t aph = 0, bph = 0, dph = 0;
+            bool ok = true, issued = false;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                Work t;
+                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+                const uint32_t idesc = idesc_f16_f32(GEMM_BM, (uint32_t)t.n_mma);
+                if (!mbar_wait(&d_empty[db], dph ^ 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(NA * 32 + db * d_stride);
+                for (int s = 0; s < n_sub_total; ++s) {
+                    if (!mbar_wait(&a_full[aslot], aph, wc) || !mbar_wait(&b_full[bslot], bph, wc)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b_addr = smem_addr(b_ring + bslot * p.b_stage_bytes);
+                    const uint32_t a_tmem = tmem + (uint32_t)(aslot * 32);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
+                                   (s | kk) != 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(&a_empty[aslot]);
+                    mma_commit(&b_empty[bslot]);
+                    if (++aslot == NA) { aslot = 0; aph ^= 1; }
+                    if (++bslot == p.n_b_stages) { bslot = 0; bph ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&d_full[db]);
+                if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
+            }
+            if (!ok && issued) {
+                mma_commit(drain_bar);
+                mbar_wait_drain(drain_bar, 0, p.wait_limit_ns);
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------ B (tokens) producer
+        if (lane == 0) tma_prefetch_desc(&p.map_b);
+        int bslot = 0;
+        uint32_t bph = 0;
+        long long b_issued = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+            // gather rows this lane issues: groups g = lane and lane + 32 (4 rows each)
+            int tok[2][4];
+            if (MODE == MODE_UP) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int row = 4 * (lane + 32 * u) + r;
+                        tok[u][r] = row < t.n_mma ? p.row_token[t.p0 + (row < t.n_valid ? row : 0)] : 0;
+                    }
+            }
+            for (int s = 0; s < n_sub_total; ++s) {
+                const bool okw = __all_sync(0xffffffffu, mbar_wait(&b_empty[bslot], bph ^ 1, wc));
+                if (!okw) { ok = false; break; }
+                uint8_t *bdst = b_ring + bslot * p.b_stage_bytes;
+                if (lane == 0) mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)t.n_mma * 128u);
+                __syncwarp();
+                if (MODE == MODE_UP) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int g = lane + 32 * u;
+                        if (4 * g < t.n_mma)
+                            tma_gather4(bdst + g * 512, &p.map_b, &b_full[bslot], s * GEMM_KA, tok[u][0], tok[u][1],
+                                        tok[u][2], tok[u][3]);
+                    }
+                } else {
+                    const int g = lane;
+                    if (16 * g < t.n_mma) tma_load_2d(bdst + g * 2048, &p.map_b, &b_full[bslot], s * GEMM_KA, t.p0 + 16 * g);
+                }
+                ++b_issued;
+                if (++bslot == p.n_b_stages) { bslot = 0; bph ^= 1; }
+            }
+        }
+        if (!ok && lane == 0) drain_ring(b_full, p.n_b_stages, b_issued, p.wait_limit_ns);
+    } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+        // ------------------------------------------------------------ decoders
+        // Two groups of four warps.  Each code stage (4 sub-stages of 64 K
+        // elements) is cut into chunks of two sub-stages; group g decodes the
+        // chunks whose running index is congruent to g modulo 2, writing TMEM
+        // lanes 32q..32q+31 of the chunk's A slots, with one handshake per chunk.
+        const int q = warp & 3;
+        const int grp = warp >= 12 ? 1 : 0;
+        const int tl = 32 * q + lane;                           // TMEM lane = A row
+        const int my_row = MODE == MODE_UP ? (16 * q + (lane & 15) + (lane >= 16 ? 64 : 0)) : tl;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        int cslot = 0, sb = 0, hb = 0;
+        uint32_t cph = 0, sph = 0, hph = 0;
+        long long sub_idx = 0;                                  // running sub-stage index (A slot sequence)
+        long long chunk_idx = 0;                                // running chunk index
+        bool ok = true;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+            const bool row_valid = MODE == MODE_UP || (t.mb * GEMM_BM + my_row < p.R);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
+            const uint8_t *srow = scale_buf + sb * scale_bytes + my_row * KB32;
+            const int c = row_shift_from_max(row_valid ? row_scale_max(srow, KB32) : -1);
+            if (grp == 0) {
+                // hand the row shift to the epilogue
+                if (!__all_sync(0xffffffffu, mbar_wait(&h_empty[hb], hph ^ 1, wc))) { ok = false; break; }
+                shift_s[hb * GEMM_BM + tl] = c;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&h_full[hb]);
+                if (++hb == 2) { hb = 0; hph ^= 1; }
+            }
+            for (int ks = 0; ks < n_cstages && ok; ++ks) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&c_full[cslot], cph, wc))) { ok = false; break; }
+                const uint8_t *crow = code_ring + cslot * GEMM_CODE_STAGE + my_row * 128;
+                const int nsub = min(4, (p.K - ks * GEMM_KS) / GEMM_KA);
+                for (int a0 = 0; a0 < nsub; a0 += 2) {
+                    const int na = min(2, nsub - a0);
+                    const bool mine = (int)(chunk_idx & 1) == grp;
+                    const long long first = sub_idx;
+                    sub_idx += na;
+                    ++chunk_idx;
+                    if (!mine) continue;
+                    bool okc = true;
+                    for (int u = 0; u < na; ++u) {
+                        const long long si = first + u;
+                        okc = okc && mbar_wait(&a_empty[(int)(si % NA)], (uint32_t)(((si / NA) & 1) ^ 1), wc);
+                    }
+                    if (!__all_sync(0xffffffffu, okc)) { ok = false; break; }
+                    tc_fence_after();
+                    const int sw = my_row & 7;
+                    for (int u = 0; u < na; ++u) {
+                        const int a = a0 + u;
+                        uint32_t out[32];
+                        if (row_valid) {
+                            const uint4 w0 = *reinterpret_cast<const uint4 *>(crow + (((2 * a) ^ sw) << 4));
+                            const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + (((2 * a + 1) ^ sw) << 4));
+                            const int kb = (ks * GEMM_KS + a * GEMM_KA) / 32;
+                            const uint32_t m0 = block_multiplier(srow[kb], c);
+                            const uint32_t m1 = block_multiplier(srow[kb + 1], c);
+                            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                uint32_t h4[4];
+                                e2m1x8_to_half2x4(words[i], h4);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) out[4 * i + j] = hmul2_u32(h4[j], i < 4 ? m0 : m1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) out[i] = 0u;
+                        }
+                        tmem_st32(lane_base + (uint32_t)((int)((first + u) % NA) * 32), out);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int u = 0; u < na; ++u) mbar_arrive(&a_full[(int)((first + u) % NA)]);
+                }
+                if (!ok) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[cslot]);
+                if (++cslot == SC) { cslot = 0; cph ^= 1; }
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            if (++sb == 2) { sb = 0; sph ^= 1; }
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // ------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int tl = 32 * q + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        int *mtok = meta_tok + q * GEMM_NB_MAX;
+        float *mval = meta_val + q * GEMM_NB_MAX;
+        int db = 0, hb = 0;
+        uint32_t dph = 0, hph = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+            int row;
+            bool row_valid;
+            if (MODE == MODE_UP) {
+                row = (lane < 16 ? 0 : p.F) + t.mb * 64 + 16 * q + (lane & 15);
+                row_valid = true;
+            } else {
+                row = t.mb * GEMM_BM + tl;
+                row_valid = row < p.R;
+            }
+            const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + row]) : 0.f;
+            // per-column token and rho (UP) or routing weight (DOWN), one warp-private copy
+            for (int cc = lane; cc < t.n_mma; cc += 32) {
+                const int col = min(cc, t.n_valid - 1);
+                const int tok = p.row_token[t.p0 + col];
+                mtok[cc] = tok;
+                mval[cc] = MODE == MODE_UP ? p.rho[tok] : p.row_w[t.p0 + col];
+            }
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, mbar_wait(&h_full[hb], hph, wc))) break;
+            const float cscale = exp2i(shift_s[hb * GEMM_BM + tl]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&h_empty[hb]);
+            if (++hb == 2) { hb = 0; hph ^= 1; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
+            tc_fence_after();
+            const uint32_t d_tmem = lane_base + (uint32_t)(NA * 32 + db * d_stride);
+            for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(d_tmem + (uint32_t)c0, v);
+                tmem_wait_ld();
+                if (MODE == MODE_UP) {
+                    float z[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[i] = __uint_as_float(v[i]) * (cscale * mval[c0 + i]) + bias;
+                    __half *hout = reinterpret_cast<__half *>(p.out);
+                    const int jrow = t.mb * 64 + 16 * q + (lane & 15);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float send = lane < 16 ? z[8 + i] : z[i];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                        const float gate = lane < 16 ? z[i] : recv;
+                        const float lin = lane < 16 ? recv : z[8 + i];
+                        const int col = c0 + (lane < 16 ? i : 8 + i);
+                        const float g = fminf(gate, 7.0f);
+                        const float u = fminf(fmaxf(lin, -7.0f), 7.0f);
+                        const float h = g / (1.0f + __expf(-1.702f * g)) * (u + 1.0f);
+                        if (col < t.n_valid) hout[(size_t)(t.p0 + col) * p.out_ld + jrow] = __float2half_rn(h);
+                    }
+                } else {
+                    // weighted outputs of this lane's row, then a 4x4 transpose inside each
+                    // quad of lanes so every lane holds 4 consecutive rows of one column
+                    float val[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) val[i] = (__uint_as_float(v[i]) * cscale + bias) * mval[c0 + i];
+                    const int j = lane & 3;
+                    float *y = reinterpret_cast<float *>(p.out);
+                    const int row4 = t.mb * GEMM_BM + 32 * q + (lane & ~3);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        float o[4];
+                        o[0] = o[1] = o[2] = o[3] = 0.f;
+                        const float own = select4(val, 4 * m, j);
+#pragma unroll
+                        for (int r = 1; r < 4; ++r) {
+                            const float send = select4(val, 4 * m, j ^ r);
+                            const float recv = __shfl_xor_sync(0xffffffffu, send, r);
+                            const int dst = j ^ r;
+                            o[0] = dst == 0 ? recv : o[0];
+                            o[1] = dst == 1 ? recv : o[1];
+                            o[2] = dst == 2 ? recv : o[2];
+                            o[3] = dst == 3 ? recv : o[3];
+                        }
+                        if (j == 0) o[0] = own;
+                        if (j == 1) o[1] = own;
+                        if (j == 2) o[2] = own;
+                        if (j == 3) o[3] = own;
+                        const int col = c0 + 4 * m + j;
+                        if (col < t.n_valid && row4 < p.R)
+                            red_add_v4(y + (size_t)mtok[col] * p.out_ld + row4, o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 3) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template __global__ void expert_gemm_kernel<MODE_UP>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_DOWN>(const __grid_constant__ GemmParams p);
+
+}  // namespace moe
+
+namespace moe {
+
+cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s) {
+    if (mode == MODE_UP) {
+        cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        expert_gemm_kernel<MODE_UP><<<grid, GEMM_THREADS, smem, s>>>(p);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        expert_gemm_kernel<MODE_DOWN><<<grid, GEMM_THREADS, smem, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,503 @@
+// Routing side of the MoE block on sm_100a:
+//   route_kernel     RMSNorm + router logits + top-k + softmax over the chosen,
+//                    plus the fp16 normalised tokens for the experts and the
+//                    fp32 output accumulator initialised to the residual x;
+//   group_kernel     expert histogram, exclusive scan and a stable permutation
+//                    of the (token, expert) pairs into expert-contiguous rows;
+//   finalize_kernel  fp32 accumulator -> bf16 y.
+#include <cfloat>
+#include <climits>
+
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// ----------------------------------------------------------------- route
+//
+// One CTA per TB tokens, NW warps; NW / TB warps share each token.
+//   xn = x / sqrt(mean(x^2) + eps) * scale in fp32 ("gpt-oss-20B" hub page,
+//   section 3.2), kept in shared memory for the router; rho = a power of two
+//   with max|xn| / rho in [2^13, 2^14), and xn / rho stored as fp16 (an exact
+//   rescaling, so fp16's range never clips a token).
+// Router: logit_e = W_r[e] . xn + b_e in fp32 ("gpt-oss-20B" page, 3.4).
+//   Warp w owns experts w, w+NW, ... (at most EPW); the loop runs over
+//   VEC-element chunks of d, holding the TB tokens' chunk in registers while
+//   it is applied to every expert of the warp.
+// Top-k: k rounds of a warp arg-max on (logit desc, index asc) -- ties go to
+//   the lower expert index; a NaN logit ranks below every number, so the k
+//   chosen indices are always distinct and in range.  Softmax over the chosen
+//   (pnsm.cn overview, section 2.2).
+template <int VEC>
+__device__ __forceinline__ void load_bf16_vec(const uint16_t *p, float (&f)[VEC]) {
+    if (VEC == 8) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+}
+
+template <int TB, int NW, int EPW, int VEC>
+__global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
+    extern __shared__ float rsm[];
+    constexpr int WPT = NW / TB;            // warps per token
+    const int d = p.d, E = p.E;
+    float *xs = rsm;                        // [TB][d]
+    float *lg = rsm + TB * d;               // [TB][E]
+    float *red = lg + TB * E;               // [NW] partial sums / maxima
+    const int t0 = blockIdx.x * TB;
+    const int ntok = min(TB, p.T - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- RMSNorm
+    const int ti = warp / WPT;              // token of this warp
+    const int u = (warp % WPT) * 32 + lane; // thread index within the token's warps
+    const bool has_tok = ti < ntok;
+    const int t = t0 + ti;
+    float *xsr = xs + ti * d;
+    float ss = 0.f;
+    if (has_tok) {
+        const uint16_t *xr = p.x + (size_t)t * d;
+        float *ya = p.y_acc + (size_t)t * d;
+        for (int j = u * 8; j < d; j += WPT * 256) {
+            float f[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xr + j), f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                ss += f[c] * f[c];
+                xsr[j + c] = f[c];
+            }
+            reinterpret_cast<float4 *>(ya + j)[0] = make_float4(f[0], f[1], f[2], f[3]);
+            reinterpret_cast<float4 *>(ya + j)[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < WPT; ++i) tot += red[ti * WPT + i];
+    const float inv_rms = 1.0f / sqrtf(tot / (float)d + p.eps);
+    float amax = 0.f;
+    if (has_tok) {
+        for (int j = u * 8; j < d; j += WPT * 256) {
+            float sc[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p.norm_scale + j), sc);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float v = xsr[j + c] * inv_rms * sc[c];
+                xsr[j + c] = v;
+                amax = fmaxf(amax, fabsf(v));
+            }
+        }
+    }
+    amax = warp_max(amax);
+    __syncthreads();
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < WPT; ++i) amax = fmaxf(amax, red[ti * WPT + i]);
+    if (has_tok) {
+        float rho = 1.f, inv_rho = 1.f;
+        if (amax > 0.f && amax <= FLT_MAX) {
+            int ex;
+            frexpf(amax, &ex);          // amax in [2^(ex-1), 2^ex)
+            rho = exp2i(ex - 14);
+            inv_rho = exp2i(14 - ex);
+        }
+        if (u == 0) p.rho[t] = rho;
+        __half *xo = p.xn16 + (size_t)t * d;
+        for (int j = u * 8; j < d; j += WPT * 256) {
+            uint32_t hw[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const __half2 h2 = __floats2half2_rn(xsr[j + 2 * c] * inv_rho, xsr[j + 2 * c + 1] * inv_rho);
+                hw[c] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            *reinterpret_cast<uint4 *>(xo + j) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+    }
+    __syncthreads();
+
+    // ---- router logits
+    {
+        float acc[EPW][TB];
+#pragma unroll
+        for (int a = 0; a < EPW; ++a)
+#pragma unroll
+            for (int i = 0; i < TB; ++i) acc[a][i] = 0.f;
+        const int n_mine = (E - warp + NW - 1) / NW;   // experts of this warp
+#pragma unroll 2
+        for (int j = lane * VEC; j < d; j += 32 * VEC) {
+            float xv[TB][VEC];
+#pragma unroll
+            for (int i = 0; i < TB; ++i)
+#pragma unroll
+                for (int c = 0; c < VEC; c += 4) {
+                    const float4 a4 = (i < ntok) ? *reinterpret_cast<const float4 *>(xs + i * d + j + c)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                    xv[i][c] = a4.x;
+                    xv[i][c + 1] = a4.y;
+                    xv[i][c + 2] = a4.z;
+                    xv[i][c + 3] = a4.w;
+                }
+#pragma unroll
+            for (int a = 0; a < EPW; ++a) {
+                if (a < n_mine) {
+                    float wf[VEC];
+                    load_bf16_vec<VEC>(p.router_w + (size_t)(warp + a * NW) * d + j, wf);
+#pragma unroll
+                    for (int i = 0; i < TB; ++i)
+#pragma unroll
+                        for (int c = 0; c < VEC; ++c) acc[a][i] = fmaf(xv[i][c], wf[c], acc[a][i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < EPW; ++a) {
+            if (a < n_mine) {
+                const int e = warp + a * NW;
+                const float b = p.router_b[e];
+#pragma unroll
+                for (int i = 0; i < TB; ++i) {
+                    const float v = warp_sum(acc[a][i]);
+                    if (lane == 0 && i < ntok) lg[i * E + e] = v + b;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- top-k and softmax, one warp per token
+    for (int i = warp; i < ntok; i += NW) {
+        const int tt = t0 + i;
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane + 32 * c;
+            const float l = e < E ? lg[i * E + e] : -INFINITY;
+            v[c] = (l != l) ? -INFINITY : l;
+        }
+        unsigned taken = 0;
+        float sel_l[8];
+        int sel_e[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (r >= p.k) break;
+            float bv = -INFINITY;
+            int be = INT_MAX;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int e = lane + 32 * c;
+                if (e < E && !((taken >> c) & 1u) && (v[c] > bv || (v[c] == bv && e < be))) {
+                    bv = v[c];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            sel_l[r] = bv;
+            sel_e[r] = be;
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        }
+        if (lane == 0) {
+            const float m = sel_l[0];
+            float wsum = 0.f;
+            float wv[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                if (r < p.k) {
+                    wv[r] = expf(sel_l[r] - m);
+                    wsum += wv[r];
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                if (r < p.k) {
+                    p.topk_idx[(size_t)tt * p.k + r] = sel_e[r];
+                    p.topk_w[(size_t)tt * p.k + r] = wv[r] / wsum;
+                }
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------- group
+//
+// One CTA of 32 warps.  Warp w owns a contiguous segment of the T*k pairs
+// (pair i = token i/k, slot i%k).  Pass 1 counts, per warp and expert, with
+// __match_any_sync; a column scan turns the per-warp counts into each warp's
+// starting position inside every expert's range; pass 2 assigns positions in
+// pair order.  The result is sorted by expert and, within an expert, by token.
+__global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
+    __shared__ int wcnt[32][257];
+    __shared__ int off_s[257];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E, P = p.P;
+    for (int i = threadIdx.x; i < 32 * 257; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int seg = (P + 31) / 32;
+    const int beg = warp * seg, end = min(P, beg + seg);
+
+    // pass 1: per-warp counts; eight rows of 32 pairs are loaded before they are counted
+    for (int base = beg; base < end; base += 256) {
+        int ev[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = base + 32 * r + lane;
+            ev[r] = i < end ? p.topk_idx[i] : -1;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = base + 32 * r + lane;
+            int e = ev[r];
+            if (i < end && (e < 0 || e >= E)) {
+                atomicOr(p.err, ERR_ROUTING);
+                e = -1;
+            }
+            const unsigned m = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp][e] += __popc(m);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+
+    if ((int)threadIdx.x < E) {
+        const int e = threadIdx.x;
+        int s = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = s;
+            s += c;
+        }
+        p.counts[e] = s;
+        off_s[e] = s;   // total for now
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // exclusive scans of counts and of token blocks; lane owns 8 experts
+        int cnt[8], blk[8];
+        int cs = 0, bs = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane * 8 + c;
+            cnt[c] = e < E ? off_s[e] : 0;
+            blk[c] = (cnt[c] + p.nb_rows - 1) / p.nb_rows;
+            cs += cnt[c];
+            bs += blk[c];
+        }
+        int ci = cs, bi = bs;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, ci, o);
+            const int b = __shfl_up_sync(0xffffffffu, bi, o);
+            if (lane >= o) {
+                ci += a;
+                bi += b;
+            }
+        }
+        int co = ci - cs, bo = bi - bs;   // exclusive
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane * 8 + c;
+            if (e < E) {
+                off_s[e] = co;
+                p.offsets[e] = co;
+                p.tiles[e] = bo;
+            }
+            co += cnt[c];
+            bo += blk[c];
+        }
+        if (lane == 31) {
+            p.offsets[E] = ci;
+            p.tiles[E] = bi;
+        }
+    }
+    __syncthreads();
+
+    // pass 2: positions, in pair order within each warp's segment
+    for (int base = beg; base < end; base += 256) {
+        int ev[8];
+        float wv[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = base + 32 * r + lane;
+            ev[r] = i < end ? p.topk_idx[i] : -1;
+            wv[r] = i < end ? p.topk_w[i] : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int i = base + 32 * r + lane;
+            int e = ev[r];
+            if (e >= E) e = -1;
+            const unsigned m = __match_any_sync(0xffffffffu, e);
+            if (e >= 0) {
+                const int pos = off_s[e] + wcnt[warp][e] + __popc(m & ((1u << lane) - 1u));
+                p.row_token[pos] = i / p.k;
+                p.row_w[pos] = wv[r];
+            }
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp][e] += __popc(m);
+            __syncwarp();
+        }
+    }
+}
+
+// -------------------------------------------------------------- finalize
+
+__global__ void __launch_bounds__(256) finalize_kernel(const float *__restrict__ y_acc, uint16_t *__restrict__ y,
+                                                       long long n8) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4 *>(y_acc)[2 * i];
+        const float4 b = reinterpret_cast<const float4 *>(y_acc)[2 * i + 1];
+        const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+        uint4 o;
+        o.x = *reinterpret_cast<const uint32_t *>(&p0);
+        o.y = *reinterpret_cast<const uint32_t *>(&p1);
+        o.z = *reinterpret_cast<const uint32_t *>(&p2);
+        o.w = *reinterpret_cast<const uint32_t *>(&p3);
+        reinterpret_cast<uint4 *>(y)[i] = o;
+    }
+}
+
+// ------------------------------------------------------------ debug decode
+//
+// The grouped GEMMs' weight decode on its own: one thread per (row, 32-element
+// block); fp16 e2m1 conversion times the block multiplier under the row shift,
+// then times 2^c back in fp32.
+__global__ void decode_kernel(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out) {
+    const int nb = K / 32;
+    const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (idx >= (long long)R * nb) return;
+    const int r = (int)(idx / nb), b = (int)(idx % nb);
+    const uint8_t *srow = scales + (size_t)r * nb;
+    int smax = -1;
+    for (int i = 0; i < nb; ++i)
+        if (srow[i] != 255 && srow[i] > smax) smax = srow[i];
+    const int c = row_shift_from_max(smax);
+    const uint32_t mult = block_multiplier(srow[b], c);
+    const float back = exp2i(c);
+    const uint32_t *cw = reinterpret_cast<const uint32_t *>(codes + (size_t)r * (K / 2) + b * 16);
+    float *o = out + (size_t)r * K + b * 32;
+    for (int wi = 0; wi < 4; ++wi) {
+        uint32_t h4[4];
+        e2m1x8_to_half2x4(cw[wi], h4);
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t v = hmul2_u32(h4[j], mult);
+            const __half2 hv = *reinterpret_cast<const __half2 *>(&v);
+            const float2 f = __half22float2(hv);
+            o[wi * 8 + 2 * j] = f.x * back;
+            o[wi * 8 + 2 * j + 1] = f.y * back;
+        }
+    }
+}
+
+// ----------------------------------------------------------- wait self-test
+
+__global__ void selftest_wait_kernel(unsigned int *err, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const WaitCtl wc{&abort_flag, err, ERR_WAIT_SELFTEST, limit_ns};
+    // nothing ever arrives on `bar`: the wait must run out and report it
+    (void)mbar_wait(&bar, 0, wc);
+}
+
+// --------------------------------------------------------------- launchers
+
+template <int TB, int NW, int EPW, int VEC>
+static cudaError_t launch_route_cfg(const RouteParams &p, cudaStream_t s) {
+    const size_t smem = ((size_t)TB * (p.d + p.E) + NW) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<TB, NW, EPW, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<TB, NW, EPW, VEC><<<(p.T + TB - 1) / TB, NW * 32, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
+    if (p.T <= 0) return cudaSuccess;
+    // few tokens: one token per CTA, 32 warps (latency); many tokens: the
+    // router weights are reused across 8 (or 4) tokens of a CTA (throughput)
+    if (p.T <= 512 || (size_t)8 * (p.d + p.E) * 4 > 200 * 1024) return launch_route_cfg<1, 32, 8, 8>(p, s);
+    if (p.E <= 128) return launch_route_cfg<8, 16, 8, 4>(p, s);
+    return launch_route_cfg<4, 32, 8, 4>(p, s);
+}
+
+cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
+    group_kernel<<<1, 1024, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float *y_acc, uint16_t *y, long long n, cudaStream_t s) {
+    const long long n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int grid = (int)min((n8 + 255) / 256, (long long)148 * 8);
+    finalize_kernel<<<grid, 256, 0, s>>>(y_acc, y, n8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s) {
+    const long long n = (long long)R * (K / 32);
+    if (n == 0) return cudaSuccess;
+    decode_kernel<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(codes, scales, R, K, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(unsigned int *err, unsigned long long limit_ns, cudaStream_t s) {
+    selftest_wait_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,319 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Every test here needs a B200 and the built library; inputs are the seeded
+synthetic workloads of ``moe_inputs``.
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+import sparse_moe_rmsnorm_b200 as moe
+from moe_inputs import CONFIGS, bf16_bits_to_f32, custom_layer, make_config_inputs
+from _parity import compare_block, excluded_tokens
+
+pytestmark = pytest.mark.gpu
+
+# Tighter bound on the fp32 accumulator y_acc (before the bf16 output cast): the fp16 rounding of
+# xn/rho and of h gives ~2e-4 mean relative error in a float64 emulation of the same rounding points.
+ACC_MEAN_REL = 1e-3
+
+
+def _bf16_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _y_numpy(y):
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def run_block(inp, k, eps=1e-5, T_max=None):
+    x = _bf16_dev(inp["x"])
+    T, d = x.shape
+    E = inp["router_w"].shape[0]
+    F = inp["w13_codes"].shape[1] // 2
+    w = moe.MoEWeights.from_numpy(inp)
+    m = moe.MoE(T_max or max(T, 1), d, F, E, k, eps)
+    y, idx, wts = m.forward(x, w, routing=True)
+    torch.cuda.synchronize()
+    assert m.sync_status() == moe.MOE_OK
+    yacc = m.workspace("y_acc", T).cpu().numpy().astype(np.float64)
+    out = dict(y=_y_numpy(y), yacc=yacc, idx=idx.cpu().numpy(), w=wts.cpu().numpy().astype(np.float64), ctx=m,
+               weights=w, x=x)
+    return out
+
+
+def check(inp, k, eps=1e-5, rows=None, label=""):
+    g = run_block(inp, k, eps)
+    if rows is None:
+        ref = oracle.moe_forward(inp, k, eps)
+        res = compare_block(g["y"], g["idx"], g["w"], ref, k, inp["router_w"].shape[0])
+    else:
+        ref = oracle.moe_forward(inp, k, eps, x=inp["x"][rows])
+        res = compare_block(g["y"][rows], g["idx"][rows], g["w"][rows], ref, k, inp["router_w"].shape[0])
+    # the fp32 accumulator before the bf16 cast: fp16 activations leave ~2e-4 of mean relative error
+    if rows is None:
+        acc = compare_block(g["yacc"], g["idx"], g["w"], ref, k, inp["router_w"].shape[0])
+    else:
+        acc = compare_block(g["yacc"][rows], g["idx"][rows], g["w"][rows], ref, k, inp["router_w"].shape[0])
+    print(label, res, "| fp32 accumulator:", {k_: acc[k_] for k_ in ("max_rel", "mean_rel")})
+    assert res["ok"], res
+    assert res["w_max_err"] < 1e-5, res
+    assert acc["mean_rel"] <= ACC_MEAN_REL, acc
+    g["ctx"].close()
+    return res
+
+
+# ----------------------------------------------------------------- decode
+
+def test_decode_uniform_rows_all_scales_exact():
+    """Every code under every E8M0 byte: the device decode equals the oracle's value in fp32."""
+    K = 64
+    R = 256
+    codes = np.zeros((R, K // 2), dtype=np.uint8)
+    # all 16 codes in every row: bytes 0..7 hold codes (2m, 2m+1)
+    codes[:, :8] = (np.arange(0, 16, 2, dtype=np.uint8) | (np.arange(1, 16, 2, dtype=np.uint8) << 4))[None, :]
+    codes[:, 8:] = np.random.default_rng(0).integers(0, 256, size=(R, K // 2 - 8), dtype=np.uint8)
+    scales = np.repeat(np.arange(256, dtype=np.uint8)[:, None], K // 32, axis=1)
+    want = oracle.decode_matrix(codes, scales).astype(np.float32)
+    out = torch.empty((R, K), dtype=torch.float32, device="cuda")
+    moe.moe_debug_decode(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), R, K, out)
+    got = out.cpu().numpy()
+    nan_w = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan_w)
+    assert np.array_equal(got[~nan_w], want[~nan_w])
+    assert np.array_equal(np.signbit(got[~nan_w]), np.signbit(want[~nan_w]))
+
+
+def test_decode_mixed_scales_within_36_exact():
+    rng = np.random.default_rng(1)
+    R, K = 300, 2880
+    codes = rng.integers(0, 256, size=(R, K // 2), dtype=np.uint8)
+    lo = rng.integers(60, 180, size=(R, 1))
+    scales = (lo + rng.integers(0, 37, size=(R, K // 32))).astype(np.uint8)
+    want = oracle.decode_matrix(codes, scales).astype(np.float32)
+    out = torch.empty((R, K), dtype=torch.float32, device="cuda")
+    moe.moe_debug_decode(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), R, K, out)
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
+def test_decode_wide_scale_spread_bounded():
+    """Blocks more than 36 binades under their row's largest may round or flush to zero in fp16; the
+    absolute error of any element stays below 6 * 2^(smax - 165), smax the row's largest E8M0 byte."""
+    rng = np.random.default_rng(2)
+    R, K = 64, 640
+    codes = rng.integers(0, 256, size=(R, K // 2), dtype=np.uint8)
+    scales = rng.integers(60, 200, size=(R, K // 32)).astype(np.uint8)
+    want = oracle.decode_matrix(codes, scales)
+    out = torch.empty((R, K), dtype=torch.float32, device="cuda")
+    moe.moe_debug_decode(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), R, K, out)
+    got = out.cpu().numpy().astype(np.float64)
+    smax = scales.max(axis=1, keepdims=True).astype(np.float64)
+    assert np.all(np.abs(got - want) <= 6.0 * 2.0 ** (smax - 165))
+    narrow = scales >= scales.max(axis=1, keepdims=True) - 36
+    assert np.array_equal(got[np.repeat(narrow, 32, axis=1)], want.astype(np.float32)[np.repeat(narrow, 32, axis=1)])
+
+
+# ------------------------------------------------------------ route, group
+
+@pytest.mark.parametrize("T,d,E,k", [(16, 128, 8, 4), (37, 2880, 32, 4), (600, 2880, 128, 4), (2100, 256, 64, 8)])
+def test_route_stage(T, d, E, k):
+    inp = custom_layer(T=T, d=d, F=64, E=E, k=k, seed=T)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(T, d, 64, E, k)
+    moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
+    idx = m.workspace("topk_idx", T).cpu().numpy()
+    wts = m.workspace("topk_w", T).cpu().numpy()
+    xn16 = m.workspace("xn16", T).float().cpu().numpy().astype(np.float64)
+    rho = m.workspace("rho", T).cpu().numpy().astype(np.float64)
+    yacc = m.workspace("y_acc", T).cpu().numpy()
+    xn = oracle.rmsnorm(inp["x"], inp["norm_scale"], 1e-5)
+    logits = oracle.router(xn, inp["router_w"], inp["router_b"])
+    ref_idx, ref_w = oracle.topk_softmax(logits, k)
+    keep = ~excluded_tokens(logits, k)
+    assert np.array_equal(idx[keep], ref_idx[keep])
+    assert np.max(np.abs(wts[keep] - ref_w[keep])) < 1e-5
+    # rho is a power of two with max|xn|/rho in [2^13, 2^14)
+    m2, e2 = np.frexp(rho)
+    assert np.all(m2 == 0.5)
+    amax = np.abs(xn16).max(axis=1)
+    assert np.all((amax >= 2.0 ** 13 * (1 - 2 ** -10)) & (amax <= 2.0 ** 14))
+    assert np.max(np.abs(xn16 * rho[:, None] - xn) / np.abs(xn).max(axis=1, keepdims=True)) < 6e-4
+    assert np.array_equal(yacc, bf16_bits_to_f32(inp["x"]))
+    m.close()
+
+
+@pytest.mark.parametrize("T,E,k", [(16, 8, 4), (8192, 32, 4), (64, 128, 4), (3000, 256, 8), (5, 3, 3)])
+def test_group_stage_invariants(T, E, k):
+    inp = custom_layer(T=T, d=64, F=64, E=E, k=k, seed=3 * T + E)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(T, 64, 64, E, k)
+    moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
+    moe.moe_group(m.ctx, T, k)
+    idx = m.workspace("topk_idx", T).cpu().numpy()
+    wts = m.workspace("topk_w", T).cpu().numpy()
+    counts = m.workspace("counts", T).cpu().numpy()
+    offsets = m.workspace("offsets", T).cpu().numpy()
+    tiles = m.workspace("tiles", T).cpu().numpy()
+    row_token = m.workspace("row_token", T).cpu().numpy()
+    row_w = m.workspace("row_w", T).cpu().numpy()
+    assert m.sync_status() == moe.MOE_OK
+    P = T * k
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts) and offsets[-1] == P
+    nb = min(256, (T + 15) // 16 * 16)
+    assert np.array_equal(np.diff(tiles), (counts + nb - 1) // nb)
+    # a stable permutation: expert-major, token-minor, every pair exactly once
+    want_tok = []
+    want_w = []
+    for e in range(E):
+        t_e, s_e = np.nonzero(idx == e)
+        want_tok.extend(t_e.tolist())
+        want_w.extend(wts[t_e, s_e].tolist())
+    assert np.array_equal(row_token, np.array(want_tok, dtype=np.int32))
+    assert np.array_equal(row_w, np.array(want_w, dtype=np.float32))
+    m.close()
+
+
+# ----------------------------------------------------------- whole block
+
+def test_tiny_config():
+    cfg = CONFIGS["tiny"]
+    check(make_config_inputs(cfg), cfg.k, label="tiny")
+
+
+SHAPES = [
+    dict(T=1, d=128, F=128, E=8, k=4),
+    dict(T=17, d=192, F=320, E=5, k=2),
+    dict(T=33, d=256, F=128, E=4, k=4),          # k == E
+    dict(T=9, d=64, F=64, E=1, k=1),             # a single expert: dense FFN
+    dict(T=40, d=512, F=256, E=16, k=8),         # largest k
+    dict(T=300, d=128, F=192, E=2, k=1),         # n_e > 256: several token blocks per expert
+    dict(T=700, d=320, F=640, E=8, k=4),         # token blocks of 256, ragged tails
+    dict(T=50, d=2880, F=2880, E=32, k=4),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "T%d_d%d_F%d_E%d_k%d" % tuple(s.values()))
+def test_shapes(shape):
+    shape = dict(shape)
+    k = shape.pop("k")
+    check(custom_layer(**shape, k=k, seed=sum(shape.values())), k, label=str(shape))
+
+
+def test_scale_extremes():
+    """E8M0 exponents far from 127 (exercises the per-row fp16 shift of the decode).
+
+    Exponents 100..136 on every weight; then huge W2 (140..150) behind normal W13, and tiny W13
+    (104..110).  Huge W13 is left out on purpose: it scales the gate pre-activations to ~1e7, where
+    the clamped SwiGLU is a step function of them and any rounding of the activations (fp16 here,
+    bf16 just as well) moves outputs across the step -- an exact-weight emulation in float64 with
+    fp16 activations shows the same ~4% deviation there."""
+    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=5, scale_lo=100, scale_hi=136)
+    check(inp, 2, label="scales 100..136")
+    rng = np.random.default_rng(7)
+    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=6)
+    inp["w2_scales"] = rng.integers(140, 151, size=inp["w2_scales"].shape, dtype=np.uint8)
+    check(inp, 2, label="W2 scales 140..150")
+    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=8)
+    inp["w13_scales"] = rng.integers(104, 111, size=inp["w13_scales"].shape, dtype=np.uint8)
+    check(inp, 2, label="W13 scales 104..110")
+
+
+def test_tied_logits_pick_lower_index():
+    inp = custom_layer(T=20, d=128, F=128, E=8, k=4, seed=9)
+    inp["router_w"][:] = 0
+    inp["router_b"][:] = 0.5
+    g = run_block(inp, 4)
+    assert np.all(g["idx"] == np.arange(4)[None, :])
+    assert np.allclose(g["w"], 0.25)
+    ref = oracle.moe_forward(inp, 4, 1e-5)
+    assert np.array_equal(ref["idx"], g["idx"])
+    d = np.abs(g["y"] - ref["y"])
+    assert d.max() <= 2e-2 * np.abs(ref["y"]).max() and d.sum() <= 5e-3 * np.abs(ref["y"]).sum()
+    g["ctx"].close()
+
+
+def test_decode20b_full():
+    cfg = CONFIGS["decode20b"]
+    check(make_config_inputs(cfg), cfg.k, label="decode20b")
+
+
+def test_decode120b_full():
+    cfg = CONFIGS["decode120b"]
+    check(make_config_inputs(cfg), cfg.k, label="decode120b")
+
+
+def test_repeat_calls_and_smaller_T():
+    """The same context serves several calls and token counts below T_max."""
+    inp = custom_layer(T=64, d=256, F=256, E=8, k=4, seed=21)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(64, 256, 256, 8, 4)
+    ref = oracle.moe_forward(inp, 4, 1e-5)
+    for T in (64, 5, 64, 1):
+        y, idx, wts = m.forward(x[:T], w, routing=True)
+        r = {k_: v[:T] for k_, v in ref.items()}
+        res = compare_block(_y_numpy(y), idx.cpu().numpy(), wts.cpu().numpy(), r, 4, 8)
+        assert res["ok"], (T, res)
+    assert m.sync_status() == moe.MOE_OK
+    m.close()
+
+
+def test_empty_batch_is_a_no_op():
+    inp = custom_layer(T=4, d=128, F=128, E=8, k=4, seed=1)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(4, 128, 128, 8, 4)
+    y = torch.full_like(x, 3.0)
+    moe.moe_forward(m.ctx, 0, x, w.router_w, w.router_b, w.w13_codes, w.w13_scales, w.b13, w.w2_codes,
+                    w.w2_scales, w.b2, w.norm_scale, 4, y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 3.0)
+    m.close()
+
+
+def test_argument_errors():
+    m = moe.MoE(8, 128, 128, 8, 4)
+    inp = custom_layer(T=8, d=128, F=128, E=8, k=4, seed=1)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    y = torch.empty_like(x)
+    args = [x, w.router_w, w.router_b, w.w13_codes, w.w13_scales, w.b13, w.w2_codes, w.w2_scales, w.b2,
+            w.norm_scale]
+    with pytest.raises(moe.MoEError) as e:
+        moe.moe_forward(m.ctx, 9, *args, 4, y)            # T > T_max
+    assert e.value.code == moe.MOE_ERR_ARG
+    with pytest.raises(moe.MoEError):
+        moe.moe_forward(m.ctx, 8, *args, 5, y)            # top_k > shape top_k
+    with pytest.raises(moe.MoEError):
+        moe.moe_forward(m.ctx, 8, *args, 0, y)
+    bad = list(args)
+    bad[3] = w.w13_codes.view(-1)[1:]                      # misaligned pointer
+    with pytest.raises(moe.MoEError):
+        moe.moe_forward(m.ctx, 8, *bad, 4, y)
+    with pytest.raises(moe.MoEError):
+        moe.moe_forward(m.ctx, 8, *args, 4, x)            # y aliases x
+    assert m.sync_status() == moe.MOE_OK
+    m.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    inp = custom_layer(T=16, d=128, F=128, E=8, k=4, seed=2)
+    m = moe.MoE(16, 128, 128, 8, 4)
+    moe.moe_set_wait_limit_ns(m.ctx, 20_000_000)           # 20 ms
+    moe.moe_selftest_wait_timeout(m.ctx)
+    assert m.sync_status() == moe.MOE_ERR_TIMEOUT
+    assert m.sync_status() == moe.MOE_OK                   # cleared once read
+    moe.moe_set_wait_limit_ns(m.ctx, 2_000_000_000)
+    w = moe.MoEWeights.from_numpy(inp)
+    y, idx, wts = m.forward(_bf16_dev(inp["x"]), w, routing=True)
+    ref = oracle.moe_forward(inp, 4, 1e-5)
+    res = compare_block(_y_numpy(y), idx.cpu().numpy(), wts.cpu().numpy(), ref, 4, 8)
+    assert res["ok"], res
+    m.close()
