@@ -188,7 +188,7 @@ def algorithmic_counts(cfg, counts):
     w2_expert = d * (F // 2) + d * (F // 32) + d * 2
     pairs = T * k
     bytes_up = touched * w13_expert + T * d * 2 + pairs * F * 2          # weights, xn16 in, h out
-    bytes_down = touched * w2_expert + pairs * F * 2 + pairs * d * 4      # weights, h in, y_acc updates
+    bytes_down = touched * w2_expert + pairs * F * 2 + pairs * d * 4      # weights, h in, weighted rows out
     flops_up = pairs * 2 * (2 * F) * d
     flops_down = pairs * 2 * d * F
     layer_bytes = touched * (w13_expert + w2_expert) + E * d * 2 + E * 4 + d * 2 + T * d * 2 * 2
@@ -276,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
         evs[3].record(stream)
         moe.moe_expert_down(m.ctx, T, cfg.k, w0.w2_codes, w0.w2_scales, w0.b2)
         evs[4].record(stream)
-        moe.moe_finalize(m.ctx, T, cfg.k, y0)
+        moe.moe_finalize(m.ctx, T, cfg.k, x, y0)
         evs[5].record(stream)
         torch.cuda.synchronize()
         for i, k_ in enumerate(stage_ms):
@@ -370,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.d * 2,
                     "d2h_bytes_per_step": T * cfg.d * 2},
-            "gpu_launches": 5 * layers * args.steps, "clocks": clocks.summary()}
+            "gpu_launches": 6 * layers * args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     m.close()
     return 0

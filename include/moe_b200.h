@@ -110,9 +110,18 @@ MOE_API int moe_forward(moe_ctx_t *ctx, int T,
                 void *stream);
 
 /* The five stages of moe_forward, callable one by one on the same context
- * and stream, in this order (moe_forward is exactly these five calls).  They
- * exist for per-stage timing and tests; intermediate results stay in the
- * context's workspace (see moe_copy_workspace). */
+ * and stream, in this order (moe_forward is exactly these five calls):
+ *   moe_route        RMSNorm, router logits, top-k and softmax;
+ *   moe_group        expert histogram, prefix sum and the stable permutation
+ *                    of (token, expert) pairs into expert-contiguous rows,
+ *                    then the expert-sorted copy of the normalised tokens;
+ *   moe_expert_up    gate/up grouped GEMM with the clamped-SwiGLU epilogue;
+ *   moe_expert_down  down grouped GEMM, each row scaled by its routing weight;
+ *   moe_finalize     y = x + the token's weighted expert rows (bf16), in a
+ *                    fixed order, so results are reproducible run to run.
+ * They exist for per-stage timing and tests; intermediate results stay in the
+ * context's workspace (see moe_copy_workspace).  moe_finalize needs the same
+ * x that moe_route was given. */
 MOE_API int moe_route(moe_ctx_t *ctx, int T, const uint16_t *x, const uint16_t *norm_scale,
               const uint16_t *router_w, const float *router_b, int top_k, void *stream);
 MOE_API int moe_group(moe_ctx_t *ctx, int T, int top_k, void *stream);
@@ -120,8 +129,8 @@ MOE_API int moe_expert_up(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w13_c
                   const uint16_t *b13, void *stream);
 MOE_API int moe_expert_down(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w2_codes, const uint8_t *w2_scales,
                     const uint16_t *b2, void *stream);
-MOE_API int moe_finalize(moe_ctx_t *ctx, int T, int top_k, uint16_t *y, int32_t *topk_idx_out, float *topk_w_out,
-                 void *stream);
+MOE_API int moe_finalize(moe_ctx_t *ctx, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,
+                 float *topk_w_out, void *stream);
 
 /* Workspace buffers readable through moe_copy_workspace. */
 enum {
@@ -134,8 +143,10 @@ enum {
     MOE_WS_ROW_TOKEN = 6,/* int32 [T*k]   token of each expert-sorted row         */
     MOE_WS_ROW_W = 7,    /* fp32 [T*k]    routing weight of each expert-sorted row */
     MOE_WS_H = 8,        /* fp16 [T*k, F] SwiGLU output, expert-sorted rows       */
-    MOE_WS_YACC = 9,     /* fp32 [T, d]   x + weighted expert outputs             */
-    MOE_WS_TILES = 10    /* int32 [E+1]   exclusive prefix of token blocks        */
+    MOE_WS_OUT_ROWS = 9, /* fp32 [T*k, d] w * (W2 h + b2), expert-sorted rows      */
+    MOE_WS_TILES = 10,   /* int32 [E+1]   exclusive prefix of token blocks        */
+    MOE_WS_PAIR_ROW = 11,/* int32 [T*k]   expert-sorted row of pair (token, slot) */
+    MOE_WS_XPERM = 12    /* fp16 [T*k, d] xn16 rows in expert-sorted order         */
 };
 
 /* Copy `bytes` bytes of workspace buffer `which` (a MOE_WS_* value) into

@@ -28,7 +28,8 @@ __all__ = [
 MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_NOMEM = 0, -1, -2, -3, -4, -5
 
 # workspace buffer ids of moe_copy_workspace
-WS = dict(xn16=0, rho=1, topk_idx=2, topk_w=3, counts=4, offsets=5, row_token=6, row_w=7, h=8, y_acc=9, tiles=10)
+WS = dict(xn16=0, rho=1, topk_idx=2, topk_w=3, counts=4, offsets=5, row_token=6, row_w=7, h=8, out_rows=9, tiles=10,
+          pair_row=11, xperm=12)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
@@ -59,7 +60,7 @@ _SIGS = {
     "moe_group": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "moe_expert_up": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
     "moe_expert_down": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
-    "moe_finalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
+    "moe_finalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5),
     "moe_copy_workspace": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                                           ctypes.c_void_p]),
     "moe_sync_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
@@ -158,8 +159,8 @@ def moe_expert_down(ctx, T, top_k, w2_codes, w2_scales, b2, stream=None) -> None
                                  _stream(stream)), "moe_expert_down")
 
 
-def moe_finalize(ctx, T, top_k, y, topk_idx_out=None, topk_w_out=None, stream=None) -> None:
-    _check(lib().moe_finalize(ctx, int(T), int(top_k), _ptr(y), _ptr(topk_idx_out), _ptr(topk_w_out),
+def moe_finalize(ctx, T, top_k, x, y, topk_idx_out=None, topk_w_out=None, stream=None) -> None:
+    _check(lib().moe_finalize(ctx, int(T), int(top_k), _ptr(x), _ptr(y), _ptr(topk_idx_out), _ptr(topk_w_out),
                               _stream(stream)), "moe_finalize")
 
 
@@ -296,8 +297,9 @@ class MoE:
             "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
             "counts": ((s.n_experts,), torch.int32), "offsets": ((s.n_experts + 1,), torch.int32),
             "row_token": ((P,), torch.int32), "row_w": ((P,), torch.float32),
-            "h": ((P, s.d_ff), torch.float16), "y_acc": ((T, s.d_model), torch.float32),
-            "tiles": ((s.n_experts + 1,), torch.int32),
+            "h": ((P, s.d_ff), torch.float16), "out_rows": ((P, s.d_model), torch.float32),
+            "tiles": ((s.n_experts + 1,), torch.int32), "pair_row": ((P,), torch.int32),
+            "xperm": ((P, s.d_model), torch.float16),
         }[name]
         out = torch.empty(spec[0], dtype=spec[1], device="cuda")
         moe_copy_workspace(self.ctx, WS[name], out, out.numel() * out.element_size(), stream)

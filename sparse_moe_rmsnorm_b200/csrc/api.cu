@@ -15,7 +15,9 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_finalize(const float *y_acc, uint16_t *y, long long n, cudaStream_t s);
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
+                           cudaStream_t s);
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
 cudaError_t launch_selftest_wait(unsigned int *err, unsigned long long limit_ns, cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
@@ -86,12 +88,14 @@ struct moe_ctx {
     int *counts, *offsets, *tiles;
     int *row_token;
     float *row_w;
+    int *pair_row;
+    __half *xperm;          // expert-sorted normalised tokens
     __half *h;
-    float *y_acc;
+    float *orows;           // weighted expert output per expert-sorted row
     unsigned int *err;
     unsigned long long wait_limit_ns;
-    CUtensorMap map_xn16;   // gather4 rows of the normalised tokens
-    CUtensorMap map_h;      // 16-row boxes of h
+    CUtensorMap map_xperm[4];  // boxes of 16/32/48/64 rows of the expert-sorted normalised tokens
+    CUtensorMap map_h[4];      // boxes of 16/32/48/64 rows of h
     const void *w13_ptr;
     CUtensorMap map_w13;
     const void *w2_ptr;
@@ -118,8 +122,10 @@ Buf ws_buffer(moe_ctx *c, int which) {
         case MOE_WS_ROW_TOKEN: return {c->row_token, P * 4};
         case MOE_WS_ROW_W: return {c->row_w, P * 4};
         case MOE_WS_H: return {c->h, P * s.d_ff * 2};
-        case MOE_WS_YACC: return {c->y_acc, T * s.d_model * 4};
+        case MOE_WS_OUT_ROWS: return {c->orows, P * s.d_model * 4};
         case MOE_WS_TILES: return {c->tiles, (E + 1) * 4};
+        case MOE_WS_PAIR_ROW: return {c->pair_row, P * 4};
+        case MOE_WS_XPERM: return {c->xperm, P * s.d_model * 2};
         default: return {nullptr, 0};
     }
 }
@@ -140,19 +146,25 @@ int token_block_rows(int T) {
     return nb < 256 ? nb : 256;
 }
 
+// Rows per B TMA box: the whole token block up to 64 rows (a TMA instruction
+// costs its issuing thread ~100+ cycles, so fewer, larger boxes).
+int b_box_rows(int nb_rows) { return nb_rows < 64 ? nb_rows : 64; }
+
 int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
                 const uint16_t *bias, cudaStream_t stream) {
     const moe_shape_t &s = c->shape;
     GemmParams p;
     memset(&p, 0, sizeof p);
     const int E = s.n_experts, d = s.d_model, F = s.d_ff;
+    p.nb_rows = token_block_rows(T);
     if (mode == MODE_UP) {
         if (codes != c->w13_ptr) {
             if (!encode_codes(&c->map_w13, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
             c->w13_ptr = codes;
         }
         p.map_codes = c->map_w13;
-        p.map_b = c->map_xn16;
+        p.b_box_rows = b_box_rows(p.nb_rows);
+        p.map_b = c->map_xperm[p.b_box_rows / 16 - 1];
         p.K = d;
         p.R = 2 * F;
         p.MB = F / 64;
@@ -164,28 +176,36 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
             c->w2_ptr = codes;
         }
         p.map_codes = c->map_w2;
-        p.map_b = c->map_h;
+        p.b_box_rows = b_box_rows(p.nb_rows);
+        p.map_b = c->map_h[p.b_box_rows / 16 - 1];
         p.K = F;
         p.R = d;
         p.MB = (d + GEMM_BM - 1) / GEMM_BM;
-        p.out = c->y_acc;
+        p.out = c->orows;
         p.out_ld = d;
     }
     p.scales = scales;
     p.bias = bias;
     p.F = F;
     p.E = E;
-    p.nb_rows = token_block_rows(T);
-    p.b_stage_bytes = p.nb_rows * 128;
-    p.n_d_bufs = p.nb_rows <= 128 ? 2 : 1;
-    // TMEM: A slots first, then the accumulator buffer(s)
-    p.n_a_slots = (512 - p.n_d_bufs * p.nb_rows) / 32;
+    p.b_stage_bytes = (p.nb_rows + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows * 128;
+    // MMA warps: a tcgen05.mma holds its issuing thread ~120 cycles, so small
+    // token blocks use up to three issuers (each its own accumulator)
+    const int n_sub = p.K / GEMM_KA;
+    int ni = 256 / p.nb_rows;
+    if (ni > GEMM_ISS_MAX) ni = GEMM_ISS_MAX;
+    if (ni > n_sub) ni = n_sub;
+    if (ni < 1) ni = 1;
+    p.n_iss = ni;
+    p.n_d_bufs = (2 * ni * p.nb_rows <= 256) ? 2 : 1;
+    // TMEM: A slots first, then the accumulators
+    p.n_a_slots = (512 - p.n_d_bufs * ni * p.nb_rows) / 32;
     if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
     p.n_a_slots &= ~1;
-    // shared memory: as many code stages as fit (up to 8) next to a B ring of at
-    // least 3 stages (up to 16), then whatever is left goes to the code ring
+    // shared memory: up to 8 code stages next to a B ring of at least 3 stages
+    // (up to 16); whatever is left goes to the code ring
     const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, p.b_stage_bytes);
-    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 24);
+    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 16);
     int nbs = 16, sc = 8;
     while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && nbs > 3) --nbs;
     while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && sc > 4) --sc;
@@ -258,7 +278,12 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
 
     const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
     const size_t sizes[] = {T * s.d_model * 2, T * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
-                            P * 4, P * 4, P * s.d_ff * 2, T * s.d_model * 4, 64};
+                            P * 4, P * 4, P * 4, P * s.d_model * 2, P * s.d_ff * 2,
+                            P * s.d_model * 4, 64};
+    void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
+                      (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
+                      (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xperm, (void **)&c->h,
+                      (void **)&c->orows, (void **)&c->err};
     size_t total = 0;
     for (size_t v : sizes) total += round256(v);
     if (cudaMalloc(&c->ws, total) != cudaSuccess) {
@@ -268,16 +293,15 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
     }
     c->ws_bytes = total;
     char *b = static_cast<char *>(c->ws);
-    void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
-                      (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
-                      (void **)&c->row_w, (void **)&c->h, (void **)&c->y_acc, (void **)&c->err};
     for (size_t i = 0; i < sizeof(sizes) / sizeof(sizes[0]); ++i) {
-        *slots[i] = b;
+        *slots[i] = sizes[i] ? b : nullptr;
         b += round256(sizes[i]);
     }
-    if (cudaMemset(c->ws, 0, total) != cudaSuccess ||
-        !encode_f16_rows(&c->map_xn16, c->xn16, s.T_max, s.d_model, 1) ||
-        !encode_f16_rows(&c->map_h, c->h, (int)P, s.d_ff, 16)) {
+    bool maps_ok = cudaMemset(c->ws, 0, total) == cudaSuccess;
+    for (int i = 0; i < 4 && maps_ok; ++i)
+        maps_ok = encode_f16_rows(&c->map_xperm[i], c->xperm, (int)P, s.d_model, 16 * (i + 1)) &&
+                  encode_f16_rows(&c->map_h[i], c->h, (int)P, s.d_ff, 16 * (i + 1));
+    if (!maps_ok) {
         cudaFree(c->ws);
         delete c;
         return MOE_ERR_CUDA;
@@ -314,7 +338,6 @@ int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale
     p.rho = c->rho;
     p.topk_idx = c->topk_idx;
     p.topk_w = c->topk_w;
-    p.y_acc = c->y_acc;
     return cuda_status(launch_route(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -334,8 +357,12 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     p.tiles = c->tiles;
     p.row_token = c->row_token;
     p.row_w = c->row_w;
+    p.pair_row = c->pair_row;
     p.err = c->err;
-    return cuda_status(launch_group(p, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc2 = cuda_status(launch_group(p, st));
+    if (rc2) return rc2;
+    return cuda_status(launch_permute(c->xn16, c->row_token, c->xperm, p.P, c->shape.d_model, st));
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
@@ -356,14 +383,14 @@ int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, con
     return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, static_cast<cudaStream_t>(stream));
 }
 
-int moe_finalize(moe_ctx_t *c, int T, int top_k, uint16_t *y, int32_t *topk_idx_out, float *topk_w_out,
-                 void *stream) {
+int moe_finalize(moe_ctx_t *c, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,
+                 float *topk_w_out, void *stream) {
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!aligned16(y)) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y) || x == y) return MOE_ERR_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(launch_finalize(c->y_acc, y, (long long)T * c->shape.d_model, s));
+    rc = cuda_status(launch_combine(x, c->orows, c->pair_row, y, T, c->shape.d_model, top_k, s));
     if (rc) return rc;
     const size_t pk = (size_t)T * top_k;
     if (topk_idx_out && cudaMemcpyAsync(topk_idx_out, c->topk_idx, pk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -390,7 +417,7 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
     if ((rc = moe_group(c, T, top_k, stream))) return rc;
     if ((rc = moe_expert_up(c, T, top_k, w13_codes, w13_scales, b13, stream))) return rc;
     if ((rc = moe_expert_down(c, T, top_k, w2_codes, w2_scales, b2, stream))) return rc;
-    return moe_finalize(c, T, top_k, y, topk_idx_out, topk_w_out, stream);
+    return moe_finalize(c, T, top_k, x, y, topk_idx_out, topk_w_out, stream);
 }
 
 int moe_copy_workspace(moe_ctx_t *c, int which, void *dst, size_t bytes, void *stream) {

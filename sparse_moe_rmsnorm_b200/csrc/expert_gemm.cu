@@ -10,25 +10,30 @@
 //     row exact in fp16) and store them straight into tensor memory, where
 //     the MMA reads A ("A from TMEM" form).  The decoded weights never touch
 //     shared memory, so shared-memory bandwidth is left to the codes and B.
-//   B (activations, N = tokens, K-major fp16): TMA into a shared-memory ring
-//     in the 128-byte swizzled canonical layout -- gathered row by row
-//     (tile::gather4) from the normalised tokens for the gate/up GEMM,
-//     contiguous expert-sorted rows of h for the down GEMM.
-//   D (fp32, 128 lanes x N columns) accumulates in TMEM; epilogue warps read
-//     it back with tcgen05.ld.
+//   B (activations, N = tokens, K-major fp16): TMA boxes of up to 64
+//     expert-sorted rows (the sorted copy of the normalised tokens for the
+//     gate/up GEMM, h for the down GEMM) into a shared-memory ring in the
+//     128-byte swizzled canonical layout.
+//   D (fp32, 128 lanes x N columns) accumulates in TMEM.  A tcgen05.mma
+//     occupies its issuing thread for about 120 cycles whatever N is, so small
+//     token blocks are spread over up to three MMA warps, each accumulating
+//     every third sub-stage into its own accumulator; the epilogue sums them.
 // Gate/up epilogue: z = D * 2^c * rho_token + b13, clamped SwiGLU
 //   h = min(g,7) * sigmoid(1.702 min(g,7)) * (clamp(u,-7,7) + 1)
 //   ("gpt-oss-20B" hub page, section 3.3); each 128-row block holds 64 gate
 //   rows and their 64 linear rows so the pair meets in one warp.
-// Down epilogue: y_acc[token] += w_token * (D * 2^c + b2) by fp32 atomics
+// Down epilogue: o = w_token * (D * 2^c + b2) written to the pair's
+//   expert-sorted row; the combine kernel adds a token's rows to its residual
 //   (weighted combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
 //
-// Warp roles (512 threads): 0 codes/scales TMA, 1 MMA issue, 2 B TMA,
-// 3 TMEM allocation, 4-7 and 12-15 two decoder groups (alternate sub-stages),
-// 8-11 epilogue.  The decoders hand each row's power-of-two shift to the
-// epilogue through shared memory.  Every mbarrier wait is
-// bounded (WaitCtl); when one runs out the CTA stops issuing work, drains its
-// copies and MMAs in flight, frees TMEM and returns with the error latched.
+// Warp roles (672 threads): 0 codes/scales producer, 20 B producer (TMA
+// instructions hold their issuing thread too, so the two streams get their
+// own threads), 1-3 MMA issue (3 also allocates TMEM), 4-7 and 12-15 two
+// decoder groups (alternate two-sub-stage chunks), 8-11 and 16-19 two
+// epilogue groups (alternate 16-column chunks).  The decoders hand each row's power-of-two shift to the
+// epilogue through shared memory.  Every mbarrier wait is bounded (WaitCtl);
+// when one runs out the CTA stops issuing work, drains its copies and MMAs in
+// flight, frees TMEM and returns with the error latched.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -89,29 +94,19 @@ __device__ __forceinline__ int row_scale_max(const uint8_t *s, int n) {
     return m;
 }
 
-__device__ __forceinline__ float select4(const float (&v)[16], int base, int i) {
-    const float a = v[base], b = v[base + 1], c = v[base + 2], d = v[base + 3];
-    return i == 0 ? a : (i == 1 ? b : (i == 2 ? c : d));
-}
-
-__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const GemmSmem plan = gemm_smem_plan(p.K, p.E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
-    const int SC = p.n_c_stages, NA = p.n_a_slots;
+    const int SC = p.n_c_stages, NA = p.n_a_slots, NBS = p.n_b_stages, NI = p.n_iss;
     uint8_t *code_ring = smem + plan.code_off;
     uint8_t *b_ring = smem + plan.b_off;
     uint8_t *scale_buf = smem + plan.scale_off;
     const int scale_bytes = align_up(GEMM_BM * (p.K / 32), 128);
-    int *meta_tok = reinterpret_cast<int *>(smem + plan.meta_off);                    // [4][NB_MAX]
-    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off + 4 * GEMM_NB_MAX * 4);  // [4][NB_MAX]
-    int *shift_s = reinterpret_cast<int *>(smem + plan.shift_off);                   // [2][128]
+    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off);    // [8 warps][NB_MAX / 2]
+    int *tok_s = reinterpret_cast<int *>(smem + plan.tok_off);            // [NB_MAX]
+    int *shift_s = reinterpret_cast<int *>(smem + plan.shift_off);        // [2][128]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bar_off);
     uint64_t *c_full = bars;
     uint64_t *c_empty = c_full + SC;
@@ -120,12 +115,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *a_full = s_empty + 2;
     uint64_t *a_empty = a_full + NA;
     uint64_t *b_full = a_empty + NA;
-    uint64_t *b_empty = b_full + p.n_b_stages;
-    uint64_t *d_full = b_empty + p.n_b_stages;
+    uint64_t *b_empty = b_full + NBS;
+    uint64_t *d_full = b_empty + NBS;
     uint64_t *d_empty = d_full + 2;
     uint64_t *h_full = d_empty + 2;
     uint64_t *h_empty = h_full + 2;
-    uint64_t *drain_bar = h_empty + 2;
+    uint64_t *drain_bar = h_empty + 2;                                     // [GEMM_ISS_MAX]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
@@ -134,7 +129,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB32 = p.K / 32;
-    const int n_sub_total = p.K / GEMM_KA;
+    const int n_sub = p.K / GEMM_KA;
     const int n_cstages = (p.K + GEMM_KS - 1) / GEMM_KS;
 
     if (threadIdx.x == 0) {
@@ -145,20 +140,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&s_empty[i], 8);
-            mbar_init(&d_full[i], 1);
-            mbar_init(&d_empty[i], 4);
+            mbar_init(&d_full[i], NI);     // one commit per MMA warp
+            mbar_init(&d_empty[i], 8);     // both epilogue groups
             mbar_init(&h_full[i], 4);
-            mbar_init(&h_empty[i], 4);
+            mbar_init(&h_empty[i], 8);
         }
         for (int i = 0; i < NA; ++i) {
             mbar_init(&a_full[i], 4);      // the four warps of the group that decoded the slot
             mbar_init(&a_empty[i], 1);
         }
-        for (int i = 0; i < p.n_b_stages; ++i) {
+        for (int i = 0; i < NBS; ++i) {
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
-        mbar_init(drain_bar, 1);
+        for (int i = 0; i < GEMM_ISS_MAX; ++i) mbar_init(&drain_bar[i], 1);
         *abort_s = 0;
         fence_barrier_init();
     }
@@ -178,7 +173,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     const int total = p.MB * tiles_s[p.E];
     const WaitCtl wc{abort_s, p.err, MODE == MODE_UP ? (unsigned)ERR_WAIT_UP : (unsigned)ERR_WAIT_DOWN,
                      p.wait_limit_ns};
-    const int d_stride = p.n_d_bufs == 2 ? p.nb_rows : 0;
+    // accumulator of MMA warp i in buffer set db: columns NA*32 + (db*NI + i)*nb_rows
+    const uint32_t d_col0 = (uint32_t)(NA * 32);
 
     if (warp == 0) {
         // ------------------------------------------------ codes + scales producer
@@ -226,21 +222,51 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 drain_ring(s_full, 2, s_issued, p.wait_limit_ns);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue
+    } else if (warp == 20) {
+        // ------------------------------------------------------------ B producer
         if (lane == 0) {
-            int aslot = 0, bslot = 0, db = 0;
-            uint32_t aph = 0, bph = 0, dph = 0;
-            bool ok = true, issued = false;
+            tma_prefetch_desc(&p.map_b);
+            int bslot = 0;
+            uint32_t bph = 0;
+            long long b_issued = 0;
+            bool ok = true;
+            const int box = p.b_box_rows;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                Work t;
+                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
+                const int nbox = (t.n_mma + box - 1) / box;
+                for (int j = 0; j < n_sub; ++j) {
+                    if (!mbar_wait(&b_empty[bslot], bph ^ 1, wc)) { ok = false; break; }
+                    uint8_t *bdst = b_ring + bslot * p.b_stage_bytes;
+                    mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)(nbox * box * 128));
+                    for (int g = 0; g < nbox; ++g)
+                        tma_load_2d(bdst + g * box * 128, &p.map_b, &b_full[bslot], j * GEMM_KA, t.p0 + box * g);
+                    ++b_issued;
+                    if (++bslot == NBS) { bslot = 0; bph ^= 1; }
+                }
+            }
+            if (!ok) drain_ring(b_full, NBS, b_issued, p.wait_limit_ns);
+        }
+    } else if (warp >= 1 && warp <= 3) {
+        // ------------------------------------------- MMA issue: warp i-1 takes sub-stages i-1, i-1+NI, ...
+        const int mi = warp - 1;
+        if (lane == 0 && mi < NI) {
+            int db = 0;
+            uint32_t dph = 0;
+            long long g0 = 0;                      // running index of the work item's first sub-stage
+            bool ok = true, issued = false;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x, g0 += n_sub) {
                 Work t;
                 work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
                 const uint32_t idesc = idesc_f16_f32(GEMM_BM, (uint32_t)t.n_mma);
                 if (!mbar_wait(&d_empty[db], dph ^ 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(NA * 32 + db * d_stride);
-                for (int s = 0; s < n_sub_total; ++s) {
-                    if (!mbar_wait(&a_full[aslot], aph, wc) || !mbar_wait(&b_full[bslot], bph, wc)) {
+                const uint32_t d_tmem = tmem + d_col0 + (uint32_t)((db * NI + mi) * p.nb_rows);
+                for (int j = mi; j < n_sub; j += NI) {
+                    const long long g = g0 + j;
+                    const int aslot = (int)(g % NA), bslot = (int)(g % NBS);
+                    if (!mbar_wait(&a_full[aslot], (uint32_t)((g / NA) & 1), wc) ||
+                        !mbar_wait(&b_full[bslot], (uint32_t)((g / NBS) & 1), wc)) {
                         ok = false;
                         break;
                     }
@@ -250,67 +276,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
-                                   (s | kk) != 0 ? 1u : 0u);
+                                   (j != mi || kk != 0) ? 1u : 0u);
                     issued = true;
                     mma_commit(&a_empty[aslot]);
                     mma_commit(&b_empty[bslot]);
-                    if (++aslot == NA) { aslot = 0; aph ^= 1; }
-                    if (++bslot == p.n_b_stages) { bslot = 0; bph ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit(&d_full[db]);
                 if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
             }
             if (!ok && issued) {
-                mma_commit(drain_bar);
-                mbar_wait_drain(drain_bar, 0, p.wait_limit_ns);
+                mma_commit(&drain_bar[mi]);
+                mbar_wait_drain(&drain_bar[mi], 0, p.wait_limit_ns);
             }
         }
-    } else if (warp == 2) {
-        // ------------------------------------------------------ B (tokens) producer
-        if (lane == 0) tma_prefetch_desc(&p.map_b);
-        int bslot = 0;
-        uint32_t bph = 0;
-        long long b_issued = 0;
-        bool ok = true;
-        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-            Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-            // gather rows this lane issues: groups g = lane and lane + 32 (4 rows each)
-            int tok[2][4];
-            if (MODE == MODE_UP) {
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int row = 4 * (lane + 32 * u) + r;
-                        tok[u][r] = row < t.n_mma ? p.row_token[t.p0 + (row < t.n_valid ? row : 0)] : 0;
-                    }
-            }
-            for (int s = 0; s < n_sub_total; ++s) {
-                const bool okw = __all_sync(0xffffffffu, mbar_wait(&b_empty[bslot], bph ^ 1, wc));
-                if (!okw) { ok = false; break; }
-                uint8_t *bdst = b_ring + bslot * p.b_stage_bytes;
-                if (lane == 0) mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)t.n_mma * 128u);
-                __syncwarp();
-                if (MODE == MODE_UP) {
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int g = lane + 32 * u;
-                        if (4 * g < t.n_mma)
-                            tma_gather4(bdst + g * 512, &p.map_b, &b_full[bslot], s * GEMM_KA, tok[u][0], tok[u][1],
-                                        tok[u][2], tok[u][3]);
-                    }
-                } else {
-                    const int g = lane;
-                    if (16 * g < t.n_mma) tma_load_2d(bdst + g * 2048, &p.map_b, &b_full[bslot], s * GEMM_KA, t.p0 + 16 * g);
-                }
-                ++b_issued;
-                if (++bslot == p.n_b_stages) { bslot = 0; bph ^= 1; }
-            }
-        }
-        if (!ok && lane == 0) drain_ring(b_full, p.n_b_stages, b_issued, p.wait_limit_ns);
-    } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+    } else if ((warp >= 4 && warp < 8) || (warp >= 12 && warp < 16)) {
         // ------------------------------------------------------------ decoders
         // Two groups of four warps.  Each code stage (4 sub-stages of 64 K
         // elements) is cut into chunks of two sub-stages; group g decodes the
@@ -375,7 +355,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                                 uint32_t h4[4];
                                 e2m1x8_to_half2x4(words[i], h4);
 #pragma unroll
-                                for (int j = 0; j < 4; ++j) out[4 * i + j] = hmul2_u32(h4[j], i < 4 ? m0 : m1);
+                                for (int jj = 0; jj < 4; ++jj) out[4 * i + jj] = hmul2_u32(h4[jj], i < 4 ? m0 : m1);
                             }
                         } else {
 #pragma unroll
@@ -399,13 +379,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (lane == 0) mbar_arrive(&s_empty[sb]);
             if (++sb == 2) { sb = 0; sph ^= 1; }
         }
-    } else if (warp >= 8 && warp < 12) {
+    } else if ((warp >= 8 && warp < 12) || (warp >= 16 && warp < 20)) {
         // ------------------------------------------------------------- epilogue
+        // Two groups of four warps; group eg takes the 16-column chunks
+        // eg, eg+2, eg+4, ... of the accumulators, summing the MMA warps' parts.
         const int q = warp & 3;
+        const int eg = warp >= 16 ? 1 : 0;
         const int tl = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        int *mtok = meta_tok + q * GEMM_NB_MAX;
-        float *mval = meta_val + q * GEMM_NB_MAX;
+        float *mval = meta_val + (eg * 4 + q) * (GEMM_NB_MAX / 2);      // value of chunk m's column i at [(m/2)*16 + i]
         int db = 0, hb = 0;
         uint32_t dph = 0, hph = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -421,12 +403,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 row_valid = row < p.R;
             }
             const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + row]) : 0.f;
-            // per-column token and rho (UP) or routing weight (DOWN), one warp-private copy
-            for (int cc = lane; cc < t.n_mma; cc += 32) {
-                const int col = min(cc, t.n_valid - 1);
-                const int tok = p.row_token[t.p0 + col];
-                mtok[cc] = tok;
-                mval[cc] = MODE == MODE_UP ? p.rho[tok] : p.row_w[t.p0 + col];
+            // per-column rho (UP) or routing weight (DOWN) of this group's columns
+            for (int cc = lane; cc < GEMM_NB_MAX / 2; cc += 32) {
+                const int col = ((cc >> 4) * 2 + eg) * 16 + (cc & 15);
+                if (col < t.n_mma) {
+                    const int pr = t.p0 + min(col, t.n_valid - 1);
+                    mval[cc] = MODE == MODE_UP ? p.rho[p.row_token[pr]] : p.row_w[pr];
+                }
             }
             __syncwarp();
             if (!__all_sync(0xffffffffu, mbar_wait(&h_full[hb], hph, wc))) break;
@@ -436,15 +419,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (++hb == 2) { hb = 0; hph ^= 1; }
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
             tc_fence_after();
-            const uint32_t d_tmem = lane_base + (uint32_t)(NA * 32 + db * d_stride);
-            for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(d_tmem + (uint32_t)c0, v);
-                tmem_wait_ld();
+            const uint32_t d_tmem = lane_base + d_col0 + (uint32_t)(db * NI * p.nb_rows);
+            for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
+                float acc[16];
+                {
+                    uint32_t v[16];
+                    tmem_ld16(d_tmem + (uint32_t)c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
+                }
+                for (int mi = 1; mi < NI; ++mi) {
+                    uint32_t v[16];
+                    tmem_ld16(d_tmem + (uint32_t)(mi * p.nb_rows + c0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+                }
+                const float *mv = mval + (c0 >> 5) * 16;
                 if (MODE == MODE_UP) {
                     float z[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) z[i] = __uint_as_float(v[i]) * (cscale * mval[c0 + i]) + bias;
+                    for (int i = 0; i < 16; ++i) z[i] = acc[i] * (cscale * mv[i]) + bias;
                     __half *hout = reinterpret_cast<__half *>(p.out);
                     const int jrow = t.mb * 64 + 16 * q + (lane & 15);
 #pragma unroll
@@ -456,40 +452,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         const int col = c0 + (lane < 16 ? i : 8 + i);
                         const float g = fminf(gate, 7.0f);
                         const float u = fminf(fmaxf(lin, -7.0f), 7.0f);
-                        const float h = g / (1.0f + __expf(-1.702f * g)) * (u + 1.0f);
+                        const float h = __fdividef(g, 1.0f + __expf(-1.702f * g)) * (u + 1.0f);
                         if (col < t.n_valid) hout[(size_t)(t.p0 + col) * p.out_ld + jrow] = __float2half_rn(h);
                     }
                 } else {
-                    // weighted outputs of this lane's row, then a 4x4 transpose inside each
-                    // quad of lanes so every lane holds 4 consecutive rows of one column
-                    float val[16];
+                    // weighted expert output w * (W2 h + b2), one expert-sorted row per column
+                    float *o = reinterpret_cast<float *>(p.out);
+                    if (row_valid) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) val[i] = (__uint_as_float(v[i]) * cscale + bias) * mval[c0 + i];
-                    const int j = lane & 3;
-                    float *y = reinterpret_cast<float *>(p.out);
-                    const int row4 = t.mb * GEMM_BM + 32 * q + (lane & ~3);
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        float o[4];
-                        o[0] = o[1] = o[2] = o[3] = 0.f;
-                        const float own = select4(val, 4 * m, j);
-#pragma unroll
-                        for (int r = 1; r < 4; ++r) {
-                            const float send = select4(val, 4 * m, j ^ r);
-                            const float recv = __shfl_xor_sync(0xffffffffu, send, r);
-                            const int dst = j ^ r;
-                            o[0] = dst == 0 ? recv : o[0];
-                            o[1] = dst == 1 ? recv : o[1];
-                            o[2] = dst == 2 ? recv : o[2];
-                            o[3] = dst == 3 ? recv : o[3];
-                        }
-                        if (j == 0) o[0] = own;
-                        if (j == 1) o[1] = own;
-                        if (j == 2) o[2] = own;
-                        if (j == 3) o[3] = own;
-                        const int col = c0 + 4 * m + j;
-                        if (col < t.n_valid && row4 < p.R)
-                            red_add_v4(y + (size_t)mtok[col] * p.out_ld + row4, o[0], o[1], o[2], o[3]);
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < t.n_valid)
+                                o[(size_t)(t.p0 + c0 + i) * p.out_ld + row] = (acc[i] * cscale + bias) * mv[i];
                     }
                 }
             }

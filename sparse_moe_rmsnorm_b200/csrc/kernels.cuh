@@ -27,7 +27,6 @@ struct RouteParams {
     float *rho;                 // fp32 [T]
     int *topk_idx;              // [T, k]
     float *topk_w;              // [T, k]
-    float *y_acc;               // fp32 [T, d] initialised to x
 };
 
 struct GroupParams {
@@ -39,18 +38,19 @@ struct GroupParams {
     int *tiles;                 // [E+1] prefix of ceil(counts / nb_rows)
     int *row_token;             // [P]
     float *row_w;               // [P]
+    int *pair_row;              // [P] expert-sorted row of pair (token, slot)
     unsigned int *err;
 };
 
 // Grouped MXFP4 x fp16 GEMM over (expert, 128-row weight block, token block)
 // work items.  MODE_UP: rows are the gate/linear pairs of W13, epilogue is the
-// clamped SwiGLU into h.  MODE_DOWN: rows are W2's, epilogue scales by the
-// routing weight and adds into the fp32 output accumulator.
+// clamped SwiGLU into h.  MODE_DOWN: rows are W2's, epilogue writes the
+// routing-weighted expert output rows.
 enum { MODE_UP = 0, MODE_DOWN = 1 };
 
 struct GemmParams {
     CUtensorMap map_codes;      // u8 [E][R][K/2], box {128 bytes, 64 (UP) or 128 (DOWN) rows, 1}, 128B swizzle
-    CUtensorMap map_b;          // UP: fp16 xn16 [T][d] box {64, 1} (gather4); DOWN: fp16 h [P][F] box {64, 16}
+    CUtensorMap map_b;          // fp16 expert-sorted B rows [P][K], box {64 elements, b_box_rows rows}
     const uint8_t *scales;      // u8 [E][R][K/32]
     const uint16_t *bias;       // bf16 [E][R]
     int K;                      // reduction length
@@ -59,42 +59,45 @@ struct GemmParams {
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= 256)
+    int b_box_rows;             // rows per B TMA box (16..64); a B stage holds round_up(nb_rows, b_box_rows) rows
     int n_b_stages;             // B ring depth
     int b_stage_bytes;          // nb_rows * 128
-    int n_d_bufs;               // 1 or 2 accumulator buffers in TMEM
     int n_c_stages;             // code ring depth (shared-memory stages of 128 rows x 128 bytes)
     int n_a_slots;              // TMEM A slots (32 columns each); accumulators follow them
+    int n_iss;                  // MMA-issuing warps, each with its own accumulator
+    int n_d_bufs;               // accumulator buffer sets (1 or 2)
     const int *counts, *offsets, *tiles;
     const int *row_token;       // [P]
     const float *row_w;         // [P]
     const float *rho;           // [T] (UP)
-    void *out;                  // UP: fp16 h [P][F]; DOWN: fp32 y_acc [T][d]
+    void *out;                  // UP: fp16 h [P][F]; DOWN: fp32 weighted outputs [P][d]
     int out_ld;                 // F (UP) or d (DOWN)
     unsigned int *err;
     unsigned long long wait_limit_ns;
 };
 
-constexpr int GEMM_THREADS = 512;
+constexpr int GEMM_THREADS = 672;     // 21 warps
 constexpr int GEMM_BM = 128;          // weight rows per work item (TMEM lanes)
 constexpr int GEMM_KS = 256;          // K elements per code stage: 128 bytes per row
 constexpr int GEMM_KA = 64;           // K elements per TMEM A slot: 32 columns
 constexpr int GEMM_SC_MAX = 10;       // code stages, at most
 constexpr int GEMM_NA_MAX = 14;       // TMEM A slots, at most
 constexpr int GEMM_NB_MAX = 256;      // token rows per work item, at most
+constexpr int GEMM_ISS_MAX = 3;       // MMA-issuing warps, at most
 constexpr int GEMM_CODE_STAGE = GEMM_BM * 128;
 constexpr int GEMM_SMEM_LIMIT = 227 * 1024;
 
 // Shared-memory plan of the GEMM kernel (all offsets from a 1024-aligned base).
 struct GemmSmem {
-    int code_off, b_off, scale_off, meta_off, shift_off, bar_off, misc_off, total;
+    int code_off, b_off, scale_off, meta_off, tok_off, shift_off, bar_off, misc_off, total;
 };
 
 __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline int gemm_num_barriers(int n_c_stages, int n_a_slots, int n_b_stages) {
     // code full/empty, scale full/empty, A full/empty, B full/empty, D full/empty,
-    // row-shift full/empty, drain
-    return 2 * n_c_stages + 4 + 2 * n_a_slots + 2 * n_b_stages + 4 + 4 + 1;
+    // row-shift full/empty, one drain barrier per MMA warp
+    return 2 * n_c_stages + 4 + 2 * n_a_slots + 2 * n_b_stages + 4 + 4 + GEMM_ISS_MAX;
 }
 
 __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int n_c_stages, int n_a_slots, int n_b_stages,
@@ -105,7 +108,8 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int n_c_stages,
     s.scale_off = s.b_off + n_b_stages * b_stage_bytes;
     const int scale_bytes = align_up(GEMM_BM * (K / 32), 128);
     s.meta_off = s.scale_off + 2 * scale_bytes;
-    s.shift_off = s.meta_off + 4 * GEMM_NB_MAX * 8;          // per epilogue warp: token + value per column
+    s.tok_off = s.meta_off + 8 * (GEMM_NB_MAX / 2) * 4;         // per epilogue warp: one value per its columns
+    s.shift_off = s.tok_off + GEMM_NB_MAX * 4;                  // producer's token list of the work item
     s.bar_off = s.shift_off + 2 * GEMM_BM * 4;
     s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_c_stages, n_a_slots, n_b_stages) * 8, 16);
     // misc: tmem base, abort flag, then counts/offsets/tiles caches

@@ -1,10 +1,10 @@
 // Routing side of the MoE block on sm_100a:
 //   route_kernel     RMSNorm + router logits + top-k + softmax over the chosen,
-//                    plus the fp16 normalised tokens for the experts and the
-//                    fp32 output accumulator initialised to the residual x;
+//                    plus the fp16 normalised tokens for the experts;
 //   group_kernel     expert histogram, exclusive scan and a stable permutation
 //                    of the (token, expert) pairs into expert-contiguous rows;
-//   finalize_kernel  fp32 accumulator -> bf16 y.
+//   permute_kernel   the expert-sorted copy of the normalised tokens;
+//   combine_kernel   y = x + the token's weighted expert rows, in bf16.
 #include <cfloat>
 #include <climits>
 
@@ -93,7 +93,6 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
     float ss = 0.f;
     if (has_tok) {
         const uint16_t *xr = p.x + (size_t)t * d;
-        float *ya = p.y_acc + (size_t)t * d;
         for (int j = u * 8; j < d; j += WPT * 256) {
             float f[8];
             bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xr + j), f);
@@ -102,8 +101,6 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
                 ss += f[c] * f[c];
                 xsr[j + c] = f[c];
             }
-            reinterpret_cast<float4 *>(ya + j)[0] = make_float4(f[0], f[1], f[2], f[3]);
-            reinterpret_cast<float4 *>(ya + j)[1] = make_float4(f[4], f[5], f[6], f[7]);
         }
     }
     ss = warp_sum(ss);
@@ -379,6 +376,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
                 const int pos = off_s[e] + wcnt[warp][e] + __popc(m & ((1u << lane) - 1u));
                 p.row_token[pos] = i / p.k;
                 p.row_w[pos] = wv[r];
+                p.pair_row[i] = pos;
             }
             __syncwarp();
             if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp][e] += __popc(m);
@@ -387,22 +385,52 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
     }
 }
 
-// -------------------------------------------------------------- finalize
+// --------------------------------------------------------------- permute
+//
+// xperm[p] = xn16[row_token[p]]: the normalised tokens in expert-sorted row
+// order, so the gate/up GEMM reads its token blocks as contiguous rows.  One
+// warp per row, 16-byte copies.
+__global__ void __launch_bounds__(256) permute_kernel(const __half *__restrict__ xn16, const int *__restrict__ row_token,
+                                                      __half *__restrict__ xperm, int P, int d) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int r = warp; r < P; r += nwarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(xn16 + (size_t)row_token[r] * d);
+        uint4 *dst = reinterpret_cast<uint4 *>(xperm + (size_t)r * d);
+        for (int j = lane; j < d / 8; j += 32) dst[j] = src[j];
+    }
+}
 
-__global__ void __launch_bounds__(256) finalize_kernel(const float *__restrict__ y_acc, uint16_t *__restrict__ y,
-                                                       long long n8) {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+// --------------------------------------------------------------- combine
+//
+// y[t] = bf16(x[t] + sum_i o[pair_row[t*k + i]]) in fp32, the k weighted
+// expert rows added in the token's slot order (descending router logit), so
+// the result does not depend on scheduling.  Each thread handles 8
+// consecutive features of one token.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict__ x, const float *__restrict__ orows,
+                                                      const int *__restrict__ pair_row, uint16_t *__restrict__ y,
+                                                      int T, int d, int k) {
+    const int per_tok = d / 8;
+    const long long n = (long long)T * per_tok;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
-        const float4 a = reinterpret_cast<const float4 *>(y_acc)[2 * i];
-        const float4 b = reinterpret_cast<const float4 *>(y_acc)[2 * i + 1];
-        const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
-        const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-        uint4 o;
-        o.x = *reinterpret_cast<const uint32_t *>(&p0);
-        o.y = *reinterpret_cast<const uint32_t *>(&p1);
-        o.z = *reinterpret_cast<const uint32_t *>(&p2);
-        o.w = *reinterpret_cast<const uint32_t *>(&p3);
-        reinterpret_cast<uint4 *>(y)[i] = o;
+        const int t = (int)(i / per_tok), j = (int)(i % per_tok) * 8;
+        float acc[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(x + (size_t)t * d + j), acc);
+        for (int s = 0; s < k; ++s) {
+            const float4 *o = reinterpret_cast<const float4 *>(orows + (size_t)pair_row[(size_t)t * k + s] * d + j);
+            const float4 a = o[0], b = o[1];
+            acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+            acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        }
+        const __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[0], acc[1]), p1 = __floats2bfloat162_rn(acc[2], acc[3]);
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[4], acc[5]), p3 = __floats2bfloat162_rn(acc[6], acc[7]);
+        uint4 out;
+        out.x = *reinterpret_cast<const uint32_t *>(&p0);
+        out.y = *reinterpret_cast<const uint32_t *>(&p1);
+        out.z = *reinterpret_cast<const uint32_t *>(&p2);
+        out.w = *reinterpret_cast<const uint32_t *>(&p3);
+        *reinterpret_cast<uint4 *>(y + (size_t)t * d + j) = out;
     }
 }
 
@@ -480,11 +508,19 @@ cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_finalize(const float *y_acc, uint16_t *y, long long n, cudaStream_t s) {
-    const long long n8 = n / 8;
-    if (n8 == 0) return cudaSuccess;
-    const int grid = (int)min((n8 + 255) / 256, (long long)148 * 8);
-    finalize_kernel<<<grid, 256, 0, s>>>(y_acc, y, n8);
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s) {
+    if (P <= 0) return cudaSuccess;
+    const int grid = min((P + 7) / 8, 148 * 8);
+    permute_kernel<<<grid, 256, 0, s>>>(xn16, row_token, xperm, P, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
+                           cudaStream_t s) {
+    const long long n = (long long)T * (d / 8);
+    if (n == 0) return cudaSuccess;
+    const int grid = (int)min((n + 255) / 256, (long long)148 * 8);
+    combine_kernel<<<grid, 256, 0, s>>>(x, orows, pair_row, y, T, d, k);
     return cudaGetLastError();
 }
 

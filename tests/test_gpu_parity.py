@@ -40,7 +40,10 @@ def run_block(inp, k, eps=1e-5, T_max=None):
     y, idx, wts = m.forward(x, w, routing=True)
     torch.cuda.synchronize()
     assert m.sync_status() == moe.MOE_OK
-    yacc = m.workspace("y_acc", T).cpu().numpy().astype(np.float64)
+    # y before the bf16 cast: x + the token's weighted expert rows, summed in float64 here
+    orows = m.workspace("out_rows", T).cpu().numpy().astype(np.float64)
+    pair_row = m.workspace("pair_row", T).cpu().numpy().reshape(T, k)
+    yacc = bf16_bits_to_f32(inp["x"]).astype(np.float64) + orows[pair_row].sum(axis=1)
     out = dict(y=_y_numpy(y), yacc=yacc, idx=idx.cpu().numpy(), w=wts.cpu().numpy().astype(np.float64), ctx=m,
                weights=w, x=x)
     return out
@@ -130,7 +133,6 @@ def test_route_stage(T, d, E, k):
     wts = m.workspace("topk_w", T).cpu().numpy()
     xn16 = m.workspace("xn16", T).float().cpu().numpy().astype(np.float64)
     rho = m.workspace("rho", T).cpu().numpy().astype(np.float64)
-    yacc = m.workspace("y_acc", T).cpu().numpy()
     xn = oracle.rmsnorm(inp["x"], inp["norm_scale"], 1e-5)
     logits = oracle.router(xn, inp["router_w"], inp["router_b"])
     ref_idx, ref_w = oracle.topk_softmax(logits, k)
@@ -143,7 +145,6 @@ def test_route_stage(T, d, E, k):
     amax = np.abs(xn16).max(axis=1)
     assert np.all((amax >= 2.0 ** 13 * (1 - 2 ** -10)) & (amax <= 2.0 ** 14))
     assert np.max(np.abs(xn16 * rho[:, None] - xn) / np.abs(xn).max(axis=1, keepdims=True)) < 6e-4
-    assert np.array_equal(yacc, bf16_bits_to_f32(inp["x"]))
     m.close()
 
 
@@ -162,8 +163,15 @@ def test_group_stage_invariants(T, E, k):
     tiles = m.workspace("tiles", T).cpu().numpy()
     row_token = m.workspace("row_token", T).cpu().numpy()
     row_w = m.workspace("row_w", T).cpu().numpy()
+    pair_row = m.workspace("pair_row", T).cpu().numpy()
+    xn16 = m.workspace("xn16", T).cpu().numpy()
+    xperm = m.workspace("xperm", T).cpu().numpy()
     assert m.sync_status() == moe.MOE_OK
     P = T * k
+    # pair_row inverts the permutation, and the sorted token copy follows it
+    assert np.array_equal(np.sort(pair_row), np.arange(P))
+    assert np.array_equal(row_token[pair_row], np.repeat(np.arange(T), k))
+    assert np.array_equal(xperm, xn16[row_token])
     assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
     assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts) and offsets[-1] == P
     nb = min(256, (T + 15) // 16 * 16)
