@@ -177,6 +177,34 @@ MOE_API int moe_selftest_wait_timeout(moe_ctx_t *ctx, void *stream);
  * of the format. */
 MOE_API int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, void *stream);
 
+/* The whole block (as moe_forward) without any device allocation, for callers
+ * that cannot call cudaMalloc: code running inside a CUDA graph capture that
+ * forbids allocation, frameworks whose allocator owns all device memory, or
+ * plugins whose host does not let library code allocate.  (The gpt-oss
+ * write-ups have no counterpart of this entry point; it is an integration
+ * convenience.)
+ *
+ * Scratch memory comes from one fixed 8 MiB __device__ array inside the
+ * library, held on every GPU that loads it until process exit; no context is
+ * needed.  Limits: T <= MOE_NOALLOC_MAX_TOKENS and the workspace for the shape
+ * (about T*(2d) + T*k*(6d + 2F) bytes, e.g. 6.3 MiB for 64 tokens of the
+ * d_model = d_ff = 2880, top-4 layers) must fit in the array; larger requests
+ * return MOE_ERR_ARG.  Shape limits otherwise as in moe_init.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current: make it outside any stream
+ * capture.  All calls share the one array and the array keeps the last call's
+ * contents, so calls that overlap on the GPU (other streams, other host
+ * threads on the same device) race; serialise them.  Device-side bounded-wait
+ * errors are not reported by this entry point (there is no context to latch
+ * them in); the return value covers argument and launch errors. */
+#define MOE_NOALLOC_MAX_TOKENS 64
+MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int top_k, float eps,
+                                const uint16_t *x, const uint16_t *router_w, const float *router_b,
+                                const uint8_t *w13_codes, const uint8_t *w13_scales, const uint16_t *b13,
+                                const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+                                const uint16_t *norm_scale, uint16_t *y, void *stream);
+
 /* A human-readable name of an error code. */
 MOE_API const char *moe_strerror(int code);
 

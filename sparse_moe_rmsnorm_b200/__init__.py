@@ -23,7 +23,10 @@ __all__ = [
     "moe_init", "moe_destroy", "moe_forward", "moe_route", "moe_group", "moe_expert_up", "moe_expert_down",
     "moe_finalize", "moe_copy_workspace", "moe_sync_status", "moe_set_wait_limit_ns",
     "moe_selftest_wait_timeout", "moe_debug_decode", "moe_strerror", "moe_version", "WS",
+    "moe_forward_noalloc", "MOE_NOALLOC_MAX_TOKENS",
 ]
+
+MOE_NOALLOC_MAX_TOKENS = 64
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_NOMEM = 0, -1, -2, -3, -4, -5
 
@@ -68,6 +71,7 @@ _SIGS = {
     "moe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "moe_debug_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_forward_noalloc": (ctypes.c_int, [ctypes.c_int] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 12),
     "moe_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_version": (ctypes.c_char_p, []),
 }
@@ -162,6 +166,15 @@ def moe_expert_down(ctx, T, top_k, w2_codes, w2_scales, b2, stream=None) -> None
 def moe_finalize(ctx, T, top_k, x, y, topk_idx_out=None, topk_w_out=None, stream=None) -> None:
     _check(lib().moe_finalize(ctx, int(T), int(top_k), _ptr(x), _ptr(y), _ptr(topk_idx_out), _ptr(topk_w_out),
                               _stream(stream)), "moe_finalize")
+
+
+def moe_forward_noalloc(T, d_model, d_ff, n_experts, top_k, eps, x, router_w, router_b, w13_codes, w13_scales, b13,
+                        w2_codes, w2_scales, b2, norm_scale, y, stream=None) -> None:
+    """The whole block with no device allocation (library-owned fixed scratch; see the C header)."""
+    _check(lib().moe_forward_noalloc(int(T), int(d_model), int(d_ff), int(n_experts), int(top_k), float(eps),
+                                     _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(w13_codes), _ptr(w13_scales),
+                                     _ptr(b13), _ptr(w2_codes), _ptr(w2_scales), _ptr(b2), _ptr(norm_scale), _ptr(y),
+                                     _stream(stream)), "moe_forward_noalloc")
 
 
 def moe_copy_workspace(ctx, which, dst, nbytes, stream=None) -> None:

@@ -1,0 +1,285 @@
+// moe_forward_noalloc: the whole MoE block without any device allocation.
+//
+// Some callers cannot call cudaMalloc at all: code that runs while a CUDA
+// graph is being captured in relaxed/global mode, custom allocators that own
+// every byte of device memory, or plugins loaded into a host that forbids
+// allocation from library code.  For them this entry point takes its scratch
+// memory from one file-scope __device__ array of fixed size (every GPU that
+// loads the library holds it until process exit).  The caller still passes
+// every input, the weights and the output.
+//
+// The scratch array's host-side name is only a stand-in: host code gets the
+// device address with cudaGetSymbolAddress, once per device, with that device
+// current; kernels receive that pointer.  The first call on a device does this
+// set-up, so make the first call outside any stream capture.
+//
+// Calls share the array: two calls that overlap on the GPU (different
+// streams, or different host threads on the same device) race on it.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "moe_b200.h"
+
+namespace moe {
+cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
+cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
+                           cudaStream_t s);
+cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+// 8 MiB of scratch: enough for decode-sized batches of the gpt-oss layers
+// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 6.3 MiB).
+constexpr size_t kScratchBytes = 8u << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+unsigned char *g_scratch_ptr[kMaxDevices];   // device address of g_noalloc_scratch, per device
+int g_num_sms[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn noalloc_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+bool enc_codes(CUtensorMap *m, const void *codes, int E, int R, int K, int box_rows) {
+    EncodeTiledFn f = noalloc_encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)R, (cuuint64_t)E};
+    const cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R * (K / 2)};
+    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool enc_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+    EncodeTiledFn f = noalloc_encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool a16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device address of the scratch array on the current device (set up once per device).
+int scratch_for_current_device(unsigned char **ptr, int *num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_ptr[dev]) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        g_num_sms[dev] = prop.multiProcessorCount;
+        g_scratch_ptr[dev] = static_cast<unsigned char *>(p);
+    }
+    *ptr = g_scratch_ptr[dev];
+    *num_sms = g_num_sms[dev];
+    return MOE_OK;
+}
+
+int token_rows(int T) {
+    int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;
+    return nb < 256 ? nb : 256;
+}
+
+// The grouped GEMM launch of one expert stage on scratch-backed buffers.
+int launch_gemm_stage(int mode, int T, int k, int d, int F, int E, int num_sms, const uint8_t *codes,
+                      const uint8_t *scales, const uint16_t *bias, const CUtensorMap *map_b, const int *counts,
+                      const int *offsets, const int *tiles, const int *row_token, const float *row_w,
+                      const float *rho, void *out, unsigned int *err, cudaStream_t stream) {
+    GemmParams p;
+    memset(&p, 0, sizeof p);
+    p.nb_rows = token_rows(T);
+    p.b_box_rows = p.nb_rows < 64 ? p.nb_rows : 64;
+    p.map_b = *map_b;
+    if (mode == MODE_UP) {
+        if (!enc_codes(&p.map_codes, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
+        p.K = d;
+        p.R = 2 * F;
+        p.MB = F / 64;
+        p.out_ld = F;
+    } else {
+        if (!enc_codes(&p.map_codes, codes, E, d, F, 128)) return MOE_ERR_CUDA;
+        p.K = F;
+        p.R = d;
+        p.MB = (d + GEMM_BM - 1) / GEMM_BM;
+        p.out_ld = d;
+    }
+    p.out = out;
+    p.scales = scales;
+    p.bias = bias;
+    p.F = F;
+    p.E = E;
+    p.b_stage_bytes = (p.nb_rows + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows * 128;
+    const int n_sub = p.K / GEMM_KA;
+    int ni = 256 / p.nb_rows;
+    if (ni > GEMM_ISS_MAX) ni = GEMM_ISS_MAX;
+    if (ni > n_sub) ni = n_sub;
+    if (ni < 1) ni = 1;
+    p.n_iss = ni;
+    p.n_d_bufs = (2 * ni * p.nb_rows <= 256) ? 2 : 1;
+    p.n_a_slots = (512 - p.n_d_bufs * ni * p.nb_rows) / 32;
+    if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
+    p.n_a_slots &= ~1;
+    const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, p.b_stage_bytes);
+    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 16);
+    int nbs = 16, sc = 8;
+    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && nbs > 3) --nbs;
+    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && sc > 4) --sc;
+    while ((sc + 1) * GEMM_CODE_STAGE + nbs * p.b_stage_bytes <= room && sc < GEMM_SC_MAX) ++sc;
+    if (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room) return MOE_ERR_ARG;
+    p.n_b_stages = nbs;
+    p.n_c_stages = sc;
+    p.counts = counts;
+    p.offsets = offsets;
+    p.tiles = tiles;
+    p.row_token = row_token;
+    p.row_w = row_w;
+    p.rho = rho;
+    p.err = err;
+    p.wait_limit_ns = 2000000000ull;
+    const GemmSmem plan = gemm_smem_plan(p.K, E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
+    if (plan.total > GEMM_SMEM_LIMIT) return MOE_ERR_ARG;
+    const long long P = (long long)T * k;
+    const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
+    const long long max_work = (long long)p.MB * max_blocks;
+    int grid = num_sms;
+    if (max_work < grid) grid = (int)(max_work > 0 ? max_work : 1);
+    return launch_expert_gemm(mode, p, grid, plan.total, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int top_k, float eps,
+                                const uint16_t *x, const uint16_t *router_w, const float *router_b,
+                                const uint8_t *w13_codes, const uint8_t *w13_scales, const uint16_t *b13,
+                                const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+                                const uint16_t *norm_scale, uint16_t *y, void *stream) {
+    const int d = d_model, F = d_ff, E = n_experts, k = top_k;
+    if (T < 0 || T > MOE_NOALLOC_MAX_TOKENS) return MOE_ERR_ARG;
+    if (d < 64 || d > 6144 || d % 64 || F < 64 || F > 6144 || F % 64) return MOE_ERR_ARG;
+    if (E < 1 || E > 256 || k < 1 || k > 8 || k > E || !(eps >= 0.0f)) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!a16(x) || !a16(router_w) || !a16(router_b) || !a16(w13_codes) || !a16(w13_scales) || !a16(b13) ||
+        !a16(w2_codes) || !a16(w2_scales) || !a16(b2) || !a16(norm_scale) || !a16(y) || y == x)
+        return MOE_ERR_ARG;
+
+    // carve the scratch; reject shapes that do not fit
+    const size_t P = (size_t)T * k;
+    const size_t sizes[] = {(size_t)T * d * 2, (size_t)T * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
+                            (size_t)(E + 1) * 4, P * 4, P * 4, P * 4, P * d * 2, P * F * 2, P * d * 4, 64};
+    size_t total = 0;
+    for (size_t v : sizes) total += r256(v);
+    if (total > kScratchBytes) return MOE_ERR_ARG;
+
+    unsigned char *base = nullptr;
+    int num_sms = 0;
+    int rc = scratch_for_current_device(&base, &num_sms);
+    if (rc) return rc;
+    unsigned char *ptrs[sizeof(sizes) / sizeof(sizes[0])];
+    for (size_t i = 0; i < sizeof(sizes) / sizeof(sizes[0]); ++i) {
+        ptrs[i] = base;
+        base += r256(sizes[i]);
+    }
+    __half *xn16 = reinterpret_cast<__half *>(ptrs[0]);
+    float *rho = reinterpret_cast<float *>(ptrs[1]);
+    int *topk_idx = reinterpret_cast<int *>(ptrs[2]);
+    float *topk_w = reinterpret_cast<float *>(ptrs[3]);
+    int *counts = reinterpret_cast<int *>(ptrs[4]);
+    int *offsets = reinterpret_cast<int *>(ptrs[5]);
+    int *tiles = reinterpret_cast<int *>(ptrs[6]);
+    int *row_token = reinterpret_cast<int *>(ptrs[7]);
+    float *row_w = reinterpret_cast<float *>(ptrs[8]);
+    int *pair_row = reinterpret_cast<int *>(ptrs[9]);
+    __half *xperm = reinterpret_cast<__half *>(ptrs[10]);
+    __half *h = reinterpret_cast<__half *>(ptrs[11]);
+    float *orows = reinterpret_cast<float *>(ptrs[12]);
+    unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[13]);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nb = token_rows(T);
+    const int box = nb < 64 ? nb : 64;
+    CUtensorMap map_xperm, map_h;
+    if (!enc_rows(&map_xperm, xperm, (int)P, d, box) || !enc_rows(&map_h, h, (int)P, F, box)) return MOE_ERR_CUDA;
+    // the error word is the one buffer that must start at zero on every call
+    if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    RouteParams rp;
+    rp.x = x;
+    rp.norm_scale = norm_scale;
+    rp.router_w = router_w;
+    rp.router_b = router_b;
+    rp.T = T;
+    rp.d = d;
+    rp.E = E;
+    rp.k = k;
+    rp.eps = eps;
+    rp.xn16 = xn16;
+    rp.rho = rho;
+    rp.topk_idx = topk_idx;
+    rp.topk_w = topk_w;
+    if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    GroupParams gp;
+    gp.topk_idx = topk_idx;
+    gp.topk_w = topk_w;
+    gp.P = (int)P;
+    gp.k = k;
+    gp.E = E;
+    gp.nb_rows = nb;
+    gp.counts = counts;
+    gp.offsets = offsets;
+    gp.tiles = tiles;
+    gp.row_token = row_token;
+    gp.row_w = row_w;
+    gp.pair_row = pair_row;
+    gp.err = err;
+    if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_permute(xn16, row_token, xperm, (int)P, d, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xperm, counts,
+                           offsets, tiles, row_token, row_w, rho, h, err, s);
+    if (rc) return rc;
+    rc = launch_gemm_stage(MODE_DOWN, T, k, d, F, E, num_sms, w2_codes, w2_scales, b2, &map_h, counts, offsets,
+                           tiles, row_token, row_w, rho, orows, err, s);
+    if (rc) return rc;
+    return launch_combine(x, orows, pair_row, y, T, d, k, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"
