@@ -173,6 +173,30 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ----------------------------------------------------------- replica plumbing
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank takes part in the same all-reduce."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(ms_total: float, tokens_per_rank: int, steps: int, world: int) -> float:
+    """Whole-job throughput: the tokens every replica processed over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_total / 1e3)
+
+
+def replica_tokens(cfg, rank: int):
+    """Rank r's token batch: rank 0 uses the workload's own tokens, other ranks their own seed."""
+    seed = cfg.seed if rank == 0 else cfg.seed + 1000 * rank
+    return make_tokens(np.random.Generator(np.random.PCG64(seed)), cfg.T, cfg.d)
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def algorithmic_counts(cfg, counts):
@@ -214,9 +238,7 @@ def run_ours(args, rank, world, local_rank):
         layer_inputs = [inp]
     else:
         layer_inputs = [make_config_inputs(cfg, l) for l in range(layers)]
-    x_np = make_tokens(np.random.Generator(np.random.PCG64(cfg.seed + 1000 * rank)), T, cfg.d) if rank else (
-        layer_inputs[0]["x"] if layers == 1 else make_tokens(np.random.Generator(np.random.PCG64(cfg.seed)), T,
-                                                             cfg.d))
+    x_np = replica_tokens(cfg, rank)
     weights = [moe.MoEWeights.from_numpy(li, device=dev) for li in layer_inputs]
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     m = moe.MoE(T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps)
@@ -250,13 +272,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1e3)
+    value = job_tokens_per_s(ms_total, T, args.steps, world)
     if m.sync_status() != moe.MOE_OK:
         raise RuntimeError("device-side error during the timed region")
 
@@ -308,12 +326,8 @@ def run_ours(args, rank, world, local_rank):
             y_host.copy_(cur, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_tokens_per_s(e2e_ms, T, args.steps, world)
 
     if rank != 0:
         m.close()
