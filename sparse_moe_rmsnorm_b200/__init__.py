@@ -312,7 +312,7 @@ class MoE:
             "row_token": ((P,), torch.int32), "row_w": ((P,), torch.float32),
             "h": ((P, s.d_ff), torch.float16), "out_rows": ((P, s.d_model), torch.float32),
             "tiles": ((s.n_experts + 1,), torch.int32), "pair_row": ((P,), torch.int32),
-            "xperm": ((P, s.d_model), torch.float16),
+            "xperm": ((P, s.d_model), torch.float16),     # K-blocked [d/64][P_max][64] when T == T_max
         }[name]
         out = torch.empty(spec[0], dtype=spec[1], device="cuda")
         moe_copy_workspace(self.ctx, WS[name], out, out.numel() * out.element_size(), stream)

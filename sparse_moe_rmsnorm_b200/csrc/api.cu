@@ -10,12 +10,14 @@
 #include <new>
 
 #include "moe_b200.h"
+#include "host_plan.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s);
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
+                           cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
@@ -26,48 +28,6 @@ cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem
 using namespace moe;
 
 namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// u8 codes [E][R][K/2]: box {128 bytes, box_rows, 1}, 128-byte swizzle, zero fill out of range.
-bool encode_codes(CUtensorMap *m, const void *codes, int E, int R, int K, int box_rows) {
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)R, (cuuint64_t)E};
-    const cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R * (K / 2)};
-    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// fp16 [rows][cols]: box {64, box_rows}, 128-byte swizzle.
-bool encode_f16_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -94,8 +54,9 @@ struct moe_ctx {
     float *orows;           // weighted expert output per expert-sorted row
     unsigned int *err;
     unsigned long long wait_limit_ns;
-    CUtensorMap map_xperm[4];  // boxes of 16/32/48/64 rows of the expert-sorted normalised tokens
-    CUtensorMap map_h[4];      // boxes of 16/32/48/64 rows of h
+    // 3-D boxes of the K-blocked expert-sorted tokens and h: [box rows 16/32/48/64][1 or 4 K blocks]
+    CUtensorMap map_xperm[4][2];
+    CUtensorMap map_h[4][2];
     const void *w13_ptr;
     CUtensorMap map_w13;
     const void *w2_ptr;
@@ -139,80 +100,35 @@ int check_call(moe_ctx *c, int T, int top_k) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Token rows per GEMM work item: the smallest multiple of 16 that holds every
-// token (an expert receives each token at most once), capped at 256.
-int token_block_rows(int T) {
-    int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;
-    return nb < 256 ? nb : 256;
-}
-
-// Rows per B TMA box: the whole token block up to 64 rows (a TMA instruction
-// costs its issuing thread ~100+ cycles, so fewer, larger boxes).
-int b_box_rows(int nb_rows) { return nb_rows < 64 ? nb_rows : 64; }
-
 int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
                 const uint16_t *bias, cudaStream_t stream) {
     const moe_shape_t &s = c->shape;
     GemmParams p;
     memset(&p, 0, sizeof p);
     const int E = s.n_experts, d = s.d_model, F = s.d_ff;
-    p.nb_rows = token_block_rows(T);
+    int grid = 0, smem = 0;
+    int rc = plan_gemm(p, mode, T, top_k, d, F, E, s.T_max * s.top_k, c->num_sms, &grid, &smem);
+    if (rc) return rc;
+    const int bi = p.b_box_rows / 16 - 1, bu = p.b_unit == 4 ? 1 : 0;
     if (mode == MODE_UP) {
         if (codes != c->w13_ptr) {
             if (!encode_codes(&c->map_w13, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
             c->w13_ptr = codes;
         }
         p.map_codes = c->map_w13;
-        p.b_box_rows = b_box_rows(p.nb_rows);
-        p.map_b = c->map_xperm[p.b_box_rows / 16 - 1];
-        p.K = d;
-        p.R = 2 * F;
-        p.MB = F / 64;
+        p.map_b = c->map_xperm[bi][bu];
         p.out = c->h;
-        p.out_ld = F;
     } else {
         if (codes != c->w2_ptr) {
             if (!encode_codes(&c->map_w2, codes, E, d, F, 128)) return MOE_ERR_CUDA;
             c->w2_ptr = codes;
         }
         p.map_codes = c->map_w2;
-        p.b_box_rows = b_box_rows(p.nb_rows);
-        p.map_b = c->map_h[p.b_box_rows / 16 - 1];
-        p.K = F;
-        p.R = d;
-        p.MB = (d + GEMM_BM - 1) / GEMM_BM;
+        p.map_b = c->map_h[bi][bu];
         p.out = c->orows;
-        p.out_ld = d;
     }
     p.scales = scales;
     p.bias = bias;
-    p.F = F;
-    p.E = E;
-    p.b_stage_bytes = (p.nb_rows + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows * 128;
-    // MMA warps: a tcgen05.mma holds its issuing thread ~120 cycles, so small
-    // token blocks use up to three issuers (each its own accumulator)
-    const int n_sub = p.K / GEMM_KA;
-    int ni = 256 / p.nb_rows;
-    if (ni > GEMM_ISS_MAX) ni = GEMM_ISS_MAX;
-    if (ni > n_sub) ni = n_sub;
-    if (ni < 1) ni = 1;
-    p.n_iss = ni;
-    p.n_d_bufs = (2 * ni * p.nb_rows <= 256) ? 2 : 1;
-    // TMEM: A slots first, then the accumulators
-    p.n_a_slots = (512 - p.n_d_bufs * ni * p.nb_rows) / 32;
-    if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
-    p.n_a_slots &= ~1;
-    // shared memory: up to 8 code stages next to a B ring of at least 3 stages
-    // (up to 16); whatever is left goes to the code ring
-    const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, p.b_stage_bytes);
-    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 16);
-    int nbs = 16, sc = 8;
-    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && nbs > 3) --nbs;
-    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && sc > 4) --sc;
-    while ((sc + 1) * GEMM_CODE_STAGE + nbs * p.b_stage_bytes <= room && sc < GEMM_SC_MAX) ++sc;
-    if (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room) return MOE_ERR_ARG;
-    p.n_b_stages = nbs;
-    p.n_c_stages = sc;
     p.counts = c->counts;
     p.offsets = c->offsets;
     p.tiles = c->tiles;
@@ -221,14 +137,7 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     p.rho = c->rho;
     p.err = c->err;
     p.wait_limit_ns = c->wait_limit_ns;
-    const GemmSmem plan = gemm_smem_plan(p.K, E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
-    if (plan.total > GEMM_SMEM_LIMIT) return MOE_ERR_ARG;
-    const long long P = (long long)T * top_k;
-    const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
-    long long max_work = (long long)p.MB * max_blocks;
-    int grid = c->num_sms;
-    if (max_work < grid) grid = (int)(max_work > 0 ? max_work : 1);
-    return cuda_status(launch_expert_gemm(mode, p, grid, plan.total, stream));
+    return cuda_status(launch_expert_gemm(mode, p, grid, smem, stream));
 }
 
 }  // namespace
@@ -299,8 +208,9 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
     }
     bool maps_ok = cudaMemset(c->ws, 0, total) == cudaSuccess;
     for (int i = 0; i < 4 && maps_ok; ++i)
-        maps_ok = encode_f16_rows(&c->map_xperm[i], c->xperm, (int)P, s.d_model, 16 * (i + 1)) &&
-                  encode_f16_rows(&c->map_h[i], c->h, (int)P, s.d_ff, 16 * (i + 1));
+        for (int u = 0; u < 2 && maps_ok; ++u)
+            maps_ok = encode_f16_blocked(&c->map_xperm[i][u], c->xperm, (int)P, s.d_model, 16 * (i + 1), u ? 4 : 1) &&
+                      encode_f16_blocked(&c->map_h[i][u], c->h, (int)P, s.d_ff, 16 * (i + 1), u ? 4 : 1);
     if (!maps_ok) {
         cudaFree(c->ws);
         delete c;
@@ -362,7 +272,8 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int rc2 = cuda_status(launch_group(p, st));
     if (rc2) return rc2;
-    return cuda_status(launch_permute(c->xn16, c->row_token, c->xperm, p.P, c->shape.d_model, st));
+    return cuda_status(
+        launch_permute(c->xn16, c->row_token, c->xperm, p.P, c->shape.T_max * c->shape.top_k, c->shape.d_model, st));
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,

@@ -28,9 +28,11 @@
 //
 // Warp roles (672 threads): 0 codes/scales producer, 20 B producer (TMA
 // instructions hold their issuing thread too, so the two streams get their
-// own threads), 1-3 MMA issue (3 also allocates TMEM), 4-7 and 12-15 two
-// decoder groups (alternate two-sub-stage chunks), 8-11 and 16-19 two
-// epilogue groups (alternate 16-column chunks).  The decoders hand each row's power-of-two shift to the
+// own threads), 1-3 MMA issue (3 also allocates TMEM), 4-7 and 12-15
+// decoder groups, 8-11 epilogue group; warps 16-19 are a third decoder group
+// for small token blocks (several MMA warps) and a second epilogue group
+// otherwise.  Decoder groups take two-sub-stage chunks in turn; epilogue
+// groups take 16-column chunks in turn.  The decoders hand each row's power-of-two shift to the
 // epilogue through shared memory.  Every mbarrier wait is bounded (WaitCtl);
 // when one runs out the CTA stops issuing work, drains its copies and MMAs in
 // flight, frees TMEM and returns with the error latched.
@@ -79,6 +81,23 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n_slots, long lon
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+// Largest and smallest E8M0 byte of a row (255 excluded from the largest; a
+// 255 makes the smallest -1), n even, row 2-byte aligned.
+__device__ __forceinline__ void row_scale_range(const uint8_t *s, int n, int &mx, int &mn) {
+    const uint16_t *w = reinterpret_cast<const uint16_t *>(s);
+    mx = -1;
+    mn = 256;
+#pragma unroll 8
+    for (int b = 0; b < n / 2; ++b) {
+        const uint32_t v = w[b];
+        const int lo = (int)(v & 0xFFu), hi = (int)(v >> 8);
+        mx = max(mx, lo == 255 ? -1 : lo);
+        mx = max(mx, hi == 255 ? -1 : hi);
+        mn = min(mn, lo == 255 ? -1 : lo);
+        mn = min(mn, hi == 255 ? -1 : hi);
+    }
+}
+
 // Largest E8M0 byte (other than 255) of a row's n scale bytes (n even, row
 // 2-byte aligned), read as 16-bit words so the loads pipeline.
 __device__ __forceinline__ int row_scale_max(const uint8_t *s, int n) {
@@ -98,8 +117,17 @@ template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const GemmSmem plan = gemm_smem_plan(p.K, p.E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
+    const int U = p.b_unit;
+    const int b_slot_bytes = U * p.b_stage_bytes;
+    const GemmSmem plan = gemm_smem_plan(p.K, p.E, p.n_c_stages, p.n_a_slots, p.n_b_stages, b_slot_bytes);
     const int SC = p.n_c_stages, NA = p.n_a_slots, NBS = p.n_b_stages, NI = p.n_iss;
+    const int NP = NA / 2;                 // A slot pairs: one pair per decoder chunk of two sub-stages
+    const int NG = p.n_dec_groups;         // decoder groups
+    const int NEG = NG == 3 ? 1 : 2;       // epilogue groups
+    const int PPG = NP / NG;               // slot pairs owned by each decoder group
+    // Chunk gc (two sub-stages of a code stage) is decoded by group gc % NG into
+    // the group's pair (gc / NG) % PPG and its MMAs are issued by MMA warp
+    // (gc % NG) % NI, so each decoder group and its MMA warp form one pipeline.
     uint8_t *code_ring = smem + plan.code_off;
     uint8_t *b_ring = smem + plan.b_off;
     uint8_t *scale_buf = smem + plan.scale_off;
@@ -135,23 +163,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     if (threadIdx.x == 0) {
         for (int i = 0; i < SC; ++i) {
             mbar_init(&c_full[i], 1);
-            mbar_init(&c_empty[i], 8);     // both decoder groups
+            mbar_init(&c_empty[i], 4 * NG);   // every decoder warp
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 8);
-            mbar_init(&d_full[i], NI);     // one commit per MMA warp
-            mbar_init(&d_empty[i], 8);     // both epilogue groups
+            mbar_init(&s_empty[i], 4 * NG);
+            mbar_init(&d_full[i], NI);        // one commit per MMA warp
+            mbar_init(&d_empty[i], 4 * NEG);  // every epilogue warp
             mbar_init(&h_full[i], 4);
-            mbar_init(&h_empty[i], 8);
+            mbar_init(&h_empty[i], 4 * NEG);
         }
-        for (int i = 0; i < NA; ++i) {
-            mbar_init(&a_full[i], 4);      // the four warps of the group that decoded the slot
-            mbar_init(&a_empty[i], 1);
+        for (int i = 0; i < NP; ++i) {
+            mbar_init(&a_full[i], 4);         // the four warps of the group that decoded the pair
+            mbar_init(&a_empty[i], 1);        // the commit of the MMA warp that consumed it
         }
         for (int i = 0; i < NBS; ++i) {
             mbar_init(&b_full[i], 1);
-            mbar_init(&b_empty[i], 1);
+            mbar_init(&b_empty[i], U);     // one commit per sub-stage of the slot
         }
         for (int i = 0; i < GEMM_ISS_MAX; ++i) mbar_init(&drain_bar[i], 1);
         *abort_s = 0;
@@ -224,6 +252,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
     } else if (warp == 20) {
         // ------------------------------------------------------------ B producer
+        // One slot holds U consecutive 64-K blocks of the work item's token
+        // rows; with U = 4 a single 3-D TMA box fills it.
         if (lane == 0) {
             tma_prefetch_desc(&p.map_b);
             int bslot = 0;
@@ -231,16 +261,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             long long b_issued = 0;
             bool ok = true;
             const int box = p.b_box_rows;
+            const int n_units = (n_sub + U - 1) / U;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 Work t;
                 work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
                 const int nbox = (t.n_mma + box - 1) / box;
-                for (int j = 0; j < n_sub; ++j) {
+                for (int u = 0; u < n_units; ++u) {
                     if (!mbar_wait(&b_empty[bslot], bph ^ 1, wc)) { ok = false; break; }
-                    uint8_t *bdst = b_ring + bslot * p.b_stage_bytes;
-                    mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)(nbox * box * 128));
+                    uint8_t *bdst = b_ring + bslot * b_slot_bytes;
+                    mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)(nbox * box * 128 * U));
                     for (int g = 0; g < nbox; ++g)
-                        tma_load_2d(bdst + g * box * 128, &p.map_b, &b_full[bslot], j * GEMM_KA, t.p0 + box * g);
+                        tma_load_3d(bdst + g * box * 128 * U, &p.map_b, &b_full[bslot], 0, t.p0 + box * g, u * U);
+                    // a slot past the last K block is consumed fewer than U times
+                    for (int r = min(U, n_sub - u * U); r < U; ++r) mbar_arrive(&b_empty[bslot]);
                     ++b_issued;
                     if (++bslot == NBS) { bslot = 0; bph ^= 1; }
                 }
@@ -253,35 +286,76 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         if (lane == 0 && mi < NI) {
             int db = 0;
             uint32_t dph = 0;
-            long long g0 = 0;                      // running index of the work item's first sub-stage
+            // Running counters instead of divisions (a 64-bit division is a long
+            // software routine): the decoder group of the next chunk, each
+            // group's next pair and its phase, and the next B fill.
+            int turn = 0;                          // decoder group of the next chunk
+            int pp0 = 0, pp1 = 0, pp2 = 0;         // next pair (within its group) of groups 0..2
+            uint32_t ph0 = 0, ph1 = 0, ph2 = 0;    // phase parity of that pair
+            int ub = 0, bslot = 0;                 // next B fill (within the work item) and its slot
+            uint32_t bph = 0;
+            const int ushift = U == 4 ? 2 : 0;
+            const int n_units = (n_sub + U - 1) / U;
+            const int n_chunks = (n_sub + 1) / 2;  // two per full code stage, ceil(r/2) for a tail of r
             bool ok = true, issued = false;
-            for (int w = blockIdx.x; w < total && ok; w += gridDim.x, g0 += n_sub) {
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 Work t;
                 work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
                 const uint32_t idesc = idesc_f16_f32(GEMM_BM, (uint32_t)t.n_mma);
                 if (!mbar_wait(&d_empty[db], dph ^ 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + d_col0 + (uint32_t)((db * NI + mi) * p.nb_rows);
-                for (int j = mi; j < n_sub; j += NI) {
-                    const long long g = g0 + j;
-                    const int aslot = (int)(g % NA), bslot = (int)(g % NBS);
-                    if (!mbar_wait(&a_full[aslot], (uint32_t)((g / NA) & 1), wc) ||
-                        !mbar_wait(&b_full[bslot], (uint32_t)((g / NBS) & 1), wc)) {
-                        ok = false;
-                        break;
+                bool first = true;
+                int u_base = 0;                    // B fills consumed before this work item, relative
+                for (int ci = 0; ci < n_chunks && ok; ++ci) {
+                    const int grp = turn;
+                    turn = turn + 1 == NG ? 0 : turn + 1;
+                    const int lp = grp == 0 ? pp0 : (grp == 1 ? pp1 : pp2);
+                    const uint32_t lph = grp == 0 ? ph0 : (grp == 1 ? ph1 : ph2);
+                    {
+                        int np_ = lp + 1;
+                        uint32_t nph = lph;
+                        if (np_ == PPG) { np_ = 0; nph ^= 1; }
+                        if (grp == 0) { pp0 = np_; ph0 = nph; } else if (grp == 1) { pp1 = np_; ph1 = nph; } else { pp2 = np_; ph2 = nph; }
                     }
-                    tc_fence_after();
-                    const uint32_t b_addr = smem_addr(b_ring + bslot * p.b_stage_bytes);
-                    const uint32_t a_tmem = tmem + (uint32_t)(aslot * 32);
+                    if (grp % NI != mi) continue;
+                    const int pair = grp * PPG + lp;
+                    if (!mbar_wait(&a_full[pair], lph, wc)) { ok = false; break; }
+                    // sub-stages of chunk ci: 2 per code stage, the tail stage may hold 1..4
+                    const int j0 = 4 * (ci >> 1) + 2 * (ci & 1);
+                    const int na = min(2, n_sub - j0);
+                    for (int u = 0; u < na; ++u) {
+                        const int j = j0 + u;
+                        const int target = j >> ushift;        // B fill of sub-stage j within the work item
+                        while (ub < u_base + target) {
+                            ++ub;
+                            if (++bslot == NBS) { bslot = 0; bph ^= 1; }
+                        }
+                        if (!mbar_wait(&b_full[bslot], bph, wc)) { ok = false; break; }
+                        tc_fence_after();
+                        // sub-stage block j % U of the slot
+                        const uint32_t b_addr =
+                            smem_addr(b_ring + bslot * b_slot_bytes + (j & (U - 1)) * p.b_stage_bytes);
+                        const uint32_t a_tmem = tmem + (uint32_t)((2 * pair + u) * 32);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
-                                   (j != mi || kk != 0) ? 1u : 0u);
-                    issued = true;
-                    mma_commit(&a_empty[aslot]);
-                    mma_commit(&b_empty[bslot]);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            mma_f16_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
+                                       first ? 0u : 1u);
+                            first = false;
+                        }
+                        issued = true;
+                        mma_commit(&b_empty[bslot]);
+                    }
+                    if (!ok) break;
+                    mma_commit(&a_empty[pair]);
                 }
                 if (!ok) break;
+                // move the B counters to the first fill of the next work item
+                while (ub < u_base + n_units) {
+                    ++ub;
+                    if (++bslot == NBS) { bslot = 0; bph ^= 1; }
+                }
+                ub -= u_base + n_units;
                 mma_commit(&d_full[db]);
                 if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
             }
@@ -290,21 +364,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 mbar_wait_drain(&drain_bar[mi], 0, p.wait_limit_ns);
             }
         }
-    } else if ((warp >= 4 && warp < 8) || (warp >= 12 && warp < 16)) {
+    } else if ((warp >= 4 && warp < 8) || (warp >= 12 && warp < 16 && NG >= 2) || (warp >= 16 && warp < 20 && NG == 3)) {
         // ------------------------------------------------------------ decoders
-        // Two groups of four warps.  Each code stage (4 sub-stages of 64 K
-        // elements) is cut into chunks of two sub-stages; group g decodes the
-        // chunks whose running index is congruent to g modulo 2, writing TMEM
-        // lanes 32q..32q+31 of the chunk's A slots, with one handshake per chunk.
+        // NG groups of four warps.  Each code stage (4 sub-stages of 64 K
+        // elements) is cut into chunks of two sub-stages; chunk gc goes to
+        // group gc mod NG and fills one of the group's own A slot pairs (TMEM
+        // lanes 32q..32q+31 of its warps), with one handshake per chunk.
         const int q = warp & 3;
-        const int grp = warp >= 12 ? 1 : 0;
+        const int grp = warp < 8 ? 0 : (warp < 16 ? 1 : 2);
         const int tl = 32 * q + lane;                           // TMEM lane = A row
         const int my_row = MODE == MODE_UP ? (16 * q + (lane & 15) + (lane >= 16 ? 64 : 0)) : tl;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int cslot = 0, sb = 0, hb = 0;
         uint32_t cph = 0, sph = 0, hph = 0;
-        long long sub_idx = 0;                                  // running sub-stage index (A slot sequence)
-        long long chunk_idx = 0;                                // running chunk index
+        int turn = 0;                                           // decoder group of the next chunk
+        int mpair = 0;                                          // this group's next pair (within the group)
+        uint32_t mph = 0;                                       // and its phase parity
         bool ok = true;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
@@ -312,7 +387,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             const bool row_valid = MODE == MODE_UP || (t.mb * GEMM_BM + my_row < p.R);
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
             const uint8_t *srow = scale_buf + sb * scale_bytes + my_row * KB32;
-            const int c = row_shift_from_max(row_valid ? row_scale_max(srow, KB32) : -1);
+            int smax = -1, smin = 256;
+            if (row_valid) row_scale_range(srow, KB32, smax, smin);
+            const int c = row_shift_from_max(smax);
+            const bool fast = row_valid && smin >= smax - 27;   // every block multiplier is a normal fp16
             if (grp == 0) {
                 // hand the row shift to the epilogue
                 if (!__all_sync(0xffffffffu, mbar_wait(&h_empty[hb], hph ^ 1, wc))) { ok = false; break; }
@@ -325,49 +403,68 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 if (!__all_sync(0xffffffffu, mbar_wait(&c_full[cslot], cph, wc))) { ok = false; break; }
                 const uint8_t *crow = code_ring + cslot * GEMM_CODE_STAGE + my_row * 128;
                 const int nsub = min(4, (p.K - ks * GEMM_KS) / GEMM_KA);
-                for (int a0 = 0; a0 < nsub; a0 += 2) {
-                    const int na = min(2, nsub - a0);
-                    const bool mine = (int)(chunk_idx & 1) == grp;
-                    const long long first = sub_idx;
-                    sub_idx += na;
-                    ++chunk_idx;
-                    if (!mine) continue;
-                    bool okc = true;
-                    for (int u = 0; u < na; ++u) {
-                        const long long si = first + u;
-                        okc = okc && mbar_wait(&a_empty[(int)(si % NA)], (uint32_t)(((si / NA) & 1) ^ 1), wc);
+                // the 8 block multipliers of this code stage
+                uint32_t mult[8];
+                {
+                    const uint16_t *sw16 = reinterpret_cast<const uint16_t *>(srow + ks * 8);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t v = (2 * i < 2 * nsub) ? (uint32_t)sw16[i] : 0x7F7Fu;
+                        const int s0 = (int)(v & 0xFFu), s1 = (int)(v >> 8);
+                        if (fast) {
+                            mult[2 * i] = block_multiplier_fast(s0, smax);
+                            mult[2 * i + 1] = block_multiplier_fast(s1, smax);
+                        } else {
+                            mult[2 * i] = block_multiplier(s0, c);
+                            mult[2 * i + 1] = block_multiplier(s1, c);
+                        }
                     }
-                    if (!__all_sync(0xffffffffu, okc)) { ok = false; break; }
+                }
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int a0 = 2 * cc;
+                    if (a0 >= nsub) break;
+                    const int na = min(2, nsub - a0);
+                    const bool mine = turn == grp;
+                    turn = turn + 1 == NG ? 0 : turn + 1;
+                    if (!mine) continue;
+                    const int pair = grp * PPG + mpair;
+                    const uint32_t pph = mph;
+                    if (++mpair == PPG) { mpair = 0; mph ^= 1; }
+                    if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[pair], pph ^ 1, wc))) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const int sw = my_row & 7;
-                    for (int u = 0; u < na; ++u) {
-                        const int a = a0 + u;
-                        uint32_t out[32];
-                        if (row_valid) {
-                            const uint4 w0 = *reinterpret_cast<const uint4 *>(crow + (((2 * a) ^ sw) << 4));
-                            const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + (((2 * a + 1) ^ sw) << 4));
-                            const int kb = (ks * GEMM_KS + a * GEMM_KA) / 32;
-                            const uint32_t m0 = block_multiplier(srow[kb], c);
-                            const uint32_t m1 = block_multiplier(srow[kb + 1], c);
-                            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                uint32_t h4[4];
-                                e2m1x8_to_half2x4(words[i], h4);
+                    for (int u = 0; u < 2; ++u) {
+                        if (u < na) {
+                            const int a = a0 + u;
+                            uint32_t out[32];
+                            if (row_valid) {
+                                const uint4 w0 = *reinterpret_cast<const uint4 *>(crow + (((2 * a) ^ sw) << 4));
+                                const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + (((2 * a + 1) ^ sw) << 4));
+                                const uint32_t m0 = mult[2 * a], m1 = mult[2 * a + 1];
+                                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                                for (int jj = 0; jj < 4; ++jj) out[4 * i + jj] = hmul2_u32(h4[jj], i < 4 ? m0 : m1);
+                                for (int i = 0; i < 8; ++i) {
+                                    uint32_t h4[4];
+                                    e2m1x8_to_half2x4(words[i], h4);
+#pragma unroll
+                                    for (int jj = 0; jj < 4; ++jj) out[4 * i + jj] = hmul2_u32(h4[jj], i < 4 ? m0 : m1);
+                                }
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) out[i] = 0u;
                             }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) out[i] = 0u;
+                            tmem_st32(lane_base + (uint32_t)((2 * pair + u) * 32), out);
                         }
-                        tmem_st32(lane_base + (uint32_t)((int)((first + u) % NA) * 32), out);
                     }
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0)
-                        for (int u = 0; u < na; ++u) mbar_arrive(&a_full[(int)((first + u) % NA)]);
+                    if (lane == 0) mbar_arrive(&a_full[pair]);
                 }
                 if (!ok) break;
                 __syncwarp();
@@ -379,7 +476,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (lane == 0) mbar_arrive(&s_empty[sb]);
             if (++sb == 2) { sb = 0; sph ^= 1; }
         }
-    } else if ((warp >= 8 && warp < 12) || (warp >= 16 && warp < 20)) {
+    } else if ((warp >= 8 && warp < 12) || (warp >= 16 && warp < 20 && NG < 3)) {
         // ------------------------------------------------------------- epilogue
         // Two groups of four warps; group eg takes the 16-column chunks
         // eg, eg+2, eg+4, ... of the accumulators, summing the MMA warps' parts.
@@ -405,7 +502,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + row]) : 0.f;
             // per-column rho (UP) or routing weight (DOWN) of this group's columns
             for (int cc = lane; cc < GEMM_NB_MAX / 2; cc += 32) {
-                const int col = ((cc >> 4) * 2 + eg) * 16 + (cc & 15);
+                const int col = ((cc >> 4) * NEG + eg) * 16 + (cc & 15);
                 if (col < t.n_mma) {
                     const int pr = t.p0 + min(col, t.n_valid - 1);
                     mval[cc] = MODE == MODE_UP ? p.rho[p.row_token[pr]] : p.row_w[pr];
@@ -420,7 +517,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
             tc_fence_after();
             const uint32_t d_tmem = lane_base + d_col0 + (uint32_t)(db * NI * p.nb_rows);
-            for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
+            for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 16 * NEG) {
                 float acc[16];
                 {
                     uint32_t v[16];
@@ -436,7 +533,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
                 }
-                const float *mv = mval + (c0 >> 5) * 16;
+                const float *mv = mval + (c0 / (16 * NEG)) * 16;
                 if (MODE == MODE_UP) {
                     float z[16];
 #pragma unroll
@@ -453,7 +550,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         const float g = fminf(gate, 7.0f);
                         const float u = fminf(fmaxf(lin, -7.0f), 7.0f);
                         const float h = __fdividef(g, 1.0f + __expf(-1.702f * g)) * (u + 1.0f);
-                        if (col < t.n_valid) hout[(size_t)(t.p0 + col) * p.out_ld + jrow] = __float2half_rn(h);
+                        if (col < t.n_valid)
+                            hout[((size_t)t.mb * p.b_rows_total + t.p0 + col) * 64 + (jrow - t.mb * 64)] =
+                                __float2half_rn(h);
                     }
                 } else {
                     // weighted expert output w * (W2 h + b2), one expert-sorted row per column

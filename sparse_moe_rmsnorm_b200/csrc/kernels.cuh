@@ -50,7 +50,7 @@ enum { MODE_UP = 0, MODE_DOWN = 1 };
 
 struct GemmParams {
     CUtensorMap map_codes;      // u8 [E][R][K/2], box {128 bytes, 64 (UP) or 128 (DOWN) rows, 1}, 128B swizzle
-    CUtensorMap map_b;          // fp16 expert-sorted B rows [P][K], box {64 elements, b_box_rows rows}
+    CUtensorMap map_b;          // fp16 expert-sorted B, K-blocked [K/64][P_max][64]; 3-D box {64, b_box_rows, b_unit}
     const uint8_t *scales;      // u8 [E][R][K/32]
     const uint16_t *bias;       // bf16 [E][R]
     int K;                      // reduction length
@@ -59,12 +59,15 @@ struct GemmParams {
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= 256)
-    int b_box_rows;             // rows per B TMA box (16..64); a B stage holds round_up(nb_rows, b_box_rows) rows
-    int n_b_stages;             // B ring depth
-    int b_stage_bytes;          // nb_rows * 128
+    int b_box_rows;             // rows per B TMA box (16..64)
+    int b_unit;                 // sub-stages (64-K blocks) per B ring slot: 4 when one box holds the token block, else 1
+    int n_b_stages;             // B ring depth (slots)
+    int b_stage_bytes;          // bytes of one sub-stage block in a slot: round_up(nb_rows, b_box_rows) * 128
+    int b_rows_total;           // P_max: rows of the K-blocked B and h buffers
     int n_c_stages;             // code ring depth (shared-memory stages of 128 rows x 128 bytes)
     int n_a_slots;              // TMEM A slots (32 columns each); accumulators follow them
     int n_iss;                  // MMA-issuing warps, each with its own accumulator
+    int n_dec_groups;           // decoder warp groups, 1..3 (with 3, warps 16-19 decode and one epilogue group remains)
     int n_d_bufs;               // accumulator buffer sets (1 or 2)
     const int *counts, *offsets, *tiles;
     const int *row_token;       // [P]
@@ -100,12 +103,13 @@ __host__ __device__ inline int gemm_num_barriers(int n_c_stages, int n_a_slots, 
     return 2 * n_c_stages + 4 + 2 * n_a_slots + 2 * n_b_stages + 4 + 4 + GEMM_ISS_MAX;
 }
 
+// b_slot_bytes = b_unit * b_stage_bytes
 __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int n_c_stages, int n_a_slots, int n_b_stages,
-                                                    int b_stage_bytes) {
+                                                    int b_slot_bytes) {
     GemmSmem s;
     s.code_off = 0;
     s.b_off = n_c_stages * GEMM_CODE_STAGE;
-    s.scale_off = s.b_off + n_b_stages * b_stage_bytes;
+    s.scale_off = s.b_off + n_b_stages * b_slot_bytes;
     const int scale_bytes = align_up(GEMM_BM * (K / 32), 128);
     s.meta_off = s.scale_off + 2 * scale_bytes;
     s.tok_off = s.meta_off + 8 * (GEMM_NB_MAX / 2) * 4;         // per epilogue warp: one value per its columns

@@ -22,13 +22,15 @@
 #include <cstring>
 #include <mutex>
 
+#include "host_plan.cuh"
 #include "kernels.cuh"
 #include "moe_b200.h"
 
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s);
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
+                           cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
@@ -47,46 +49,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 unsigned char *g_scratch_ptr[kMaxDevices];   // device address of g_noalloc_scratch, per device
 int g_num_sms[kMaxDevices];
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn noalloc_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-bool enc_codes(CUtensorMap *m, const void *codes, int E, int R, int K, int box_rows) {
-    EncodeTiledFn f = noalloc_encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)R, (cuuint64_t)E};
-    const cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R * (K / 2)};
-    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool enc_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
-    EncodeTiledFn f = noalloc_encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -111,11 +73,6 @@ int scratch_for_current_device(unsigned char **ptr, int *num_sms) {
     return MOE_OK;
 }
 
-int token_rows(int T) {
-    int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;
-    return nb < 256 ? nb : 256;
-}
-
 // The grouped GEMM launch of one expert stage on scratch-backed buffers.
 int launch_gemm_stage(int mode, int T, int k, int d, int F, int E, int num_sms, const uint8_t *codes,
                       const uint8_t *scales, const uint16_t *bias, const CUtensorMap *map_b, const int *counts,
@@ -123,47 +80,16 @@ int launch_gemm_stage(int mode, int T, int k, int d, int F, int E, int num_sms, 
                       const float *rho, void *out, unsigned int *err, cudaStream_t stream) {
     GemmParams p;
     memset(&p, 0, sizeof p);
-    p.nb_rows = token_rows(T);
-    p.b_box_rows = p.nb_rows < 64 ? p.nb_rows : 64;
+    int grid = 0, smem = 0;
+    int rc = plan_gemm(p, mode, T, k, d, F, E, T * k, num_sms, &grid, &smem);
+    if (rc) return rc;
+    if (!encode_codes(&p.map_codes, codes, E, mode == MODE_UP ? 2 * F : d, mode == MODE_UP ? d : F,
+                      mode == MODE_UP ? 64 : 128))
+        return MOE_ERR_CUDA;
     p.map_b = *map_b;
-    if (mode == MODE_UP) {
-        if (!enc_codes(&p.map_codes, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
-        p.K = d;
-        p.R = 2 * F;
-        p.MB = F / 64;
-        p.out_ld = F;
-    } else {
-        if (!enc_codes(&p.map_codes, codes, E, d, F, 128)) return MOE_ERR_CUDA;
-        p.K = F;
-        p.R = d;
-        p.MB = (d + GEMM_BM - 1) / GEMM_BM;
-        p.out_ld = d;
-    }
     p.out = out;
     p.scales = scales;
     p.bias = bias;
-    p.F = F;
-    p.E = E;
-    p.b_stage_bytes = (p.nb_rows + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows * 128;
-    const int n_sub = p.K / GEMM_KA;
-    int ni = 256 / p.nb_rows;
-    if (ni > GEMM_ISS_MAX) ni = GEMM_ISS_MAX;
-    if (ni > n_sub) ni = n_sub;
-    if (ni < 1) ni = 1;
-    p.n_iss = ni;
-    p.n_d_bufs = (2 * ni * p.nb_rows <= 256) ? 2 : 1;
-    p.n_a_slots = (512 - p.n_d_bufs * ni * p.nb_rows) / 32;
-    if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
-    p.n_a_slots &= ~1;
-    const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, p.b_stage_bytes);
-    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 16);
-    int nbs = 16, sc = 8;
-    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && nbs > 3) --nbs;
-    while (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room && sc > 4) --sc;
-    while ((sc + 1) * GEMM_CODE_STAGE + nbs * p.b_stage_bytes <= room && sc < GEMM_SC_MAX) ++sc;
-    if (sc * GEMM_CODE_STAGE + nbs * p.b_stage_bytes > room) return MOE_ERR_ARG;
-    p.n_b_stages = nbs;
-    p.n_c_stages = sc;
     p.counts = counts;
     p.offsets = offsets;
     p.tiles = tiles;
@@ -172,14 +98,7 @@ int launch_gemm_stage(int mode, int T, int k, int d, int F, int E, int num_sms, 
     p.rho = rho;
     p.err = err;
     p.wait_limit_ns = 2000000000ull;
-    const GemmSmem plan = gemm_smem_plan(p.K, E, p.n_c_stages, p.n_a_slots, p.n_b_stages, p.b_stage_bytes);
-    if (plan.total > GEMM_SMEM_LIMIT) return MOE_ERR_ARG;
-    const long long P = (long long)T * k;
-    const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
-    const long long max_work = (long long)p.MB * max_blocks;
-    int grid = num_sms;
-    if (max_work < grid) grid = (int)(max_work > 0 ? max_work : 1);
-    return launch_expert_gemm(mode, p, grid, plan.total, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_expert_gemm(mode, p, grid, smem, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -233,10 +152,11 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[13]);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int nb = token_rows(T);
-    const int box = nb < 64 ? nb : 64;
+    const int nb = token_block_rows(T);
     CUtensorMap map_xperm, map_h;
-    if (!enc_rows(&map_xperm, xperm, (int)P, d, box) || !enc_rows(&map_h, h, (int)P, F, box)) return MOE_ERR_CUDA;
+    if (!encode_f16_blocked(&map_xperm, xperm, (int)P, d, b_box_rows(nb), b_unit(nb)) ||
+        !encode_f16_blocked(&map_h, h, (int)P, F, b_box_rows(nb), b_unit(nb)))
+        return MOE_ERR_CUDA;
     // the error word is the one buffer that must start at zero on every call
     if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -271,7 +191,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.pair_row = pair_row;
     gp.err = err;
     if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_permute(xn16, row_token, xperm, (int)P, d, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_permute(xn16, row_token, xperm, (int)P, (int)P, d, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xperm, counts,
                            offsets, tiles, row_token, row_w, rho, h, err, s);

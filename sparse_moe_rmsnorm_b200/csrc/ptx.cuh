@@ -247,6 +247,14 @@ __device__ __forceinline__ float exp2i(int e) {
 // of 255 (NaN) are left out of the maximum.
 __device__ __forceinline__ int row_shift_from_max(int smax) { return smax < 0 ? 0 : smax - 140; }
 
+// Fast multiplier for rows whose E8M0 bytes all lie within 27 of the row's
+// largest (and none is 255): 2^(s-127-c) with c = smax - 140 is then a normal
+// fp16 number, bits ((s - smax + 28) << 10), duplicated into both halves.
+__device__ __forceinline__ uint32_t block_multiplier_fast(int s, int smax) {
+    const uint32_t b = (uint32_t)(s - smax + 28) << 10;
+    return b | (b << 16);
+}
+
 // Multiplier of one block (E8M0 byte s) under row shift c, as an fp16 pair:
 // 2^(s-127-c), rounded to fp16 (exact down to 2^-24), NaN for s = 255.
 __device__ __forceinline__ uint32_t block_multiplier(int s, int c) {

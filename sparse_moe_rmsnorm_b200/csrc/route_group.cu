@@ -387,17 +387,20 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
 
 // --------------------------------------------------------------- permute
 //
-// xperm[p] = xn16[row_token[p]]: the normalised tokens in expert-sorted row
-// order, so the gate/up GEMM reads its token blocks as contiguous rows.  One
-// warp per row, 16-byte copies.
+// The normalised tokens in expert-sorted row order, K-blocked:
+// xperm[kb][r][0:64] = xn16[row_token[r]][64 kb : 64 kb + 64] for r < P, with
+// P_max rows per block, so one 3-D TMA box reads several 64-K blocks of a
+// run of rows.  One warp per row, 16-byte copies.
 __global__ void __launch_bounds__(256) permute_kernel(const __half *__restrict__ xn16, const int *__restrict__ row_token,
-                                                      __half *__restrict__ xperm, int P, int d) {
+                                                      __half *__restrict__ xperm, int P, int P_max, int d) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     for (int r = warp; r < P; r += nwarps) {
         const uint4 *src = reinterpret_cast<const uint4 *>(xn16 + (size_t)row_token[r] * d);
-        uint4 *dst = reinterpret_cast<uint4 *>(xperm + (size_t)r * d);
-        for (int j = lane; j < d / 8; j += 32) dst[j] = src[j];
+        for (int j = lane; j < d / 8; j += 32) {
+            const int kb = j >> 3;
+            reinterpret_cast<uint4 *>(xperm + ((size_t)kb * P_max + r) * 64)[j & 7] = src[j];
+        }
     }
 }
 
@@ -508,10 +511,11 @@ cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int d, cudaStream_t s) {
+cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
+                           cudaStream_t s) {
     if (P <= 0) return cudaSuccess;
     const int grid = min((P + 7) / 8, 148 * 8);
-    permute_kernel<<<grid, 256, 0, s>>>(xn16, row_token, xperm, P, d);
+    permute_kernel<<<grid, 256, 0, s>>>(xn16, row_token, xperm, P, P_max, d);
     return cudaGetLastError();
 }
 

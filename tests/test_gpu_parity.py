@@ -165,16 +165,18 @@ def test_group_stage_invariants(T, E, k):
     row_w = m.workspace("row_w", T).cpu().numpy()
     pair_row = m.workspace("pair_row", T).cpu().numpy()
     xn16 = m.workspace("xn16", T).cpu().numpy()
-    xperm = m.workspace("xperm", T).cpu().numpy()
-    assert m.sync_status() == moe.MOE_OK
     P = T * k
+    # the workspace holds it K-blocked: [d/64][T*k][64]
+    dd = xn16.shape[1]
+    xperm = m.workspace("xperm", T).cpu().numpy().reshape(dd // 64, P, 64).transpose(1, 0, 2).reshape(P, dd)
+    assert m.sync_status() == moe.MOE_OK
     # pair_row inverts the permutation, and the sorted token copy follows it
     assert np.array_equal(np.sort(pair_row), np.arange(P))
     assert np.array_equal(row_token[pair_row], np.repeat(np.arange(T), k))
     assert np.array_equal(xperm, xn16[row_token])
     assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
     assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts) and offsets[-1] == P
-    nb = min(256, (T + 15) // 16 * 16)
+    nb = 16 if T <= 64 else min(256, (T + 15) // 16 * 16)
     assert np.array_equal(np.diff(tiles), (counts + nb - 1) // nb)
     # a stable permutation: expert-major, token-minor, every pair exactly once
     want_tok = []
