@@ -24,7 +24,8 @@
  * Conventions
  *   - Every tensor argument is a DEVICE pointer owned by the caller, row-major,
  *     with no padding.  bf16 tensors are passed as uint16_t bit patterns.
- *     Every pointer must be 16-byte aligned.
+ *     Every pointer must be 16-byte aligned, the two code tensors (w13_codes,
+ *     w2_codes) 32-byte aligned (cudaMalloc gives 256).
  *   - Calls are asynchronous on `stream` (a cudaStream_t, may be NULL for the
  *     legacy default stream).  A return value reports argument or launch
  *     errors only; errors raised on the device (a bounded wait that ran out)
@@ -83,8 +84,9 @@ typedef struct moe_ctx moe_ctx_t;
 
 /* Create a context for `shape` on the current CUDA device.  Allocates the
  * device workspace sized for shape->T_max (routing arrays, the fp16 normalised
- * activations, the fp16 SwiGLU output h [T_max*k, F] and the fp32 output
- * accumulator [T_max, d]).  The context owns the workspace; free it with
+ * activations, the expert-sorted activations and the SwiGLU output h in the
+ * two-term E4M3 form the block-scaled expert GEMMs read, and the fp32
+ * weighted expert rows [T_max*k, d]).  The context owns the workspace; free it with
  * moe_destroy.  Returns MOE_ERR_ARG for an invalid shape, MOE_ERR_UNSUPPORTED
  * off B200, MOE_ERR_NOMEM when the workspace does not fit. */
 MOE_API int moe_init(const moe_shape_t *shape, moe_ctx_t **out);
@@ -142,11 +144,17 @@ enum {
     MOE_WS_OFFSETS = 5,  /* int32 [E+1]   exclusive prefix of counts              */
     MOE_WS_ROW_TOKEN = 6,/* int32 [T*k]   token of each expert-sorted row         */
     MOE_WS_ROW_W = 7,    /* fp32 [T*k]    routing weight of each expert-sorted row */
-    MOE_WS_H = 8,        /* fp16 [T*k, F] SwiGLU output, expert-sorted rows       */
+    MOE_WS_H = 8,        /* u8 [2, T_max*k, Kf] SwiGLU output h of the expert-sorted rows as
+                            E4M3 hi (plane 0) and lo (plane 1) terms: h ~ hi 2^s + lo 2^(s-4) with
+                            s the block's scale in MOE_WS_HSF; Kf = d_ff rounded up to 128      */
     MOE_WS_OUT_ROWS = 9, /* fp32 [T*k, d] w * (W2 h + b2), expert-sorted rows      */
     MOE_WS_TILES = 10,   /* int32 [E+1]   exclusive prefix of token blocks        */
     MOE_WS_PAIR_ROW = 11,/* int32 [T*k]   expert-sorted row of pair (token, slot) */
-    MOE_WS_XPERM = 12    /* fp16 [T*k, d] xn16 rows in expert-sorted order         */
+    MOE_WS_XPERM = 12,   /* u8 [2, T_max*k, Kd] normalised tokens in expert-sorted order, E4M3
+                            hi and lo planes as MOE_WS_H; Kd = d_model rounded up to 128      */
+    MOE_WS_XSF = 13,     /* u32 [Kd/128, 2, T_max*k] E8M0 scales of MOE_WS_XPERM: word (g, plane,
+                            row), byte i = the scale of 32-block 4g+i                          */
+    MOE_WS_HSF = 14      /* u32 [Kf/128, 2, T_max*k] E8M0 scales of MOE_WS_H, same layout      */
 };
 
 /* Copy `bytes` bytes of workspace buffer `which` (a MOE_WS_* value) into
@@ -171,10 +179,10 @@ MOE_API int moe_set_wait_limit_ns(moe_ctx_t *ctx, unsigned long long ns);
 MOE_API int moe_selftest_wait_timeout(moe_ctx_t *ctx, void *stream);
 
 /* Decode an R x K MXFP4 matrix (codes u8 [R, K/2], scales u8 [R, K/32],
- * device pointers) into fp32 out [R, K] with the same device decode the
- * grouped GEMMs use (fp16 E2M1 conversion times the block's power of two,
- * relative to a per-row power of two 2^c_r, then multiplied back).  For tests
- * of the format. */
+ * device pointers) into fp32 out [R, K] on the device (hardware E2M1
+ * conversion to fp16 times the block's power of two, relative to a per-row
+ * power of two 2^c_r, then multiplied back).  For tests of the format; the
+ * grouped GEMMs hand the codes and scales to the tensor core as they are. */
 MOE_API int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, void *stream);
 
 /* The whole block (as moe_forward) without any device allocation, for callers

@@ -32,7 +32,7 @@ MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR
 
 # workspace buffer ids of moe_copy_workspace
 WS = dict(xn16=0, rho=1, topk_idx=2, topk_w=3, counts=4, offsets=5, row_token=6, row_w=7, h=8, out_rows=9, tiles=10,
-          pair_row=11, xperm=12)
+          pair_row=11, xperm=12, xsf=13, hsf=14)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
@@ -300,19 +300,28 @@ class MoE:
         return y_host
 
     def workspace(self, name: str, T: int, top_k: Optional[int] = None, stream=None):
-        """A device copy of one workspace buffer for the first T tokens."""
+        """A device copy of one workspace buffer for the first T tokens.
+
+        The two-term E4M3 operands (``xperm``, ``h``) and their scale words
+        (``xsf``, ``hsf``) are returned whole, sized by T_max:
+        ``xperm`` u8 [2, T_max*k, Kd], ``xsf`` int32 [Kd/128, 2, T_max*k]
+        (Kd = d_model rounded up to 128; ``h`` / ``hsf`` likewise with d_ff)."""
         import torch
         k = self.top_k if top_k is None else int(top_k)
         s = self.shape
         P = T * k
+        P_max = s.T_max * s.top_k
+        Kd = (s.d_model + 127) // 128 * 128
+        Kf = (s.d_ff + 127) // 128 * 128
         spec = {
             "xn16": ((T, s.d_model), torch.float16), "rho": ((T,), torch.float32),
             "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
             "counts": ((s.n_experts,), torch.int32), "offsets": ((s.n_experts + 1,), torch.int32),
             "row_token": ((P,), torch.int32), "row_w": ((P,), torch.float32),
-            "h": ((P, s.d_ff), torch.float16), "out_rows": ((P, s.d_model), torch.float32),
+            "out_rows": ((P, s.d_model), torch.float32),
             "tiles": ((s.n_experts + 1,), torch.int32), "pair_row": ((P,), torch.int32),
-            "xperm": ((P, s.d_model), torch.float16),     # K-blocked [d/64][P_max][64] when T == T_max
+            "xperm": ((2, P_max, Kd), torch.uint8), "xsf": ((Kd // 128, 2, P_max), torch.int32),
+            "h": ((2, P_max, Kf), torch.uint8), "hsf": ((Kf // 128, 2, P_max), torch.int32),
         }[name]
         out = torch.empty(spec[0], dtype=spec[1], device="cuda")
         moe_copy_workspace(self.ctx, WS[name], out, out.numel() * out.element_size(), stream)

@@ -16,8 +16,8 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
-                           cudaStream_t s);
+cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
+                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
@@ -30,6 +30,8 @@ using namespace moe;
 namespace {
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// the unpacked-type TMA of the weight codes needs a 32-byte aligned base
+bool aligned32(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -41,6 +43,7 @@ struct moe_ctx {
     int num_sms;
     void *ws;
     size_t ws_bytes;
+    int Kd, Kf;             // d_model and d_ff rounded up to 128
     __half *xn16;
     float *rho;
     int *topk_idx;
@@ -49,14 +52,17 @@ struct moe_ctx {
     int *row_token;
     float *row_w;
     int *pair_row;
-    __half *xperm;          // expert-sorted normalised tokens
-    __half *h;
+    uint8_t *xq;            // gate/up B: two E4M3 planes [2][P_max][Kd] of the expert-sorted tokens
+    uint32_t *xsf;          // their E8M0 scales [Kd/128][2][P_max]
+    uint8_t *hq;            // down B: two E4M3 planes [2][P_max][Kf] of h
+    uint32_t *hsf;          // [Kf/128][2][P_max]
     float *orows;           // weighted expert output per expert-sorted row
     unsigned int *err;
     unsigned long long wait_limit_ns;
-    // 3-D boxes of the K-blocked expert-sorted tokens and h: [box rows 16/32/48/64][1 or 4 K blocks]
-    CUtensorMap map_xperm[4][2];
-    CUtensorMap map_h[4][2];
+    // B tensor maps, one per token-block height (16 * (i + 1) rows), made on first use
+    CUtensorMap map_xq[GEMM_NB_MAX / 16];
+    CUtensorMap map_hq[GEMM_NB_MAX / 16];
+    bool have_xq[GEMM_NB_MAX / 16], have_hq[GEMM_NB_MAX / 16];
     const void *w13_ptr;
     CUtensorMap map_w13;
     const void *w2_ptr;
@@ -82,11 +88,13 @@ Buf ws_buffer(moe_ctx *c, int which) {
         case MOE_WS_OFFSETS: return {c->offsets, (E + 1) * 4};
         case MOE_WS_ROW_TOKEN: return {c->row_token, P * 4};
         case MOE_WS_ROW_W: return {c->row_w, P * 4};
-        case MOE_WS_H: return {c->h, P * s.d_ff * 2};
+        case MOE_WS_H: return {c->hq, 2 * P * c->Kf};
         case MOE_WS_OUT_ROWS: return {c->orows, P * s.d_model * 4};
         case MOE_WS_TILES: return {c->tiles, (E + 1) * 4};
         case MOE_WS_PAIR_ROW: return {c->pair_row, P * 4};
-        case MOE_WS_XPERM: return {c->xperm, P * s.d_model * 2};
+        case MOE_WS_XPERM: return {c->xq, 2 * P * c->Kd};
+        case MOE_WS_XSF: return {c->xsf, (size_t)(c->Kd / 128) * 2 * P * 4};
+        case MOE_WS_HSF: return {c->hsf, (size_t)(c->Kf / 128) * 2 * P * 4};
         default: return {nullptr, 0};
     }
 }
@@ -106,27 +114,40 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     GemmParams p;
     memset(&p, 0, sizeof p);
     const int E = s.n_experts, d = s.d_model, F = s.d_ff;
+    const int P_max = s.T_max * s.top_k;
     int grid = 0, smem = 0;
-    int rc = plan_gemm(p, mode, T, top_k, d, F, E, s.T_max * s.top_k, c->num_sms, &grid, &smem);
+    int rc = plan_gemm(p, mode, T, top_k, d, F, E, P_max, c->num_sms, &grid, &smem);
     if (rc) return rc;
-    const int bi = p.b_box_rows / 16 - 1, bu = p.b_unit == 4 ? 1 : 0;
+    const int bi = p.nb_rows / 16 - 1;
     if (mode == MODE_UP) {
         if (codes != c->w13_ptr) {
-            if (!encode_codes(&c->map_w13, codes, E, 2 * F, d, 64)) return MOE_ERR_CUDA;
+            if (p.K_main >= 128 && !encode_a_up(&c->map_w13, codes, E, F, d, p.K_main)) return MOE_ERR_CUDA;
             c->w13_ptr = codes;
         }
-        p.map_codes = c->map_w13;
-        p.map_b = c->map_xperm[bi][bu];
-        p.out = c->h;
+        if (!c->have_xq[bi]) {
+            if (!encode_bq(&c->map_xq[bi], c->xq, 2 * P_max, c->Kd, p.nb_rows)) return MOE_ERR_CUDA;
+            c->have_xq[bi] = true;
+        }
+        p.map_a = c->map_w13;
+        p.map_b = c->map_xq[bi];
+        p.b_sf = c->xsf;
+        p.h_q = c->hq;
+        p.h_sf = reinterpret_cast<uint8_t *>(c->hsf);
     } else {
         if (codes != c->w2_ptr) {
-            if (!encode_codes(&c->map_w2, codes, E, d, F, 128)) return MOE_ERR_CUDA;
+            if (p.K_main >= 128 && !encode_a_down(&c->map_w2, codes, E, d, F, p.K_main)) return MOE_ERR_CUDA;
             c->w2_ptr = codes;
         }
-        p.map_codes = c->map_w2;
-        p.map_b = c->map_h[bi][bu];
-        p.out = c->orows;
+        if (!c->have_hq[bi]) {
+            if (!encode_bq(&c->map_hq[bi], c->hq, 2 * P_max, c->Kf, p.nb_rows)) return MOE_ERR_CUDA;
+            c->have_hq[bi] = true;
+        }
+        p.map_a = c->map_w2;
+        p.map_b = c->map_hq[bi];
+        p.b_sf = c->hsf;
+        p.out_rows = c->orows;
     }
+    p.codes = codes;
     p.scales = scales;
     p.bias = bias;
     p.counts = c->counts;
@@ -134,7 +155,6 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     p.tiles = c->tiles;
     p.row_token = c->row_token;
     p.row_w = c->row_w;
-    p.rho = c->rho;
     p.err = c->err;
     p.wait_limit_ns = c->wait_limit_ns;
     return cuda_status(launch_expert_gemm(mode, p, grid, smem, stream));
@@ -185,14 +205,18 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
     c->num_sms = prop.multiProcessorCount;
     c->wait_limit_ns = 2000000000ull;
 
+    c->Kd = round_up_128(s.d_model);
+    c->Kf = round_up_128(s.d_ff);
     const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
     const size_t sizes[] = {T * s.d_model * 2, T * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
-                            P * 4, P * 4, P * 4, P * s.d_model * 2, P * s.d_ff * 2,
+                            P * 4, P * 4, P * 4,
+                            2 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
+                            2 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
                             P * s.d_model * 4, 64};
     void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
-                      (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xperm, (void **)&c->h,
-                      (void **)&c->orows, (void **)&c->err};
+                      (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xq, (void **)&c->xsf,
+                      (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err};
     size_t total = 0;
     for (size_t v : sizes) total += round256(v);
     if (cudaMalloc(&c->ws, total) != cudaSuccess) {
@@ -206,12 +230,7 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
         *slots[i] = sizes[i] ? b : nullptr;
         b += round256(sizes[i]);
     }
-    bool maps_ok = cudaMemset(c->ws, 0, total) == cudaSuccess;
-    for (int i = 0; i < 4 && maps_ok; ++i)
-        for (int u = 0; u < 2 && maps_ok; ++u)
-            maps_ok = encode_f16_blocked(&c->map_xperm[i][u], c->xperm, (int)P, s.d_model, 16 * (i + 1), u ? 4 : 1) &&
-                      encode_f16_blocked(&c->map_h[i][u], c->h, (int)P, s.d_ff, 16 * (i + 1), u ? 4 : 1);
-    if (!maps_ok) {
+    if (cudaMemset(c->ws, 0, total) != cudaSuccess) {
         cudaFree(c->ws);
         delete c;
         return MOE_ERR_CUDA;
@@ -272,8 +291,8 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int rc2 = cuda_status(launch_group(p, st));
     if (rc2) return rc2;
-    return cuda_status(
-        launch_permute(c->xn16, c->row_token, c->xperm, p.P, c->shape.T_max * c->shape.top_k, c->shape.d_model, st));
+    return cuda_status(launch_quant_permute(c->xn16, c->rho, c->row_token, c->xq, c->xsf, p.P,
+                                            c->shape.T_max * c->shape.top_k, c->shape.d_model, c->Kd, st));
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
@@ -281,7 +300,7 @@ int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, cons
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!aligned16(w13_codes) || !aligned16(w13_scales) || !aligned16(b13)) return MOE_ERR_ARG;
+    if (!aligned32(w13_codes) || !aligned16(w13_scales) || !aligned16(b13)) return MOE_ERR_ARG;
     return gemm_launch(c, MODE_UP, T, top_k, w13_codes, w13_scales, b13, static_cast<cudaStream_t>(stream));
 }
 
@@ -290,7 +309,7 @@ int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, con
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!aligned16(w2_codes) || !aligned16(w2_scales) || !aligned16(b2)) return MOE_ERR_ARG;
+    if (!aligned32(w2_codes) || !aligned16(w2_scales) || !aligned16(b2)) return MOE_ERR_ARG;
     return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, static_cast<cudaStream_t>(stream));
 }
 
@@ -319,8 +338,8 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!aligned16(x) || !aligned16(router_w) || !aligned16(router_b) || !aligned16(w13_codes) ||
-        !aligned16(w13_scales) || !aligned16(b13) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(router_b) || !aligned32(w13_codes) ||
+        !aligned16(w13_scales) || !aligned16(b13) || !aligned32(w2_codes) || !aligned16(w2_scales) ||
         !aligned16(b2) || !aligned16(norm_scale) || !aligned16(y))
         return MOE_ERR_ARG;
     if (y == x) return MOE_ERR_ARG;

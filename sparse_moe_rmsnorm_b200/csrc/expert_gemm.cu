@@ -1,41 +1,44 @@
-// Grouped MXFP4-weight GEMMs of the MoE experts on sm_100a (tcgen05 + TMEM + TMA).
+// Grouped MXFP4 expert GEMMs of the MoE block on sm_100a: block-scaled
+// tcgen05 MMAs (kind::mxf8f6f4, E2M1 weights x E4M3 activations, E8M0 block
+// scales) with TMA-fed shared-memory rings and fp32 accumulators in TMEM.
 //
 // One persistent CTA per SM walks the work items (expert e, 128-row weight
-// block, block of up to 256 tokens routed to e).  For each item:
-//   A (weights, M = 128 rows): packed E2M1 codes arrive by TMA (128-byte
-//     swizzle) into a shared-memory ring; the E8M0 scales of the 128 rows by
-//     one untiled bulk copy.  Decoder warps convert 64 K-elements per row at a
-//     time to fp16 (hardware e2m1x2 conversion times the block's power of
-//     two, relative to a per-row power of two that keeps every block of the
-//     row exact in fp16) and store them straight into tensor memory, where
-//     the MMA reads A ("A from TMEM" form).  The decoded weights never touch
-//     shared memory, so shared-memory bandwidth is left to the codes and B.
-//   B (activations, N = tokens, K-major fp16): TMA boxes of up to 64
-//     expert-sorted rows (the sorted copy of the normalised tokens for the
-//     gate/up GEMM, h for the down GEMM) into a shared-memory ring in the
-//     128-byte swizzled canonical layout.
-//   D (fp32, 128 lanes x N columns) accumulates in TMEM.  A tcgen05.mma
-//     occupies its issuing thread for about 120 cycles whatever N is, so small
-//     token blocks are spread over up to three MMA warps, each accumulating
-//     every third sub-stage into its own accumulator; the epilogue sums them.
-// Gate/up epilogue: z = D * 2^c * rho_token + b13, clamped SwiGLU
+// block, block of up to GEMM_NB_MAX tokens routed to e).  Per 128-K stage:
+//   A (weights, M = 128 rows): the packed E2M1 codes go from HBM to shared
+//     memory by TMA with the unpacked 4-bit type (16 codes per 16 bytes, the
+//     operand layout of the block-scaled MMA) and a 128-byte swizzle.  No
+//     thread touches a weight element: the tensor core applies the E8M0 block
+//     scales itself ("MXFP4": 32 elements share one power of two, pnsm.cn
+//     overview sections 1 and 4).  A K tail of 64 (K = 2880 = 22.5 x 128) is
+//     copied and unpacked by the scale-factor warps.
+//   B (activations, N = tokens): two E4M3 terms, hi = e4m3(v / 2^s) and
+//     lo = e4m3((v - hi 2^s) / 2^(s-4)), per 32-element block with E8M0 scale
+//     s chosen so the block maximum fits 448.  hi + lo keeps about 8
+//     significant bits of every element (the precision of bf16).  The hi rows
+//     and lo rows of a token block sit one after the other in the B ring; small
+//     blocks feed both in one MMA (N = 2 x rows, the epilogue adds the halves),
+//     large ones in two MMAs into the same accumulator.
+//   Scale factors: per stage the scale-factor warps write A's and B's E8M0
+//     bytes into a TMEM slot, one 32-bit column per 32 rows, the byte index
+//     being the 32-block within the stage, replicated in all four lane
+//     quarters (the layout the block-scaled MMA reads).
+// Gate/up epilogue: z = D + b13, clamped SwiGLU
 //   h = min(g,7) * sigmoid(1.702 min(g,7)) * (clamp(u,-7,7) + 1)
-//   ("gpt-oss-20B" hub page, section 3.3); each 128-row block holds 64 gate
-//   rows and their 64 linear rows so the pair meets in one warp.
-// Down epilogue: o = w_token * (D * 2^c + b2) written to the pair's
-//   expert-sorted row; the combine kernel adds a token's rows to its residual
-//   (weighted combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
+//   ("gpt-oss-20B" hub page, section 3.3).  Each 128-row weight block holds 64
+//   gate rows and their 64 linear rows, interleaved in groups of 16 by the
+//   tensor map, so each pair meets in one warp.  h is written directly as the
+//   down GEMM's two-term B: the block maxima over 32 consecutive h rows are
+//   exchanged between the two warps holding them.
+// Down epilogue: o = w_token * (D + b2) written to the pair's expert-sorted
+//   row; the combine kernel adds a token's rows to its residual (weighted
+//   combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
 //
-// Warp roles (672 threads): 0 codes/scales producer, 20 B producer (TMA
-// instructions hold their issuing thread too, so the two streams get their
-// own threads), 1-3 MMA issue (3 also allocates TMEM), 4-7 and 12-15
-// decoder groups, 8-11 epilogue group; warps 16-19 are a third decoder group
-// for small token blocks (several MMA warps) and a second epilogue group
-// otherwise.  Decoder groups take two-sub-stage chunks in turn; epilogue
-// groups take 16-column chunks in turn.  The decoders hand each row's power-of-two shift to the
-// epilogue through shared memory.  Every mbarrier wait is bounded (WaitCtl);
-// when one runs out the CTA stops issuing work, drains its copies and MMAs in
-// flight, frees TMEM and returns with the error latched.
+// Warp roles (512 threads): 0 TMA producer, 1 MMA issue, 2 TMEM allocation,
+// 4-7 scale-factor warps (one per TMEM lane quarter), 8-11 and 12-15 two
+// epilogue groups taking 16-column chunks in turn.  Producer and MMA run as
+// whole converged warps, one elected lane issuing.  Every mbarrier wait is
+// bounded (WaitCtl); when one runs out the CTA stops issuing work, drains its
+// copies and MMAs in flight, frees TMEM and returns with the error latched.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -81,74 +84,53 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n_slots, long lon
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-// Largest and smallest E8M0 byte of a row (255 excluded from the largest; a
-// 255 makes the smallest -1), n even, row 2-byte aligned.
-__device__ __forceinline__ void row_scale_range(const uint8_t *s, int n, int &mx, int &mn) {
-    const uint16_t *w = reinterpret_cast<const uint16_t *>(s);
-    mx = -1;
-    mn = 256;
-#pragma unroll 8
-    for (int b = 0; b < n / 2; ++b) {
-        const uint32_t v = w[b];
-        const int lo = (int)(v & 0xFFu), hi = (int)(v >> 8);
-        mx = max(mx, lo == 255 ? -1 : lo);
-        mx = max(mx, hi == 255 ? -1 : hi);
-        mn = min(mn, lo == 255 ? -1 : lo);
-        mn = min(mn, hi == 255 ? -1 : hi);
+// Source row (0..127) in the work item's scale buffer of tile row r (the A
+// row in shared memory and TMEM lane r).  UP: the buffer holds the 64 gate rows
+// then the 64 linear rows; tile row 32q + l is gate row 16q + l (l < 16) or
+// linear row 16q + l - 16.
+template <int MODE>
+__device__ __forceinline__ int tile_scale_row(int r) {
+    if (MODE == MODE_UP) {
+        const int q = r >> 5, l = r & 31;
+        return l < 16 ? 16 * q + l : 64 + 16 * q + (l - 16);
     }
+    return r;
 }
 
-// Largest E8M0 byte (other than 255) of a row's n scale bytes (n even, row
-// 2-byte aligned), read as 16-bit words so the loads pipeline.
-__device__ __forceinline__ int row_scale_max(const uint8_t *s, int n) {
-    const uint16_t *w = reinterpret_cast<const uint16_t *>(s);
-    int m = -1;
-#pragma unroll 8
-    for (int b = 0; b < n / 2; ++b) {
-        const uint32_t v = w[b];
-        const int lo = (int)(v & 0xFFu), hi = (int)(v >> 8);
-        m = max(m, lo == 255 ? -1 : lo);
-        m = max(m, hi == 255 ? -1 : hi);
+// Weight row of tile row r in the expert's row space (UP: [0, 2F); DOWN: [0, d)).
+template <int MODE>
+__device__ __forceinline__ int tile_weight_row(int r, int mb, int F) {
+    if (MODE == MODE_UP) {
+        const int q = r >> 5, l = r & 31;
+        return l < 16 ? mb * 64 + 16 * q + l : F + mb * 64 + 16 * q + (l - 16);
     }
-    return m;
+    return mb * GEMM_BM + r;
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int U = p.b_unit;
-    const int b_slot_bytes = U * p.b_stage_bytes;
-    const GemmSmem plan = gemm_smem_plan(p.K, p.E, p.n_c_stages, p.n_a_slots, p.n_b_stages, b_slot_bytes);
-    const int SC = p.n_c_stages, NA = p.n_a_slots, NBS = p.n_b_stages, NI = p.n_iss;
-    const int NP = NA / 2;                 // A slot pairs: one pair per decoder chunk of two sub-stages
-    const int NG = p.n_dec_groups;         // decoder groups
-    const int NEG = NG == 3 ? 1 : 2;       // epilogue groups
-    const int PPG = NP / NG;               // slot pairs owned by each decoder group
-    // Chunk gc (two sub-stages of a code stage) is decoded by group gc % NG into
-    // the group's pair (gc / NG) % PPG and its MMAs are issued by MMA warp
-    // (gc % NG) % NI, so each decoder group and its MMA warp form one pipeline.
-    uint8_t *code_ring = smem + plan.code_off;
+    const int NS = p.n_stages;
+    const int NB = p.nb_rows;
+    const GemmSmem plan = gemm_smem_plan(p.K, p.E, NB, NS);
+    uint8_t *a_ring = smem + plan.a_off;
     uint8_t *b_ring = smem + plan.b_off;
+    const int b_stage = gemm_b_stage_bytes(NB);
     uint8_t *scale_buf = smem + plan.scale_off;
-    const int scale_bytes = align_up(GEMM_BM * (p.K / 32), 128);
-    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off);    // [8 warps][NB_MAX / 2]
-    int *tok_s = reinterpret_cast<int *>(smem + plan.tok_off);            // [NB_MAX]
-    int *shift_s = reinterpret_cast<int *>(smem + plan.shift_off);        // [2][128]
+    const int KB32 = p.K / 32;
+    const int scale_bytes = align_up(GEMM_BM * KB32, 128);
+    float *amax_s = reinterpret_cast<float *>(smem + plan.amax_off);   // [2 groups][2 parities][4 warps][16 columns]
+    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off);  // [8 warps][GEMM_NB_MAX]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bar_off);
-    uint64_t *c_full = bars;
-    uint64_t *c_empty = c_full + SC;
-    uint64_t *s_full = c_empty + SC;
+    uint64_t *full = bars;
+    uint64_t *empty = full + NS;
+    uint64_t *s_full = empty + NS;
     uint64_t *s_empty = s_full + 2;
-    uint64_t *a_full = s_empty + 2;
-    uint64_t *a_empty = a_full + NA;
-    uint64_t *b_full = a_empty + NA;
-    uint64_t *b_empty = b_full + NBS;
-    uint64_t *d_full = b_empty + NBS;
+    uint64_t *d_full = s_empty + 2;
     uint64_t *d_empty = d_full + 2;
-    uint64_t *h_full = d_empty + 2;
-    uint64_t *h_empty = h_full + 2;
-    uint64_t *drain_bar = h_empty + 2;                                     // [GEMM_ISS_MAX]
+    uint64_t *drain_bar = d_empty + 2;
+    uint64_t *ex_bar = drain_bar + 1;                                     // [2 groups][2 parities]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
@@ -156,32 +138,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     int *tiles_s = offsets_s + (p.E + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB32 = p.K / 32;
-    const int n_sub = p.K / GEMM_KA;
-    const int n_cstages = (p.K + GEMM_KS - 1) / GEMM_KS;
+    const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;     // stages per work item
+    const int n_main = p.K_main / GEMM_KS;              // stages loaded by TMA; a last one past them is the K tail
+    const int d_cols = gemm_d_cols(NB, p.stacked);
+    const uint32_t sf_col0 = (uint32_t)(2 * d_cols);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SC; ++i) {
-            mbar_init(&c_full[i], 1);
-            mbar_init(&c_empty[i], 4 * NG);   // every decoder warp
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1 + 4);   // producer's expect_tx arrive + the four scale-factor warps
+            mbar_init(&empty[i], 1);      // MMA commit
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4 * NG);
-            mbar_init(&d_full[i], NI);        // one commit per MMA warp
-            mbar_init(&d_empty[i], 4 * NEG);  // every epilogue warp
-            mbar_init(&h_full[i], 4);
-            mbar_init(&h_empty[i], 4 * NEG);
+            mbar_init(&s_empty[i], 4);
+            mbar_init(&d_full[i], 1);
+            mbar_init(&d_empty[i], 8);    // every epilogue warp
         }
-        for (int i = 0; i < NP; ++i) {
-            mbar_init(&a_full[i], 4);         // the four warps of the group that decoded the pair
-            mbar_init(&a_empty[i], 1);        // the commit of the MMA warp that consumed it
-        }
-        for (int i = 0; i < NBS; ++i) {
-            mbar_init(&b_full[i], 1);
-            mbar_init(&b_empty[i], U);     // one commit per sub-stage of the slot
-        }
-        for (int i = 0; i < GEMM_ISS_MAX; ++i) mbar_init(&drain_bar[i], 1);
+        mbar_init(drain_bar, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&ex_bar[i], 4);   // the four warps of an epilogue group
         *abort_s = 0;
         fence_barrier_init();
     }
@@ -190,7 +164,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         offsets_s[i] = p.offsets[i];
         tiles_s[i] = p.tiles[i];
     }
-    if (warp == 3) {
+    if (warp == 2) {
         tmem_alloc(tmem_base_s, 512);
         tmem_relinquish();
     }
@@ -201,323 +175,233 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     const int total = p.MB * tiles_s[p.E];
     const WaitCtl wc{abort_s, p.err, MODE == MODE_UP ? (unsigned)ERR_WAIT_UP : (unsigned)ERR_WAIT_DOWN,
                      p.wait_limit_ns};
-    // accumulator of MMA warp i in buffer set db: columns NA*32 + (db*NI + i)*nb_rows
-    const uint32_t d_col0 = (uint32_t)(NA * 32);
 
     if (warp == 0) {
-        // ------------------------------------------------ codes + scales producer
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&p.map_codes);
-            int cslot = 0, sb = 0;
-            uint32_t cph = 0, sph = 0;
-            long long c_issued = 0, s_issued = 0;
-            bool ok = true;
-            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                Work t;
-                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-                if (!mbar_wait(&s_empty[sb], sph ^ 1, wc)) { ok = false; break; }
-                uint8_t *sdst = scale_buf + sb * scale_bytes;
-                if (MODE == MODE_UP) {
-                    const int j0 = t.mb * 64;
-                    const uint32_t bytes = 64u * KB32;
-                    mbar_arrive_expect_tx(&s_full[sb], 2 * bytes);
-                    bulk_load(sdst, p.scales + ((size_t)t.e * p.R + j0) * KB32, bytes, &s_full[sb]);
-                    bulk_load(sdst + bytes, p.scales + ((size_t)t.e * p.R + p.F + j0) * KB32, bytes, &s_full[sb]);
-                } else {
-                    const int m0 = t.mb * GEMM_BM;
-                    const uint32_t bytes = (uint32_t)min(GEMM_BM, p.R - m0) * KB32;
-                    mbar_arrive_expect_tx(&s_full[sb], bytes);
-                    bulk_load(sdst, p.scales + ((size_t)t.e * p.R + m0) * KB32, bytes, &s_full[sb]);
-                }
-                ++s_issued;
-                if (++sb == 2) { sb = 0; sph ^= 1; }
-                for (int ks = 0; ks < n_cstages; ++ks) {
-                    if (!mbar_wait(&c_empty[cslot], cph ^ 1, wc)) { ok = false; break; }
-                    uint8_t *cdst = code_ring + cslot * GEMM_CODE_STAGE;
-                    mbar_arrive_expect_tx(&c_full[cslot], GEMM_CODE_STAGE);
-                    if (MODE == MODE_UP) {
-                        tma_load_3d(cdst, &p.map_codes, &c_full[cslot], ks * 128, t.mb * 64, t.e);
-                        tma_load_3d(cdst + 64 * 128, &p.map_codes, &c_full[cslot], ks * 128, p.F + t.mb * 64, t.e);
-                    } else {
-                        tma_load_3d(cdst, &p.map_codes, &c_full[cslot], ks * 128, t.mb * GEMM_BM, t.e);
-                    }
-                    ++c_issued;
-                    if (++cslot == SC) { cslot = 0; cph ^= 1; }
-                }
-            }
-            if (!ok) {
-                drain_ring(c_full, SC, c_issued, p.wait_limit_ns);
-                drain_ring(s_full, 2, s_issued, p.wait_limit_ns);
-            }
-        }
-    } else if (warp == 20) {
-        // ------------------------------------------------------------ B producer
-        // One slot holds U consecutive 64-K blocks of the work item's token
-        // rows; with U = 4 a single 3-D TMA box fills it.
-        if (lane == 0) {
+            if (n_main > 0) tma_prefetch_desc(&p.map_a);
             tma_prefetch_desc(&p.map_b);
-            int bslot = 0;
-            uint32_t bph = 0;
-            long long b_issued = 0;
-            bool ok = true;
-            const int box = p.b_box_rows;
-            const int n_units = (n_sub + U - 1) / U;
-            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                Work t;
-                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-                const int nbox = (t.n_mma + box - 1) / box;
-                for (int u = 0; u < n_units; ++u) {
-                    if (!mbar_wait(&b_empty[bslot], bph ^ 1, wc)) { ok = false; break; }
-                    uint8_t *bdst = b_ring + bslot * b_slot_bytes;
-                    mbar_arrive_expect_tx(&b_full[bslot], (uint32_t)(nbox * box * 128 * U));
-                    for (int g = 0; g < nbox; ++g)
-                        tma_load_3d(bdst + g * box * 128 * U, &p.map_b, &b_full[bslot], 0, t.p0 + box * g, u * U);
-                    // a slot past the last K block is consumed fewer than U times
-                    for (int r = min(U, n_sub - u * U); r < U; ++r) mbar_arrive(&b_empty[bslot]);
-                    ++b_issued;
-                    if (++bslot == NBS) { bslot = 0; bph ^= 1; }
-                }
-            }
-            if (!ok) drain_ring(b_full, NBS, b_issued, p.wait_limit_ns);
         }
-    } else if (warp >= 1 && warp <= 3) {
-        // ------------------------------------------- MMA issue: warp i-1 takes sub-stages i-1, i-1+NI, ...
-        const int mi = warp - 1;
-        if (lane == 0 && mi < NI) {
-            int db = 0;
-            uint32_t dph = 0;
-            // Running counters instead of divisions (a 64-bit division is a long
-            // software routine): the decoder group of the next chunk, each
-            // group's next pair and its phase, and the next B fill.
-            int turn = 0;                          // decoder group of the next chunk
-            int pp0 = 0, pp1 = 0, pp2 = 0;         // next pair (within its group) of groups 0..2
-            uint32_t ph0 = 0, ph1 = 0, ph2 = 0;    // phase parity of that pair
-            int ub = 0, bslot = 0;                 // next B fill (within the work item) and its slot
-            uint32_t bph = 0;
-            const int ushift = U == 4 ? 2 : 0;
-            const int n_units = (n_sub + U - 1) / U;
-            const int n_chunks = (n_sub + 1) / 2;  // two per full code stage, ceil(r/2) for a tail of r
-            bool ok = true, issued = false;
-            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                Work t;
-                work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-                const uint32_t idesc = idesc_f16_f32(GEMM_BM, (uint32_t)t.n_mma);
-                if (!mbar_wait(&d_empty[db], dph ^ 1, wc)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + d_col0 + (uint32_t)((db * NI + mi) * p.nb_rows);
-                bool first = true;
-                int u_base = 0;                    // B fills consumed before this work item, relative
-                for (int ci = 0; ci < n_chunks && ok; ++ci) {
-                    const int grp = turn;
-                    turn = turn + 1 == NG ? 0 : turn + 1;
-                    const int lp = grp == 0 ? pp0 : (grp == 1 ? pp1 : pp2);
-                    const uint32_t lph = grp == 0 ? ph0 : (grp == 1 ? ph1 : ph2);
-                    {
-                        int np_ = lp + 1;
-                        uint32_t nph = lph;
-                        if (np_ == PPG) { np_ = 0; nph ^= 1; }
-                        if (grp == 0) { pp0 = np_; ph0 = nph; } else if (grp == 1) { pp1 = np_; ph1 = nph; } else { pp2 = np_; ph2 = nph; }
-                    }
-                    if (grp % NI != mi) continue;
-                    const int pair = grp * PPG + lp;
-                    if (!mbar_wait(&a_full[pair], lph, wc)) { ok = false; break; }
-                    // sub-stages of chunk ci: 2 per code stage, the tail stage may hold 1..4
-                    const int j0 = 4 * (ci >> 1) + 2 * (ci & 1);
-                    const int na = min(2, n_sub - j0);
-                    for (int u = 0; u < na; ++u) {
-                        const int j = j0 + u;
-                        const int target = j >> ushift;        // B fill of sub-stage j within the work item
-                        while (ub < u_base + target) {
-                            ++ub;
-                            if (++bslot == NBS) { bslot = 0; bph ^= 1; }
-                        }
-                        if (!mbar_wait(&b_full[bslot], bph, wc)) { ok = false; break; }
-                        tc_fence_after();
-                        // sub-stage block j % U of the slot
-                        const uint32_t b_addr =
-                            smem_addr(b_ring + bslot * b_slot_bytes + (j & (U - 1)) * p.b_stage_bytes);
-                        const uint32_t a_tmem = tmem + (uint32_t)((2 * pair + u) * 32);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            mma_f16_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
-                                       first ? 0u : 1u);
-                            first = false;
-                        }
-                        issued = true;
-                        mma_commit(&b_empty[bslot]);
-                    }
-                    if (!ok) break;
-                    mma_commit(&a_empty[pair]);
-                }
-                if (!ok) break;
-                // move the B counters to the first fill of the next work item
-                while (ub < u_base + n_units) {
-                    ++ub;
-                    if (++bslot == NBS) { bslot = 0; bph ^= 1; }
-                }
-                ub -= u_base + n_units;
-                mma_commit(&d_full[db]);
-                if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
-            }
-            if (!ok && issued) {
-                mma_commit(&drain_bar[mi]);
-                mbar_wait_drain(&drain_bar[mi], 0, p.wait_limit_ns);
-            }
-        }
-    } else if ((warp >= 4 && warp < 8) || (warp >= 12 && warp < 16 && NG >= 2) || (warp >= 16 && warp < 20 && NG == 3)) {
-        // ------------------------------------------------------------ decoders
-        // NG groups of four warps.  Each code stage (4 sub-stages of 64 K
-        // elements) is cut into chunks of two sub-stages; chunk gc goes to
-        // group gc mod NG and fills one of the group's own A slot pairs (TMEM
-        // lanes 32q..32q+31 of its warps), with one handshake per chunk.
-        const int q = warp & 3;
-        const int grp = warp < 8 ? 0 : (warp < 16 ? 1 : 2);
-        const int tl = 32 * q + lane;                           // TMEM lane = A row
-        const int my_row = MODE == MODE_UP ? (16 * q + (lane & 15) + (lane >= 16 ? 64 : 0)) : tl;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        int cslot = 0, sb = 0, hb = 0;
-        uint32_t cph = 0, sph = 0, hph = 0;
-        int turn = 0;                                           // decoder group of the next chunk
-        int mpair = 0;                                          // this group's next pair (within the group)
-        uint32_t mph = 0;                                       // and its phase parity
+        int slot = 0, sb = 0;
+        uint32_t ph = 0, sph = 0;
+        long long issued = 0, s_issued = 0;
         bool ok = true;
+        const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-            const bool row_valid = MODE == MODE_UP || (t.mb * GEMM_BM + my_row < p.R);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
-            const uint8_t *srow = scale_buf + sb * scale_bytes + my_row * KB32;
-            int smax = -1, smin = 256;
-            if (row_valid) row_scale_range(srow, KB32, smax, smin);
-            const int c = row_shift_from_max(smax);
-            const bool fast = row_valid && smin >= smax - 27;   // every block multiplier is a normal fp16
-            if (grp == 0) {
-                // hand the row shift to the epilogue
-                if (!__all_sync(0xffffffffu, mbar_wait(&h_empty[hb], hph ^ 1, wc))) { ok = false; break; }
-                shift_s[hb * GEMM_BM + tl] = c;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&h_full[hb]);
-                if (++hb == 2) { hb = 0; hph ^= 1; }
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            // the work item's A scales
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[sb], sph ^ 1, wc))) { ok = false; break; }
+            uint8_t *sdst = scale_buf + sb * scale_bytes;
+            if (MODE == MODE_UP) {
+                const int j0 = t.mb * 64;
+                const uint32_t bytes = 64u * KB32;
+                mbar_arrive_expect_tx_w(&s_full[sb], 2 * bytes);
+                bulk_load_w(sdst, p.scales + ((size_t)t.e * p.R + j0) * KB32, bytes, &s_full[sb]);
+                bulk_load_w(sdst + bytes, p.scales + ((size_t)t.e * p.R + p.F + j0) * KB32, bytes, &s_full[sb]);
+            } else {
+                const int m0 = t.mb * GEMM_BM;
+                const uint32_t bytes = (uint32_t)min(GEMM_BM, p.R - m0) * KB32;
+                mbar_arrive_expect_tx_w(&s_full[sb], bytes);
+                bulk_load_w(sdst, p.scales + ((size_t)t.e * p.R + m0) * KB32, bytes, &s_full[sb]);
             }
-            for (int ks = 0; ks < n_cstages && ok; ++ks) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&c_full[cslot], cph, wc))) { ok = false; break; }
-                const uint8_t *crow = code_ring + cslot * GEMM_CODE_STAGE + my_row * 128;
-                const int nsub = min(4, (p.K - ks * GEMM_KS) / GEMM_KA);
-                // the 8 block multipliers of this code stage
-                uint32_t mult[8];
+            ++s_issued;
+            if (++sb == 2) { sb = 0; sph ^= 1; }
+            for (int st = 0; st < n_st; ++st) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                const bool has_a = st < n_main;
+                // the unpacked-type TMA counts the packed bytes: 128 rows x 64
+                mbar_arrive_expect_tx_w(&full[slot], (has_a ? 128u * 64u : 0u) + b_bytes);
+                if (has_a) {
+                    if (MODE == MODE_UP)
+                        tma_load_5d_w(a_ring + slot * GEMM_A_STAGE, &p.map_a, &full[slot], st * GEMM_KS, 0, 0,
+                                      4 * t.mb, t.e);
+                    else
+                        tma_load_3d_w(a_ring + slot * GEMM_A_STAGE, &p.map_a, &full[slot], st * GEMM_KS,
+                                      t.mb * GEMM_BM, t.e);
+                }
+                uint8_t *bdst = b_ring + slot * b_stage;
+                tma_load_2d_w(bdst, &p.map_b, &full[slot], st * GEMM_KS, t.p0);
+                tma_load_2d_w(bdst + NB * 128, &p.map_b, &full[slot], st * GEMM_KS, p.P_max + t.p0);
+                ++issued;
+                if (++slot == NS) { slot = 0; ph ^= 1; }
+            }
+        }
+        if (!ok) {
+            drain_ring(full, NS, issued, p.wait_limit_ns);
+            drain_ring(s_full, 2, s_issued, p.wait_limit_ns);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issue
+        int slot = 0, db = 0;
+        uint32_t ph = 0, dph = 0;
+        bool ok = true, issued = false;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            const uint32_t n = p.stacked ? (uint32_t)(2 * NB) : (uint32_t)t.n_mma;
+            // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
+            // E8M0 scales, M >> 4; the scale byte of each MMA is set per K block below
+            const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
+            if (!__all_sync(0xffffffffu, mbar_wait(&d_empty[db], dph ^ 1, wc))) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + (uint32_t)(db * d_cols);
+            uint32_t acc = 0;
+            for (int st = 0; st < n_st; ++st) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_addr = smem_addr(a_ring + slot * GEMM_A_STAGE);
+                const uint32_t b_addr = smem_addr(b_ring + slot * b_stage);
+                const uint32_t sf = tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                const int nkb = st < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const uint32_t idesc = idesc0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
+                    const uint64_t ad = smem_desc_sw128(a_addr + kb * 32);
+                    mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + kb * 32), idesc, sf, sf + 8, acc);
+                    if (!p.stacked)
+                        mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + NB * 128 + kb * 32), idesc, sf, sf + 16, 1u);
+                    acc = 1;
+                }
+                issued = true;
+                mma_commit_w(&empty[slot]);
+                if (++slot == NS) { slot = 0; ph ^= 1; }
+            }
+            if (!ok) break;
+            mma_commit_w(&d_full[db]);
+            if (++db == 2) { db = 0; dph ^= 1; }
+        }
+        if (!ok && issued) {
+            mma_commit_w(drain_bar);
+            mbar_wait_drain(drain_bar, 0, p.wait_limit_ns);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------ scale-factor warps
+        // Warp q writes TMEM lane quarter q: column c of a region holds, in
+        // lane 32q + i, the four E8M0 bytes (32-blocks 4st..4st+3) of row
+        // 32c + i of the operand.
+        const int q = warp & 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        int slot = 0, sb = 0;
+        uint32_t ph = 0, sph = 0;
+        bool ok = true;
+        const int n_sfb = p.stacked ? (2 * NB + 31) / 32 : (NB + 31) / 32;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
+            const uint8_t *sbase = scale_buf + sb * scale_bytes;
+            const uint8_t *srow[4];
+            bool row_ok[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                srow[c] = sbase + tile_scale_row<MODE>(32 * c + lane) * KB32;
+                row_ok[c] = MODE == MODE_UP || t.mb * GEMM_BM + 32 * c + lane < p.R;
+            }
+            for (int st = 0; st < n_st; ++st) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                // A: four columns
                 {
-                    const uint16_t *sw16 = reinterpret_cast<const uint16_t *>(srow + ks * 8);
+                    const int nblk = KB32 - 4 * st;     // 32-blocks of this stage inside K: 2 or >= 4
+                    uint32_t v[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t v = (2 * i < 2 * nsub) ? (uint32_t)sw16[i] : 0x7F7Fu;
-                        const int s0 = (int)(v & 0xFFu), s1 = (int)(v >> 8);
-                        if (fast) {
-                            mult[2 * i] = block_multiplier_fast(s0, smax);
-                            mult[2 * i + 1] = block_multiplier_fast(s1, smax);
-                        } else {
-                            mult[2 * i] = block_multiplier(s0, c);
-                            mult[2 * i + 1] = block_multiplier(s1, c);
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t wv = 0x7F7F7F7Fu;
+                        if (row_ok[c]) {
+                            const uint16_t *s16 = reinterpret_cast<const uint16_t *>(srow[c] + 4 * st);
+                            const uint32_t lo = s16[0];
+                            const uint32_t hi = nblk > 2 ? (uint32_t)s16[1] : 0x7F7Fu;
+                            wv = lo | (hi << 16);
                         }
+                        v[c] = wv;
                     }
+                    tmem_st4(sf, v);
                 }
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int a0 = 2 * cc;
-                    if (a0 >= nsub) break;
-                    const int na = min(2, nsub - a0);
-                    const bool mine = turn == grp;
-                    turn = turn + 1 == NG ? 0 : turn + 1;
-                    if (!mine) continue;
-                    const int pair = grp * PPG + mpair;
-                    const uint32_t pph = mph;
-                    if (++mpair == PPG) { mpair = 0; mph ^= 1; }
-                    if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[pair], pph ^ 1, wc))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const int sw = my_row & 7;
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        if (u < na) {
-                            const int a = a0 + u;
-                            uint32_t out[32];
-                            if (row_valid) {
-                                const uint4 w0 = *reinterpret_cast<const uint4 *>(crow + (((2 * a) ^ sw) << 4));
-                                const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + (((2 * a + 1) ^ sw) << 4));
-                                const uint32_t m0 = mult[2 * a], m1 = mult[2 * a + 1];
-                                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    uint32_t h4[4];
-                                    e2m1x8_to_half2x4(words[i], h4);
-#pragma unroll
-                                    for (int jj = 0; jj < 4; ++jj) out[4 * i + jj] = hmul2_u32(h4[jj], i < 4 ? m0 : m1);
-                                }
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) out[i] = 0u;
+                // B: hi (and lo) rows of the token block
+                {
+                    const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max;
+                    if (p.stacked) {
+                        for (int c = 0; c < n_sfb; ++c) {
+                            const int r = 32 * c + lane;            // stacked row: hi rows [0, NB), lo rows [NB, 2NB)
+                            const int plane = r >= NB ? 1 : 0;
+                            const int j = r - plane * NB;
+                            uint32_t wv = 0x7F7F7F7Fu;
+                            if (r < 2 * NB && j < t.n_valid) wv = bsf[(size_t)plane * p.P_max + t.p0 + j];
+                            tmem_st1(sf + 8 + (uint32_t)c, wv);
+                        }
+                    } else {
+                        for (int c = 0; c < n_sfb; ++c) {
+                            const int j = 32 * c + lane;
+                            uint32_t w0 = 0x7F7F7F7Fu, w1 = 0x7F7F7F7Fu;
+                            if (j < t.n_valid) {
+                                w0 = bsf[t.p0 + j];
+                                w1 = bsf[(size_t)p.P_max + t.p0 + j];
                             }
-                            tmem_st32(lane_base + (uint32_t)((2 * pair + u) * 32), out);
+                            tmem_st1(sf + 8 + (uint32_t)c, w0);
+                            tmem_st1(sf + 16 + (uint32_t)c, w1);
                         }
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&a_full[pair]);
                 }
-                if (!ok) break;
+                if (st >= n_main) {
+                    // the K tail of tile rows 32q..32q+31: up to 2 x 16 code bytes ->
+                    // the first four 16-byte units of the row (8 code bytes each, the
+                    // rest zero), 128-byte swizzle
+                    const int r = 32 * q + lane;
+                    const int wrow = tile_weight_row<MODE>(r, t.mb, p.F);
+                    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+                    if (wrow < p.R) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
+                        c0 = src[0];
+                        c1 = src[1];
+                    }
+                    uint8_t *row = a_ring + slot * GEMM_A_STAGE + r * 128;
+                    const int sw = r & 7;
+                    *reinterpret_cast<uint4 *>(row + ((0 ^ sw) << 4)) = make_uint4(c0.x, c0.y, 0, 0);
+                    *reinterpret_cast<uint4 *>(row + ((1 ^ sw) << 4)) = make_uint4(c0.z, c0.w, 0, 0);
+                    *reinterpret_cast<uint4 *>(row + ((2 ^ sw) << 4)) = make_uint4(c1.x, c1.y, 0, 0);
+                    *reinterpret_cast<uint4 *>(row + ((3 ^ sw) << 4)) = make_uint4(c1.z, c1.w, 0, 0);
+                    fence_proxy_async_smem();
+                }
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[cslot]);
-                if (++cslot == SC) { cslot = 0; cph ^= 1; }
+                mbar_arrive_w(&full[slot]);
+                if (++slot == NS) { slot = 0; ph ^= 1; }
             }
             if (!ok) break;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            mbar_arrive_w(&s_empty[sb]);
             if (++sb == 2) { sb = 0; sph ^= 1; }
         }
-    } else if ((warp >= 8 && warp < 12) || (warp >= 16 && warp < 20 && NG < 3)) {
-        // ------------------------------------------------------------- epilogue
+    } else if (warp >= 8) {
+        // ---------------------------------------------------------------- epilogue
         // Two groups of four warps; group eg takes the 16-column chunks
-        // eg, eg+2, eg+4, ... of the accumulators, summing the MMA warps' parts.
+        // eg, eg+2, eg+4, ... of the accumulator.
         const int q = warp & 3;
-        const int eg = warp >= 16 ? 1 : 0;
+        const int eg = (warp - 8) >> 2;
         const int tl = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        float *mval = meta_val + (eg * 4 + q) * (GEMM_NB_MAX / 2);      // value of chunk m's column i at [(m/2)*16 + i]
-        int db = 0, hb = 0;
-        uint32_t dph = 0, hph = 0;
-        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        float *mval = meta_val + (warp - 8) * GEMM_NB_MAX;
+        int db = 0;
+        uint32_t dph = 0;
+        bool ok = true;
+        int chunk_par = 0;
+        uint32_t ex_ph = 0;                  // bit i: phase parity of exchange buffer i
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, p.nb_rows, t);
-            int row;
-            bool row_valid;
-            if (MODE == MODE_UP) {
-                row = (lane < 16 ? 0 : p.F) + t.mb * 64 + 16 * q + (lane & 15);
-                row_valid = true;
-            } else {
-                row = t.mb * GEMM_BM + tl;
-                row_valid = row < p.R;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            const int wrow = tile_weight_row<MODE>(tl, t.mb, p.F);
+            const bool row_valid = wrow < p.R;
+            const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + wrow]) : 0.f;
+            if (MODE == MODE_DOWN) {
+                for (int c = lane; c < t.n_valid; c += 32) mval[c] = p.row_w[t.p0 + c];
+                __syncwarp();
             }
-            const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + row]) : 0.f;
-            // per-column rho (UP) or routing weight (DOWN) of this group's columns
-            for (int cc = lane; cc < GEMM_NB_MAX / 2; cc += 32) {
-                const int col = ((cc >> 4) * NEG + eg) * 16 + (cc & 15);
-                if (col < t.n_mma) {
-                    const int pr = t.p0 + min(col, t.n_valid - 1);
-                    mval[cc] = MODE == MODE_UP ? p.rho[p.row_token[pr]] : p.row_w[pr];
-                }
-            }
-            __syncwarp();
-            if (!__all_sync(0xffffffffu, mbar_wait(&h_full[hb], hph, wc))) break;
-            const float cscale = exp2i(shift_s[hb * GEMM_BM + tl]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&h_empty[hb]);
-            if (++hb == 2) { hb = 0; hph ^= 1; }
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
             tc_fence_after();
-            const uint32_t d_tmem = lane_base + d_col0 + (uint32_t)(db * NI * p.nb_rows);
-            for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 16 * NEG) {
+            const uint32_t d_tmem = lane_base + (uint32_t)(db * d_cols);
+            for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
                 float acc[16];
                 {
                     uint32_t v[16];
@@ -525,56 +409,102 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
-                }
-                for (int mi = 1; mi < NI; ++mi) {
-                    uint32_t v[16];
-                    tmem_ld16(d_tmem + (uint32_t)(mi * p.nb_rows + c0), v);
-                    tmem_wait_ld();
+                    if (p.stacked) {
+                        tmem_ld16(d_tmem + (uint32_t)(NB + c0), v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+                        for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+                    }
                 }
-                const float *mv = mval + (c0 / (16 * NEG)) * 16;
                 if (MODE == MODE_UP) {
-                    float z[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) z[i] = acc[i] * (cscale * mv[i]) + bias;
-                    __half *hout = reinterpret_cast<__half *>(p.out);
-                    const int jrow = t.mb * 64 + 16 * q + (lane & 15);
+                    // SwiGLU: lanes < 16 hold gate rows, lanes >= 16 the linear rows of the
+                    // same h rows; lanes < 16 finish columns 0..7, lanes >= 16 columns 8..15
+                    const int half = lane >> 4;
+                    float hv[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float send = lane < 16 ? z[8 + i] : z[i];
+                        const float send = lane < 16 ? acc[8 + i] + bias : acc[i] + bias;
                         const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-                        const float gate = lane < 16 ? z[i] : recv;
-                        const float lin = lane < 16 ? recv : z[8 + i];
-                        const int col = c0 + (lane < 16 ? i : 8 + i);
+                        const float gate = lane < 16 ? acc[i] + bias : recv;
+                        const float lin = lane < 16 ? recv : acc[8 + i] + bias;
                         const float g = fminf(gate, 7.0f);
                         const float u = fminf(fmaxf(lin, -7.0f), 7.0f);
-                        const float h = __fdividef(g, 1.0f + __expf(-1.702f * g)) * (u + 1.0f);
-                        if (col < t.n_valid)
-                            hout[((size_t)t.mb * p.b_rows_total + t.p0 + col) * 64 + (jrow - t.mb * 64)] =
-                                __float2half_rn(h);
+                        hv[i] = __fdividef(g, 1.0f + __expf(-1.702f * g)) * (u + 1.0f);
+                    }
+                    // block maxima over the 32 h rows of warps q and q^1 (one 32-block of F)
+                    float m[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float a = fabsf(hv[i]);
+                        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+                        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+                        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+                        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+                        m[i] = a;
+                    }
+                    float *ex = amax_s + (eg * 2 + chunk_par) * 4 * 16;     // [4 warps][16 columns]
+                    if ((lane & 15) < 8) {
+                        float mine = m[0];
+#pragma unroll
+                        for (int i = 1; i < 8; ++i)
+                            if ((lane & 7) == i) mine = m[i];
+                        ex[q * 16 + half * 8 + (lane & 7)] = mine;
+                    }
+                    // all four warps of the group have written their maxima (bounded wait)
+                    __syncwarp();
+                    mbar_arrive_w(&ex_bar[eg * 2 + chunk_par]);
+                    if (!__all_sync(0xffffffffu, mbar_wait(&ex_bar[eg * 2 + chunk_par], (ex_ph >> chunk_par) & 1u, wc))) {
+                        ok = false;
+                        break;
+                    }
+                    ex_ph ^= 1u << chunk_par;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], ex[(q ^ 1) * 16 + half * 8 + i]);
+                    chunk_par ^= 1;
+                    const int j = t.mb * 64 + 16 * q + (lane & 15);     // h row (F index)
+                    const int fblk = j >> 5;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int col = c0 + half * 8 + i;
+                        const int s_hi = e4m3_block_exp(m[i]);
+                        const int s_lo = max(s_hi - 4, -126);
+                        const float v = hv[i];
+                        const uint32_t qh = f32x2_to_e4m3x2(v * pow2f(-s_hi), 0.0f) & 0xFFu;
+                        const float res = v - e4m3_to_f32(qh) * pow2f(s_hi);
+                        const uint32_t ql = f32x2_to_e4m3x2(res * pow2f(-s_lo), 0.0f) & 0xFFu;
+                        if (col < t.n_valid) {
+                            const size_t prow = (size_t)(t.p0 + col);
+                            p.h_q[prow * p.Kf + j] = (uint8_t)qh;
+                            p.h_q[((size_t)p.P_max + prow) * p.Kf + j] = (uint8_t)ql;
+                            if ((q & 1) == 0 && (lane & 15) == 0) {
+                                // one lane per (column, 32-block): the two scale bytes
+                                const size_t wi = (size_t)(fblk >> 2) * 2 * p.P_max;
+                                p.h_sf[(wi + prow) * 4 + (fblk & 3)] = (uint8_t)(s_hi + 127);
+                                p.h_sf[(wi + p.P_max + prow) * 4 + (fblk & 3)] = (uint8_t)(s_lo + 127);
+                            }
+                        }
                     }
                 } else {
                     // weighted expert output w * (W2 h + b2), one expert-sorted row per column
-                    float *o = reinterpret_cast<float *>(p.out);
                     if (row_valid) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             if (c0 + i < t.n_valid)
-                                o[(size_t)(t.p0 + c0 + i) * p.out_ld + row] = (acc[i] * cscale + bias) * mv[i];
+                                p.out_rows[(size_t)(t.p0 + c0 + i) * p.R + wrow] = (acc[i] + bias) * mval[c0 + i];
                     }
                 }
             }
+            if (!ok) break;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&d_empty[db]);
-            if (++db == p.n_d_bufs) { db = 0; dph ^= 1; }
+            if (++db == 2) { db = 0; dph ^= 1; }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 3) {
+    if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -582,10 +512,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 
 template __global__ void expert_gemm_kernel<MODE_UP>(const __grid_constant__ GemmParams p);
 template __global__ void expert_gemm_kernel<MODE_DOWN>(const __grid_constant__ GemmParams p);
-
-}  // namespace moe
-
-namespace moe {
 
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s) {
     if (mode == MODE_UP) {

@@ -28,115 +28,100 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// u8 codes [E][R][K/2]: box {128 bytes, box_rows, 1}, 128-byte swizzle, zero fill out of range.
-inline bool encode_codes(CUtensorMap *m, const void *codes, int E, int R, int K, int box_rows) {
+// E2M1 codes of W13 (u8 [E][2F][K/2]) for the gate/up GEMM, unpacked by TMA
+// to one byte per element in shared memory.  A 5-D view whose box is 16 gate
+// rows, their 16 linear rows, then the next group of 16 of each, four times:
+// shared row 32q + l holds gate row 16q + l (l < 16) or linear row 16q + l - 16
+// of the 64-row block, so each gate row and its linear partner land in one warp's
+// TMEM lanes.  Only the first K_main (multiple of 128) columns are mapped.
+inline bool encode_a_up(CUtensorMap *m, const void *codes, int E, int F, int K, int K_main) {
     EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)R, (cuuint64_t)E};
-    const cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R * (K / 2)};
-    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, es,
+    if (!f || K_main < 128) return false;
+    const cuuint64_t row = (cuuint64_t)K / 2;
+    const cuuint64_t dims[5] = {(cuuint64_t)K_main, 16, 2, (cuuint64_t)(F / 16), (cuuint64_t)E};
+    const cuuint64_t strides[4] = {row, (cuuint64_t)F * row, 16 * row, 2 * (cuuint64_t)F * row};
+    const cuuint32_t box[5] = {128, 16, 2, 4, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 5, const_cast<void *>(codes), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp16 K-blocked [cols/64][rows][64]: 3-D box {64, box_rows, box_kb}, 128-byte swizzle.
-inline bool encode_f16_blocked(CUtensorMap *m, const void *base, int rows, int cols, int box_rows, int box_kb) {
+// E2M1 codes of W2 (u8 [E][d][K/2]) for the down GEMM: box {128, 128 rows, 1};
+// rows past d read as zero.
+inline bool encode_a_down(CUtensorMap *m, const void *codes, int E, int d, int K, int K_main) {
     EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)rows * 128};
-    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_kb};
+    if (!f || K_main < 128) return false;
+    const cuuint64_t row = (cuuint64_t)K / 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)K_main, (cuuint64_t)d, (cuuint64_t)E};
+    const cuuint64_t strides[2] = {row, (cuuint64_t)d * row};
+    const cuuint32_t box[3] = {128, 128, 1};
     const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(codes), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// Two-term E4M3 B operand u8 [rows][Kpad] (hi plane rows then lo plane rows):
+// box {128 bytes, box_rows}, 128-byte swizzle, zero fill past the last row.
+inline bool encode_bq(CUtensorMap *m, const void *base, int rows, int Kpad, int box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)Kpad, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)Kpad};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int round_up_128(int v) { return (v + 127) / 128 * 128; }
 
 // Token rows per GEMM work item.  Decode-sized batches (T <= 64) use blocks of
-// 16 rows: experts then rarely hold more than one block, and the small
-// accumulators leave TMEM to the A slots; an expert with more tokens takes
-// extra blocks whose weight re-reads hit L2.  Larger batches use the smallest
-// multiple of 16 that holds every token (an expert receives each token at
-// most once), capped at 256.
+// 16 rows: experts then rarely hold more than one block and the accumulator
+// stays small; an expert with more tokens takes extra blocks whose weight
+// re-reads hit L2.  Larger batches use the smallest multiple of 16 that holds
+// every token (an expert receives each token at most once), capped at
+// GEMM_NB_MAX.
 inline int token_block_rows(int T) {
     if (T <= 64) return 16;
     int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;
-    return nb < 256 ? nb : 256;
+    return nb < GEMM_NB_MAX ? nb : GEMM_NB_MAX;
 }
 
-// Rows per B TMA box: the whole token block up to 64 rows (a TMA instruction
-// holds its issuing thread ~100+ cycles, so fewer, larger boxes).  When one
-// box holds the whole token block it also spans four 64-K blocks.
-inline int b_box_rows(int nb_rows) { return nb_rows < 64 ? nb_rows : 64; }
-inline int b_unit(int nb_rows) { return nb_rows <= 64 ? 4 : 1; }
-
-// Shapes, ring depths, MMA warps and the TMEM split of one grouped GEMM
-// launch for T tokens; fills everything of p except the pointers and the
-// tensor maps.  Returns MOE_ERR_ARG when the plan does not fit.
+// Shapes, ring depth and TMEM split of one grouped GEMM launch for T tokens;
+// fills everything of p except the pointers and the tensor maps.  Returns
+// MOE_ERR_ARG when the plan does not fit.
 inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, int E, int P_max, int num_sms,
                      int *grid, int *smem) {
     p.nb_rows = token_block_rows(T);
-    p.b_box_rows = b_box_rows(p.nb_rows);
-    p.b_unit = b_unit(p.nb_rows);
+    // small token blocks: one MMA over the hi rows and the lo rows together
+    p.stacked = p.nb_rows <= 64 ? 1 : 0;
     if (mode == MODE_UP) {
         p.K = d;
         p.R = 2 * F;
         p.MB = F / 64;
-        p.out_ld = F;
     } else {
         p.K = F;
         p.R = d;
         p.MB = (d + GEMM_BM - 1) / GEMM_BM;
-        p.out_ld = d;
     }
+    p.K_main = p.K / GEMM_KS * GEMM_KS;
     p.F = F;
     p.E = E;
-    p.b_stage_bytes = (p.nb_rows + p.b_box_rows - 1) / p.b_box_rows * p.b_box_rows * 128;
-    p.b_rows_total = P_max;
-    const int b_slot = p.b_unit * p.b_stage_bytes;
-    // MMA warps: a tcgen05.mma holds its issuing thread ~120 cycles, so small
-    // token blocks use up to three issuers (each its own accumulator)
-    const int n_sub = p.K / GEMM_KA;
-    const int n_chunks = (n_sub + 1) / 2;              // decoder chunks of two sub-stages per work item
-    int ni = 256 / p.nb_rows;
-    if (ni > GEMM_ISS_MAX) ni = GEMM_ISS_MAX;
-    if (ni < 1) ni = 1;
-    // decoder groups: three when several MMA warps share the work (small token
-    // blocks, decode is the scarce resource), else two; never more groups than
-    // chunks per work item, and never more MMA warps than groups, so every MMA
-    // warp gets a chunk of every work item
-    int ng = ni >= 2 ? 3 : 2;
-    if (ng > n_chunks) ng = n_chunks;
-    if (ni > ng) ni = ng;
-    p.n_iss = ni;
-    p.n_dec_groups = ng;
-    p.n_d_bufs = (2 * ni * p.nb_rows <= 256) ? 2 : 1;
-    // TMEM: A slots first, then the accumulators
-    p.n_a_slots = (512 - p.n_d_bufs * ni * p.nb_rows) / 32;
-    if (p.n_a_slots > GEMM_NA_MAX) p.n_a_slots = GEMM_NA_MAX;
-    p.n_a_slots &= ~1;
-    if (p.n_a_slots / 2 < p.n_dec_groups) return MOE_ERR_ARG;   // every decoder group owns a slot pair
-    // shared memory: up to 8 code stages next to the B ring, then whatever is
-    // left goes to the code ring
-    const GemmSmem fixed = gemm_smem_plan(p.K, E, 0, p.n_a_slots, 0, b_slot);
-    const int room = GEMM_SMEM_LIMIT - fixed.total - 8 * 2 * (GEMM_SC_MAX + 16);
-    // B fills of 4 sub-stages are shared by two decoder/MMA pipelines and must
-    // run well ahead of both: up to 8 of them (32 sub-stages); per-sub-stage
-    // fills (large token blocks) up to 16
-    int nbs = p.b_unit == 4 ? 8 : 16, sc = 8;
-    const int nbs_min = p.b_unit == 4 ? 2 : 3;
-    while (sc * GEMM_CODE_STAGE + nbs * b_slot > room && sc > 6) --sc;
-    while (sc * GEMM_CODE_STAGE + nbs * b_slot > room && nbs > nbs_min) --nbs;
-    while (sc * GEMM_CODE_STAGE + nbs * b_slot > room && sc > 4) --sc;
-    while ((sc + 1) * GEMM_CODE_STAGE + nbs * b_slot <= room && sc < GEMM_SC_MAX) ++sc;
-    if (sc * GEMM_CODE_STAGE + nbs * b_slot > room) return MOE_ERR_ARG;
-    p.n_b_stages = nbs;
-    p.n_c_stages = sc;
-    const GemmSmem plan = gemm_smem_plan(p.K, E, p.n_c_stages, p.n_a_slots, p.n_b_stages, b_slot);
-    if (plan.total > GEMM_SMEM_LIMIT) return MOE_ERR_ARG;
-    *smem = plan.total;
+    p.P_max = P_max;
+    p.Kf = round_up_128(F);
+    // as many stages as shared memory and TMEM hold
+    int ns = GEMM_STAGES_MAX;
+    while (ns > 2 && (gemm_smem_plan(p.K, E, p.nb_rows, ns).total > GEMM_SMEM_LIMIT ||
+                      gemm_tmem_cols(p.nb_rows, p.stacked, ns) > 512))
+        --ns;
+    if (gemm_smem_plan(p.K, E, p.nb_rows, ns).total > GEMM_SMEM_LIMIT ||
+        gemm_tmem_cols(p.nb_rows, p.stacked, ns) > 512)
+        return MOE_ERR_ARG;
+    p.n_stages = ns;
+    *smem = gemm_smem_plan(p.K, E, p.nb_rows, ns).total;
     const long long P = (long long)T * top_k;
     const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
     const long long max_work = (long long)p.MB * max_blocks;

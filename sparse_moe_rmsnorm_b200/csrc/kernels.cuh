@@ -42,84 +42,91 @@ struct GroupParams {
     unsigned int *err;
 };
 
-// Grouped MXFP4 x fp16 GEMM over (expert, 128-row weight block, token block)
-// work items.  MODE_UP: rows are the gate/linear pairs of W13, epilogue is the
-// clamped SwiGLU into h.  MODE_DOWN: rows are W2's, epilogue writes the
-// routing-weighted expert output rows.
+// Grouped block-scaled GEMM over (expert, 128-row weight block, token block)
+// work items: MXFP4 weights (E2M1 codes, E8M0 block scales) times the
+// activations held as two E4M3 terms (hi + lo, each with its own E8M0 block
+// scales), fp32 accumulation in TMEM.  MODE_UP: rows are the gate/linear pairs
+// of W13, epilogue is the clamped SwiGLU, written as the down GEMM's two-term
+// B.  MODE_DOWN: rows are W2's, epilogue writes the routing-weighted expert
+// output rows.
 enum { MODE_UP = 0, MODE_DOWN = 1 };
 
 struct GemmParams {
-    CUtensorMap map_codes;      // u8 [E][R][K/2], box {128 bytes, 64 (UP) or 128 (DOWN) rows, 1}, 128B swizzle
-    CUtensorMap map_b;          // fp16 expert-sorted B, K-blocked [K/64][P_max][64]; 3-D box {64, b_box_rows, b_unit}
+    CUtensorMap map_a;          // E2M1 codes, 16 x 4-bit per 16 bytes in shared memory (unpacked TMA type);
+                                //   UP: 5-D {K_main, 16 rows, 2 halves, F/16 groups, E}, box {128, 16, 2, 4, 1}
+                                //   DOWN: 3-D {K_main, d, E}, box {128, 128, 1}
+    CUtensorMap map_b;          // u8 [2 * P_max][Kpad] E4M3 hi plane then lo plane; box {128, nb_rows}
+    const uint8_t *codes;       // u8 [E][R][K/2] (the K tail is read directly)
     const uint8_t *scales;      // u8 [E][R][K/32]
     const uint16_t *bias;       // bf16 [E][R]
-    int K;                      // reduction length
+    const uint32_t *b_sf;       // [Kpad/128][2][P_max] words: E8M0 scales of 4 consecutive 32-blocks of B
+    int K;                      // reduction length (multiple of 64)
+    int K_main;                 // K rounded down to a multiple of 128 (TMA-loaded part)
     int R;                      // rows per expert: 2F (UP) or d (DOWN)
     int F;                      // d_ff (UP: gate rows [0,F), linear rows [F,2F))
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
-    int nb_rows;                // token rows per work item (multiple of 16, <= 256)
-    int b_box_rows;             // rows per B TMA box (16..64)
-    int b_unit;                 // sub-stages (64-K blocks) per B ring slot: 4 when one box holds the token block, else 1
-    int n_b_stages;             // B ring depth (slots)
-    int b_stage_bytes;          // bytes of one sub-stage block in a slot: round_up(nb_rows, b_box_rows) * 128
-    int b_rows_total;           // P_max: rows of the K-blocked B and h buffers
-    int n_c_stages;             // code ring depth (shared-memory stages of 128 rows x 128 bytes)
-    int n_a_slots;              // TMEM A slots (32 columns each); accumulators follow them
-    int n_iss;                  // MMA-issuing warps, each with its own accumulator
-    int n_dec_groups;           // decoder warp groups, 1..3 (with 3, warps 16-19 decode and one epilogue group remains)
-    int n_d_bufs;               // accumulator buffer sets (1 or 2)
+    int nb_rows;                // token rows per work item (multiple of 16, <= GEMM_NB_MAX)
+    int stacked;                // 1: one MMA covers the hi and lo rows (N = 2 nb_rows); 0: one MMA per term
+    int n_stages;               // shared-memory / TMEM scale-factor ring depth
+    int P_max;                  // rows of each B plane
     const int *counts, *offsets, *tiles;
     const int *row_token;       // [P]
     const float *row_w;         // [P]
-    const float *rho;           // [T] (UP)
-    void *out;                  // UP: fp16 h [P][F]; DOWN: fp32 weighted outputs [P][d]
-    int out_ld;                 // F (UP) or d (DOWN)
+    // UP output: the down GEMM's B (two E4M3 planes [2][P_max][Kf]) and its scales
+    uint8_t *h_q;
+    uint8_t *h_sf;              // bytes of [Kf/128][2][P_max] words
+    int Kf;                     // F rounded up to 128
+    // DOWN output: fp32 weighted rows [P][d]
+    float *out_rows;
     unsigned int *err;
     unsigned long long wait_limit_ns;
 };
 
-constexpr int GEMM_THREADS = 672;     // 21 warps
+constexpr int GEMM_THREADS = 512;     // 16 warps
 constexpr int GEMM_BM = 128;          // weight rows per work item (TMEM lanes)
-constexpr int GEMM_KS = 256;          // K elements per code stage: 128 bytes per row
-constexpr int GEMM_KA = 64;           // K elements per TMEM A slot: 32 columns
-constexpr int GEMM_SC_MAX = 10;       // code stages, at most
-constexpr int GEMM_NA_MAX = 14;       // TMEM A slots, at most
-constexpr int GEMM_NB_MAX = 256;      // token rows per work item, at most
-constexpr int GEMM_ISS_MAX = 3;       // MMA-issuing warps, at most
-constexpr int GEMM_CODE_STAGE = GEMM_BM * 128;
+constexpr int GEMM_KS = 128;          // K elements per stage (4 MMAs of K = 32)
+constexpr int GEMM_NB_MAX = 192;      // token rows per work item, at most
+constexpr int GEMM_STAGES_MAX = 12;
+constexpr int GEMM_A_STAGE = GEMM_BM * 128;   // unpacked E2M1: one byte per element in shared memory
+constexpr int GEMM_SF_COLS = 24;      // TMEM columns per scale-factor slot: A at +0, B hi at +8, B lo at +16
 constexpr int GEMM_SMEM_LIMIT = 227 * 1024;
 
 // Shared-memory plan of the GEMM kernel (all offsets from a 1024-aligned base).
 struct GemmSmem {
-    int code_off, b_off, scale_off, meta_off, tok_off, shift_off, bar_off, misc_off, total;
+    int a_off, b_off, scale_off, amax_off, meta_off, bar_off, misc_off, total;
 };
 
 __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline int gemm_num_barriers(int n_c_stages, int n_a_slots, int n_b_stages) {
-    // code full/empty, scale full/empty, A full/empty, B full/empty, D full/empty,
-    // row-shift full/empty, one drain barrier per MMA warp
-    return 2 * n_c_stages + 4 + 2 * n_a_slots + 2 * n_b_stages + 4 + 4 + GEMM_ISS_MAX;
+__host__ __device__ inline int gemm_num_barriers(int n_stages) {
+    // stage full/empty, A-scale full/empty, D full/empty, drain, epilogue exchange [2][2]
+    return 2 * n_stages + 4 + 4 + 1 + 4;
 }
 
-// b_slot_bytes = b_unit * b_stage_bytes
-__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int n_c_stages, int n_a_slots, int n_b_stages,
-                                                    int b_slot_bytes) {
+__host__ __device__ inline int gemm_b_stage_bytes(int nb_rows) { return 2 * nb_rows * 128; }
+
+__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int n_stages) {
     GemmSmem s;
-    s.code_off = 0;
-    s.b_off = n_c_stages * GEMM_CODE_STAGE;
-    s.scale_off = s.b_off + n_b_stages * b_slot_bytes;
+    s.a_off = 0;
+    s.b_off = n_stages * GEMM_A_STAGE;
+    s.scale_off = s.b_off + n_stages * gemm_b_stage_bytes(nb_rows);
     const int scale_bytes = align_up(GEMM_BM * (K / 32), 128);
-    s.meta_off = s.scale_off + 2 * scale_bytes;
-    s.tok_off = s.meta_off + 8 * (GEMM_NB_MAX / 2) * 4;         // per epilogue warp: one value per its columns
-    s.shift_off = s.tok_off + GEMM_NB_MAX * 4;                  // producer's token list of the work item
-    s.bar_off = s.shift_off + 2 * GEMM_BM * 4;
-    s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_c_stages, n_a_slots, n_b_stages) * 8, 16);
+    s.amax_off = s.scale_off + 2 * scale_bytes;
+    s.meta_off = s.amax_off + 2 * 2 * 4 * 16 * 4;                 // [2 groups][2 parities][4 warps][16 columns] fp32
+    s.bar_off = s.meta_off + 8 * GEMM_NB_MAX * 4;                  // per epilogue warp: one value per column
+    s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_stages) * 8, 16);
     // misc: tmem base, abort flag, then counts/offsets/tiles caches
     s.total = s.misc_off + 16 + 3 * (E + 1) * 4;
     s.total = align_up(s.total, 128) + 1024;  // slack for aligning the base
     return s;
+}
+
+// TMEM columns of the plan: accumulators (2 buffers) first, then the ring of
+// scale-factor slots.
+__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 2 * nb_rows : nb_rows; }
+__host__ __device__ inline int gemm_tmem_cols(int nb_rows, int stacked, int n_stages) {
+    return 2 * gemm_d_cols(nb_rows, stacked) + GEMM_SF_COLS * n_stages;
 }
 
 }  // namespace moe

@@ -29,8 +29,8 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
-                           cudaStream_t s);
+cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
+                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
@@ -41,7 +41,7 @@ using namespace moe;
 namespace {
 
 // 8 MiB of scratch: enough for decode-sized batches of the gpt-oss layers
-// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 6.3 MiB).
+// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 4.8 MiB).
 constexpr size_t kScratchBytes = 8u << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -53,6 +53,7 @@ int g_num_sms[kMaxDevices];
 size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
 
 bool a16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool a32(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Device address of the scratch array on the current device (set up once per device).
 int scratch_for_current_device(unsigned char **ptr, int *num_sms) {
@@ -75,27 +76,33 @@ int scratch_for_current_device(unsigned char **ptr, int *num_sms) {
 
 // The grouped GEMM launch of one expert stage on scratch-backed buffers.
 int launch_gemm_stage(int mode, int T, int k, int d, int F, int E, int num_sms, const uint8_t *codes,
-                      const uint8_t *scales, const uint16_t *bias, const CUtensorMap *map_b, const int *counts,
-                      const int *offsets, const int *tiles, const int *row_token, const float *row_w,
-                      const float *rho, void *out, unsigned int *err, cudaStream_t stream) {
+                      const uint8_t *scales, const uint16_t *bias, const CUtensorMap *map_b, const uint32_t *b_sf,
+                      const int *counts, const int *offsets, const int *tiles, const int *row_token,
+                      const float *row_w, uint8_t *h_q, uint32_t *h_sf, float *out_rows, unsigned int *err,
+                      cudaStream_t stream) {
     GemmParams p;
     memset(&p, 0, sizeof p);
     int grid = 0, smem = 0;
     int rc = plan_gemm(p, mode, T, k, d, F, E, T * k, num_sms, &grid, &smem);
     if (rc) return rc;
-    if (!encode_codes(&p.map_codes, codes, E, mode == MODE_UP ? 2 * F : d, mode == MODE_UP ? d : F,
-                      mode == MODE_UP ? 64 : 128))
-        return MOE_ERR_CUDA;
+    if (p.K_main >= 128) {
+        const bool ok = mode == MODE_UP ? encode_a_up(&p.map_a, codes, E, F, d, p.K_main)
+                                        : encode_a_down(&p.map_a, codes, E, d, F, p.K_main);
+        if (!ok) return MOE_ERR_CUDA;
+    }
     p.map_b = *map_b;
-    p.out = out;
+    p.codes = codes;
     p.scales = scales;
     p.bias = bias;
+    p.b_sf = b_sf;
     p.counts = counts;
     p.offsets = offsets;
     p.tiles = tiles;
     p.row_token = row_token;
     p.row_w = row_w;
-    p.rho = rho;
+    p.h_q = h_q;
+    p.h_sf = reinterpret_cast<uint8_t *>(h_sf);
+    p.out_rows = out_rows;
     p.err = err;
     p.wait_limit_ns = 2000000000ull;
     return launch_expert_gemm(mode, p, grid, smem, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -115,14 +122,17 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     if (d < 64 || d > 6144 || d % 64 || F < 64 || F > 6144 || F % 64) return MOE_ERR_ARG;
     if (E < 1 || E > 256 || k < 1 || k > 8 || k > E || !(eps >= 0.0f)) return MOE_ERR_ARG;
     if (T == 0) return MOE_OK;
-    if (!a16(x) || !a16(router_w) || !a16(router_b) || !a16(w13_codes) || !a16(w13_scales) || !a16(b13) ||
-        !a16(w2_codes) || !a16(w2_scales) || !a16(b2) || !a16(norm_scale) || !a16(y) || y == x)
+    if (!a16(x) || !a16(router_w) || !a16(router_b) || !a32(w13_codes) || !a16(w13_scales) || !a16(b13) ||
+        !a32(w2_codes) || !a16(w2_scales) || !a16(b2) || !a16(norm_scale) || !a16(y) || y == x)
         return MOE_ERR_ARG;
 
     // carve the scratch; reject shapes that do not fit
     const size_t P = (size_t)T * k;
+    const int Kd = round_up_128(d), Kf = round_up_128(F);
     const size_t sizes[] = {(size_t)T * d * 2, (size_t)T * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
-                            (size_t)(E + 1) * 4, P * 4, P * 4, P * 4, P * d * 2, P * F * 2, P * d * 4, 64};
+                            (size_t)(E + 1) * 4, P * 4, P * 4, P * 4,
+                            2 * P * Kd, (size_t)(Kd / 128) * 2 * P * 4, 2 * P * Kf, (size_t)(Kf / 128) * 2 * P * 4,
+                            P * d * 4, 64};
     size_t total = 0;
     for (size_t v : sizes) total += r256(v);
     if (total > kScratchBytes) return MOE_ERR_ARG;
@@ -146,16 +156,17 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     int *row_token = reinterpret_cast<int *>(ptrs[7]);
     float *row_w = reinterpret_cast<float *>(ptrs[8]);
     int *pair_row = reinterpret_cast<int *>(ptrs[9]);
-    __half *xperm = reinterpret_cast<__half *>(ptrs[10]);
-    __half *h = reinterpret_cast<__half *>(ptrs[11]);
-    float *orows = reinterpret_cast<float *>(ptrs[12]);
-    unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[13]);
+    uint8_t *xq = reinterpret_cast<uint8_t *>(ptrs[10]);
+    uint32_t *xsf = reinterpret_cast<uint32_t *>(ptrs[11]);
+    uint8_t *hq = reinterpret_cast<uint8_t *>(ptrs[12]);
+    uint32_t *hsf = reinterpret_cast<uint32_t *>(ptrs[13]);
+    float *orows = reinterpret_cast<float *>(ptrs[14]);
+    unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[15]);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nb = token_block_rows(T);
-    CUtensorMap map_xperm, map_h;
-    if (!encode_f16_blocked(&map_xperm, xperm, (int)P, d, b_box_rows(nb), b_unit(nb)) ||
-        !encode_f16_blocked(&map_h, h, (int)P, F, b_box_rows(nb), b_unit(nb)))
+    CUtensorMap map_xq, map_hq;
+    if (!encode_bq(&map_xq, xq, 2 * (int)P, Kd, nb) || !encode_bq(&map_hq, hq, 2 * (int)P, Kf, nb))
         return MOE_ERR_CUDA;
     // the error word is the one buffer that must start at zero on every call
     if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -191,13 +202,14 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.pair_row = pair_row;
     gp.err = err;
     if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_permute(xn16, row_token, xperm, (int)P, (int)P, d, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_quant_permute(xn16, rho, row_token, xq, xsf, (int)P, (int)P, d, Kd, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
 
-    rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xperm, counts,
-                           offsets, tiles, row_token, row_w, rho, h, err, s);
+    rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xq, xsf, counts,
+                           offsets, tiles, row_token, row_w, hq, hsf, orows, err, s);
     if (rc) return rc;
-    rc = launch_gemm_stage(MODE_DOWN, T, k, d, F, E, num_sms, w2_codes, w2_scales, b2, &map_h, counts, offsets,
-                           tiles, row_token, row_w, rho, orows, err, s);
+    rc = launch_gemm_stage(MODE_DOWN, T, k, d, F, E, num_sms, w2_codes, w2_scales, b2, &map_hq, hsf, counts,
+                           offsets, tiles, row_token, row_w, hq, hsf, orows, err, s);
     if (rc) return rc;
     return launch_combine(x, orows, pair_row, y, T, d, k, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

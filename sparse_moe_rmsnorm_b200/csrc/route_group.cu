@@ -3,7 +3,8 @@
 //                    plus the fp16 normalised tokens for the experts;
 //   group_kernel     expert histogram, exclusive scan and a stable permutation
 //                    of the (token, expert) pairs into expert-contiguous rows;
-//   permute_kernel   the expert-sorted copy of the normalised tokens;
+//   quant_permute_kernel  the expert-sorted two-term E4M3 copy of the normalised
+//                    tokens (the gate/up GEMM's B operand);
 //   combine_kernel   y = x + the token's weighted expert rows, in bf16.
 #include <cfloat>
 #include <climits>
@@ -385,21 +386,82 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
     }
 }
 
-// --------------------------------------------------------------- permute
+// --------------------------------------------------------------- permute + quantise
 //
-// The normalised tokens in expert-sorted row order, K-blocked:
-// xperm[kb][r][0:64] = xn16[row_token[r]][64 kb : 64 kb + 64] for r < P, with
-// P_max rows per block, so one 3-D TMA box reads several 64-K blocks of a
-// run of rows.  One warp per row, 16-byte copies.
-__global__ void __launch_bounds__(256) permute_kernel(const __half *__restrict__ xn16, const int *__restrict__ row_token,
-                                                      __half *__restrict__ xperm, int P, int P_max, int d) {
+// Row r (< P) of the gate/up GEMM's B operand: the normalised activations of
+// token row_token[r], v = xn16 * rho, as two E4M3 terms per 32-element block
+// with E8M0 scale s (the exponent that fits the block maximum to 448):
+//   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)).
+// Out: xq[plane][r][0:Kd] (plane 0 hi, plane 1 lo; columns d..Kd zero) and
+// xsf[g][plane][r] = the scale bytes of the 32-blocks 4g..4g+3 (byte i is
+// block 4g+i).  One warp per row; lane l takes the 32-blocks l, l+32, ...
+__global__ void __launch_bounds__(256, 1) quant_permute_kernel(const __half *__restrict__ xn16,
+                                                            const float *__restrict__ rho,
+                                                            const int *__restrict__ row_token,
+                                                            uint8_t *__restrict__ xq, uint32_t *__restrict__ xsf,
+                                                            int P, int P_max, int d, int Kd) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nblk = d / 32, nblk_pad = Kd / 32;
     for (int r = warp; r < P; r += nwarps) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(xn16 + (size_t)row_token[r] * d);
-        for (int j = lane; j < d / 8; j += 32) {
-            const int kb = j >> 3;
-            reinterpret_cast<uint4 *>(xperm + ((size_t)kb * P_max + r) * 64)[j & 7] = src[j];
+        const int tok = row_token[r];
+        const float sc = rho[tok];
+        const uint4 *src = reinterpret_cast<const uint4 *>(xn16 + (size_t)tok * d);
+        for (int b0 = 0; b0 < nblk_pad; b0 += 32) {
+            const int b = b0 + lane;
+            uint32_t s_hi = 127, s_lo = 127;
+            uint32_t qh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ql[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (b < nblk) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 u = src[4 * b + i];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t wk = k == 0 ? u.x : (k == 1 ? u.y : (k == 2 ? u.z : u.w));
+                        v[8 * i + 2 * k] = __half2float(__ushort_as_half((unsigned short)(wk & 0xFFFFu))) * sc;
+                        v[8 * i + 2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(wk >> 16))) * sc;
+                    }
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                const int e_hi = e4m3_block_exp(amax);
+                const int e_lo = max(e_hi - 4, -126);
+                const float inv_hi = pow2f(-e_hi), inv_lo = pow2f(-e_lo), mul_hi = pow2f(e_hi);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t h = f32x2_to_e4m3x2(v[2 * i] * inv_hi, v[2 * i + 1] * inv_hi);
+                    float d0, d1;
+                    e4m3x2_to_f32x2(h, d0, d1);
+                    const uint32_t l = f32x2_to_e4m3x2((v[2 * i] - d0 * mul_hi) * inv_lo,
+                                                       (v[2 * i + 1] - d1 * mul_hi) * inv_lo);
+                    qh[i >> 1] |= h << (16 * (i & 1));
+                    ql[i >> 1] |= l << (16 * (i & 1));
+                }
+                s_hi = (uint32_t)(e_hi + 127);
+                s_lo = (uint32_t)(e_lo + 127);
+            }
+            if (b < nblk_pad) {
+                uint4 *dh = reinterpret_cast<uint4 *>(xq + (size_t)r * Kd + 32 * b);
+                uint4 *dl = reinterpret_cast<uint4 *>(xq + ((size_t)P_max + r) * Kd + 32 * b);
+                dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
+                dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
+                dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
+                dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
+            }
+            // the scale bytes of four consecutive blocks (lanes 4m..4m+3) as one word
+            uint32_t wh = s_hi, wl = s_lo;
+#pragma unroll
+            for (int i = 1; i < 4; ++i) {
+                wh |= __shfl_down_sync(0xffffffffu, s_hi, i) << (8 * i);
+                wl |= __shfl_down_sync(0xffffffffu, s_lo, i) << (8 * i);
+            }
+            if ((lane & 3) == 0 && b < nblk_pad) {
+                const size_t g = (size_t)(b >> 2);
+                xsf[(g * 2) * P_max + r] = wh;
+                xsf[(g * 2 + 1) * P_max + r] = wl;
+            }
         }
     }
 }
@@ -511,11 +573,11 @@ cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_permute(const __half *xn16, const int *row_token, __half *xperm, int P, int P_max, int d,
-                           cudaStream_t s) {
+cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
+                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s) {
     if (P <= 0) return cudaSuccess;
     const int grid = min((P + 7) / 8, 148 * 8);
-    permute_kernel<<<grid, 256, 0, s>>>(xn16, row_token, xperm, P, P_max, d);
+    quant_permute_kernel<<<grid, 256, 0, s>>>(xn16, rho, row_token, xq, xsf, P, P_max, d, Kd);
     return cudaGetLastError();
 }
 

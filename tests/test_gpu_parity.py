@@ -14,12 +14,15 @@ import oracle
 import sparse_moe_rmsnorm_b200 as moe
 from moe_inputs import CONFIGS, bf16_bits_to_f32, custom_layer, make_config_inputs
 from _parity import compare_block, excluded_tokens
+from _e4m3 import decode_two_term, encode_two_term, scale_bytes_from_words
 
 pytestmark = pytest.mark.gpu
 
-# Tighter bound on the fp32 accumulator y_acc (before the bf16 output cast): the fp16 rounding of
-# xn/rho and of h gives ~2e-4 mean relative error in a float64 emulation of the same rounding points.
-ACC_MEAN_REL = 1e-3
+# Tighter bound on the fp32 accumulator y_acc (before the bf16 output cast).  The expert GEMMs see
+# the activations (normalised tokens, h) as two E4M3 terms per 32-block, at most 2^-9 relative error
+# per element; a float64 emulation of those rounding points gives 1.1e-3 mean relative error on the
+# 2880-wide layers (5e-4 on small ones).  2.5e-3 leaves room for the fp32 accumulation order.
+ACC_MEAN_REL = 2.5e-3
 
 
 def _bf16_dev(a):
@@ -49,7 +52,7 @@ def run_block(inp, k, eps=1e-5, T_max=None):
     return out
 
 
-def check(inp, k, eps=1e-5, rows=None, label=""):
+def check(inp, k, eps=1e-5, rows=None, label="", acc_mean_rel=ACC_MEAN_REL):
     g = run_block(inp, k, eps)
     if rows is None:
         ref = oracle.moe_forward(inp, k, eps)
@@ -65,7 +68,8 @@ def check(inp, k, eps=1e-5, rows=None, label=""):
     print(label, res, "| fp32 accumulator:", {k_: acc[k_] for k_ in ("max_rel", "mean_rel")})
     assert res["ok"], res
     assert res["w_max_err"] < 1e-5, res
-    assert acc["mean_rel"] <= ACC_MEAN_REL, acc
+    if acc_mean_rel is not None:
+        assert acc["mean_rel"] <= acc_mean_rel, acc
     g["ctx"].close()
     return res
 
@@ -122,6 +126,19 @@ def test_decode_wide_scale_spread_bounded():
 
 # ------------------------------------------------------------ route, group
 
+def _assert_same_e4m3(got, want, what):
+    """Byte-exact E4M3 codes, except that the conversion may give -0 (0x80) where the definition
+    gives +0."""
+    got = np.asarray(got, dtype=np.uint8)
+    want = np.asarray(want, dtype=np.uint8)
+    same = (got == want) | (((got & 0x7F) == 0) & ((want & 0x7F) == 0))
+    if not same.all():
+        r, c = np.nonzero(~same)
+        print(what, "mismatches", r.size, "first", [(int(a), int(b), int(got[a, b]), int(want[a, b]))
+                                                     for a, b in zip(r[:12], c[:12])])
+    assert same.all(), what
+
+
 @pytest.mark.parametrize("T,d,E,k", [(16, 128, 8, 4), (37, 2880, 32, 4), (600, 2880, 128, 4), (2100, 256, 64, 8)])
 def test_route_stage(T, d, E, k):
     inp = custom_layer(T=T, d=d, F=64, E=E, k=k, seed=T)
@@ -165,18 +182,26 @@ def test_group_stage_invariants(T, E, k):
     row_w = m.workspace("row_w", T).cpu().numpy()
     pair_row = m.workspace("pair_row", T).cpu().numpy()
     xn16 = m.workspace("xn16", T).cpu().numpy()
+    rho = m.workspace("rho", T).cpu().numpy()
+    xq = m.workspace("xperm", T).cpu().numpy()
+    xsf = m.workspace("xsf", T).cpu().numpy()
     P = T * k
-    # the workspace holds it K-blocked: [d/64][T*k][64]
-    dd = xn16.shape[1]
-    xperm = m.workspace("xperm", T).cpu().numpy().reshape(dd // 64, P, 64).transpose(1, 0, 2).reshape(P, dd)
     assert m.sync_status() == moe.MOE_OK
-    # pair_row inverts the permutation, and the sorted token copy follows it
+    # pair_row inverts the permutation
     assert np.array_equal(np.sort(pair_row), np.arange(P))
     assert np.array_equal(row_token[pair_row], np.repeat(np.arange(T), k))
-    assert np.array_equal(xperm, xn16[row_token])
+    # the expert-sorted B operand is exactly the two-term E4M3 encoding of xn16 * rho of each row's token
+    v = (xn16[row_token].astype(np.float32) * rho[row_token][:, None]).astype(np.float32)
+    hi, lo, s_hi, s_lo = encode_two_term(v)
+    d = v.shape[1]
+    _assert_same_e4m3(xq[0, :P, :d], hi, "hi")
+    _assert_same_e4m3(xq[1, :P, :d], lo, "lo")
+    assert not xq[:, :P, d:].any()                        # K padding to a multiple of 128
+    assert np.array_equal(scale_bytes_from_words(xsf, 0, np.arange(P), d // 32), s_hi)
+    assert np.array_equal(scale_bytes_from_words(xsf, 1, np.arange(P), d // 32), s_lo)
     assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
     assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts) and offsets[-1] == P
-    nb = 16 if T <= 64 else min(256, (T + 15) // 16 * 16)
+    nb = 16 if T <= 64 else min(192, (T + 15) // 16 * 16)
     assert np.array_equal(np.diff(tiles), (counts + nb - 1) // nb)
     # a stable permutation: expert-major, token-minor, every pair exactly once
     want_tok = []
@@ -203,8 +228,8 @@ SHAPES = [
     dict(T=33, d=256, F=128, E=4, k=4),          # k == E
     dict(T=9, d=64, F=64, E=1, k=1),             # a single expert: dense FFN
     dict(T=40, d=512, F=256, E=16, k=8),         # largest k
-    dict(T=300, d=128, F=192, E=2, k=1),         # n_e > 256: several token blocks per expert
-    dict(T=700, d=320, F=640, E=8, k=4),         # token blocks of 256, ragged tails
+    dict(T=300, d=128, F=192, E=2, k=1),         # n_e > 192: several token blocks per expert
+    dict(T=700, d=320, F=640, E=8, k=4),         # token blocks of 192, ragged tails
     dict(T=50, d=2880, F=2880, E=32, k=4),
 ]
 
@@ -217,15 +242,27 @@ def test_shapes(shape):
 
 
 def test_scale_extremes():
-    """E8M0 exponents far from 127 (exercises the per-row fp16 shift of the decode).
+    """E8M0 exponents far from 127, outside the layers' distribution.
 
     Exponents 100..136 on every weight; then huge W2 (140..150) behind normal W13, and tiny W13
-    (104..110).  Huge W13 is left out on purpose: it scales the gate pre-activations to ~1e7, where
-    the clamped SwiGLU is a step function of them and any rounding of the activations (fp16 here,
-    bf16 just as well) moves outputs across the step -- an exact-weight emulation in float64 with
-    fp16 activations shows the same ~4% deviation there."""
-    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=5, scale_lo=100, scale_hi=136)
-    check(inp, 2, label="scales 100..136")
+    (104..110).  The block scales reach the tensor core unchanged, so extreme exponents cost no
+    precision in the weights; the activations, though, carry 2^-9 relative rounding (two E4M3
+    terms), and with 36 binades of weight scales the few largest blocks dominate sums that partly
+    cancel.  A float64 emulation of the same rounding points gives max 0.068 / mean 0.0028 relative
+    error for the first case, so the max bound here is 0.1 and the accumulator bound is skipped;
+    the indices and the 5e-3 mean bound still hold.  (Huge W13 is left out: it scales the gate
+    pre-activations to ~1e7, where the clamped SwiGLU is a step function of them and any rounding
+    of the activations moves outputs across the step.)"""
+    def loose(inp, label):
+        g = run_block(inp, 2)
+        ref = oracle.moe_forward(inp, 2, 1e-5)
+        res = compare_block(g["y"], g["idx"], g["w"], ref, 2, inp["router_w"].shape[0])
+        print(label, res)
+        assert res["idx_mismatch"] == 0 and res["w_max_err"] < 1e-5, res
+        assert res["max_rel"] <= 0.1 and res["mean_rel"] <= 5e-3, res
+        g["ctx"].close()
+
+    loose(custom_layer(T=24, d=256, F=256, E=4, k=2, seed=5, scale_lo=100, scale_hi=136), "scales 100..136")
     rng = np.random.default_rng(7)
     inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=6)
     inp["w2_scales"] = rng.integers(140, 151, size=inp["w2_scales"].shape, dtype=np.uint8)
@@ -233,6 +270,54 @@ def test_scale_extremes():
     inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=8)
     inp["w13_scales"] = rng.integers(104, 111, size=inp["w13_scales"].shape, dtype=np.uint8)
     check(inp, 2, label="W13 scales 104..110")
+
+
+def _np_swiglu(gate, lin):
+    g = np.minimum(gate, 7.0)
+    u = np.clip(lin, -7.0, 7.0)
+    return g / (1.0 + np.exp(-1.702 * g)) * (u + 1.0)
+
+
+@pytest.mark.parametrize("T,d,F,E,k", [(16, 128, 128, 8, 4), (50, 2880, 2880, 32, 4), (300, 192, 320, 4, 2)])
+def test_up_stage_h_encoding(T, d, F, E, k):
+    """The gate/up GEMM + SwiGLU epilogue against float64 on the same (decoded) operands: h, read back
+    from its two-term E4M3 encoding, within the encoding's rounding of the float64 value (2^-9 of the
+    32-block maximum, plus the fp32 accumulation)."""
+    inp = custom_layer(T=T, d=d, F=F, E=E, k=k, seed=T + d)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(T, d, F, E, k)
+    moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
+    moe.moe_group(m.ctx, T, k)
+    moe.moe_expert_up(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13)
+    torch.cuda.synchronize()
+    assert m.sync_status() == moe.MOE_OK
+    P = T * k
+    counts = m.workspace("counts", T).cpu().numpy()
+    offsets = m.workspace("offsets", T).cpu().numpy()
+    xq = m.workspace("xperm", T).cpu().numpy()
+    xsf = m.workspace("xsf", T).cpu().numpy()
+    hq = m.workspace("h", T).cpu().numpy()
+    hsf = m.workspace("hsf", T).cpu().numpy()
+    rows = np.arange(P)
+    xb = decode_two_term(xq[0, :P, :d], xq[1, :P, :d], scale_bytes_from_words(xsf, 0, rows, d // 32),
+                         scale_bytes_from_words(xsf, 1, rows, d // 32))
+    h = decode_two_term(hq[0, :P, :F], hq[1, :P, :F], scale_bytes_from_words(hsf, 0, rows, F // 32),
+                        scale_bytes_from_words(hsf, 1, rows, F // 32))
+    W13 = oracle.decode_matrix(inp["w13_codes"].reshape(-1, d // 2), inp["w13_scales"].reshape(-1, d // 32))
+    W13 = W13.reshape(E, 2 * F, d)
+    b13 = bf16_bits_to_f32(inp["b13"]).astype(np.float64)
+    want = np.zeros((P, F))
+    for e in range(E):
+        r = slice(offsets[e], offsets[e] + counts[e])
+        z = xb[r] @ W13[e].T + b13[e]
+        want[r] = _np_swiglu(z[:, :F], z[:, F:])
+    blk_max = np.abs(want).reshape(P, F // 32, 32).max(axis=2, keepdims=True)
+    err = np.abs(h - want).reshape(P, F // 32, 32)
+    bound = 2.0 ** -8 * blk_max + 1e-5 * np.abs(want).max()
+    print("h max err / block max", float(np.max(err / np.maximum(blk_max, 1e-30))))
+    assert np.all(err <= bound)
+    m.close()
 
 
 def test_tied_logits_pick_lower_index():
