@@ -125,7 +125,7 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
             c->w13_ptr = codes;
         }
         if (!c->have_xq[bi]) {
-            if (!encode_bq(&c->map_xq[bi], c->xq, 2 * P_max, c->Kd, p.nb_rows)) return MOE_ERR_CUDA;
+            if (!encode_bq(&c->map_xq[bi], c->xq, P_max, c->Kd, p.nb_rows)) return MOE_ERR_CUDA;
             c->have_xq[bi] = true;
         }
         p.map_a = c->map_w13;
@@ -139,7 +139,7 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
             c->w2_ptr = codes;
         }
         if (!c->have_hq[bi]) {
-            if (!encode_bq(&c->map_hq[bi], c->hq, 2 * P_max, c->Kf, p.nb_rows)) return MOE_ERR_CUDA;
+            if (!encode_bq(&c->map_hq[bi], c->hq, P_max, c->Kf, p.nb_rows)) return MOE_ERR_CUDA;
             c->have_hq[bi] = true;
         }
         p.map_a = c->map_w2;

@@ -33,16 +33,20 @@
 //   row; the combine kernel adds a token's rows to its residual (weighted
 //   combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
 //
-// Warp roles (512 threads): 0 TMA producer, 1 MMA issue, 2 TMEM allocation,
-// 4-7 scale-factor warps (one per TMEM lane quarter), 8-11 and 12-15 two
-// epilogue groups taking 16-column chunks in turn.  Producer and MMA run as
-// whole converged warps, one elected lane issuing.  Every mbarrier wait is
+// Warp roles (512 threads): 0 TMA producer of A (weights), 3 TMA producer of
+// B (activations), 1 MMA issue, 2 TMEM allocation, 4-7 scale-factor warps (one
+// per TMEM lane quarter), 8-11 and 12-15 two epilogue groups taking 16-column
+// chunks in turn.  Producers and MMA run as whole converged warps, one elected
+// lane issuing.  Every mbarrier wait is
 // bounded (WaitCtl); when one runs out the CTA stops issuing work, drains its
 // copies and MMAs in flight, frees TMEM and returns with the error latched.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace moe {
+
+constexpr int SF_PD = 4;        // stages of B scale words the scale-factor warps load ahead
+constexpr int SF_WORDS = 12;    // B scale words per lane and stage, at most (6 columns x hi/lo)
 
 struct Work {
     int e, mb, p0, n_valid, n_mma;
@@ -107,7 +111,7 @@ __device__ __forceinline__ int tile_weight_row(int r, int mb, int F) {
     return mb * GEMM_BM + r;
 }
 
-template <int MODE>
+template <int MODE, bool SFI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,12 +129,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bar_off);
     uint64_t *full = bars;
     uint64_t *empty = full + NS;
-    uint64_t *s_full = empty + NS;
+    uint64_t *s_full = empty + NS;          // [2] A scale bytes of a work item in shared memory
     uint64_t *s_empty = s_full + 2;
-    uint64_t *d_full = s_empty + 2;
-    uint64_t *d_empty = d_full + 2;
-    uint64_t *drain_bar = d_empty + 2;
-    uint64_t *ex_bar = drain_bar + 1;                                     // [2 groups][2 parities]
+    uint64_t *d_full = s_empty + 2;         // [2 MMA warps][2 accumulator buffers]
+    uint64_t *d_empty = d_full + 4;         // [2]
+    uint64_t *drain_bar = d_empty + 2;      // [2 MMA warps]
+    uint64_t *ex_bar = drain_bar + 2;       // [2 groups][2 parities]
+    uint64_t *f_full = ex_bar + 4;          // [2] a work item's scale factors in TMEM (per-item mode)
+    uint64_t *f_empty = f_full + 2;
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
@@ -141,21 +147,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;     // stages per work item
     const int n_main = p.K_main / GEMM_KS;              // stages loaded by TMA; a last one past them is the K tail
     const int d_cols = gemm_d_cols(NB, p.stacked);
-    const uint32_t sf_col0 = (uint32_t)(2 * d_cols);
+    // MMA warps: two taking alternate stages in per-item mode (the second only
+    // when an item has more than one stage), one otherwise
+    const int n_mma_warps = SFI && n_st > 1 ? 2 : 1;
+    // TMEM columns: accumulators first, then the scale factors
+    const uint32_t sf_col0 = (uint32_t)((SFI ? 4 : 2) * d_cols);
+    const int sfi_cols = GEMM_SFI_COLS * n_st;           // one item region (per-item mode)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
-            mbar_init(&full[i], 1 + 4);   // producer's expect_tx arrive + the four scale-factor warps
+            // the two producers' arrivals (+ the four scale-factor warps per stage)
+            mbar_init(&full[i], SFI ? 2 : 2 + 4);
             mbar_init(&empty[i], 1);      // MMA commit
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&s_empty[i], 4);
-            mbar_init(&d_full[i], 1);
             mbar_init(&d_empty[i], 8);    // every epilogue warp
+            mbar_init(&drain_bar[i], 1);
+            mbar_init(&f_full[i], 4);     // the four scale-factor warps
+            mbar_init(&f_empty[i], n_mma_warps);
         }
-        mbar_init(drain_bar, 1);
-        for (int i = 0; i < 4; ++i) mbar_init(&ex_bar[i], 4);   // the four warps of an epilogue group
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&d_full[i], 1);
+            mbar_init(&ex_bar[i], 4);     // the four warps of an epilogue group
+        }
         *abort_s = 0;
         fence_barrier_init();
     }
@@ -177,21 +193,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                      p.wait_limit_ns};
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            if (n_main > 0) tma_prefetch_desc(&p.map_a);
-            tma_prefetch_desc(&p.map_b);
-        }
+        // ------------------------------------------------- A producer (weights)
+        // Per work item the 128 rows' E8M0 bytes (one or two untiled bulk
+        // copies), issued one item ahead so the scale-factor warps can prepare
+        // an item while the MMAs work on the one before; per stage one TMA box
+        // of E2M1 codes (128 rows x 128 K).  The K tail (K not a multiple of
+        // 128) is copied into its stage's slot here, four rows per lane.
+        if (lane == 0 && n_main > 0) tma_prefetch_desc(&p.map_a);
         int slot = 0, sb = 0;
         uint32_t ph = 0, sph = 0;
         long long issued = 0, s_issued = 0;
         bool ok = true;
-        const uint32_t b_bytes = (uint32_t)b_stage;
-        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-            Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
-            // the work item's A scales
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[sb], sph ^ 1, wc))) { ok = false; break; }
+        auto load_scales = [&](const Work &t) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[sb], sph ^ 1, wc))) return false;
             uint8_t *sdst = scale_buf + sb * scale_bytes;
             if (MODE == MODE_UP) {
                 const int j0 = t.mb * 64;
@@ -207,35 +221,106 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             }
             ++s_issued;
             if (++sb == 2) { sb = 0; sph ^= 1; }
+            return true;
+        };
+        Work t;
+        if (blockIdx.x < total) {
+            work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            ok = load_scales(t);
+        }
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work tn;
+            if (w + (int)gridDim.x < total) {
+                work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, tn);
+                if (!load_scales(tn)) { ok = false; break; }
+            }
             for (int st = 0; st < n_st; ++st) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
-                const bool has_a = st < n_main;
-                // the unpacked-type TMA counts the packed bytes: 128 rows x 64
-                mbar_arrive_expect_tx_w(&full[slot], (has_a ? 128u * 64u : 0u) + b_bytes);
-                if (has_a) {
+                uint8_t *adst = a_ring + slot * GEMM_A_STAGE;
+                if (st < n_main) {
+                    // the unpacked-type TMA counts the packed bytes: 128 rows x 64
+                    mbar_arrive_expect_tx_w(&full[slot], 128u * 64u);
                     if (MODE == MODE_UP)
-                        tma_load_5d_w(a_ring + slot * GEMM_A_STAGE, &p.map_a, &full[slot], st * GEMM_KS, 0, 0,
-                                      4 * t.mb, t.e);
+                        tma_load_5d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, 0, 0, 4 * t.mb, t.e);
                     else
-                        tma_load_3d_w(a_ring + slot * GEMM_A_STAGE, &p.map_a, &full[slot], st * GEMM_KS,
-                                      t.mb * GEMM_BM, t.e);
+                        tma_load_3d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, t.mb * GEMM_BM, t.e);
+                } else {
+                    // K tail of rows lane + 32j: 2 x 16 code bytes -> the first four
+                    // 16-byte units of the row (8 code bytes each, the rest zero),
+                    // 128-byte swizzle
+                    uint4 tail[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int wrow = tile_weight_row<MODE>(lane + 32 * j, t.mb, p.F);
+                        tail[2 * j] = tail[2 * j + 1] = make_uint4(0, 0, 0, 0);
+                        if (wrow < p.R) {
+                            const uint4 *src = reinterpret_cast<const uint4 *>(
+                                p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
+                            tail[2 * j] = __ldg(src);
+                            tail[2 * j + 1] = __ldg(src + 1);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = lane + 32 * j;
+                        uint8_t *row = adst + r * 128;
+                        const int sw = r & 7;
+                        const uint4 c0 = tail[2 * j], c1 = tail[2 * j + 1];
+                        *reinterpret_cast<uint4 *>(row + ((0 ^ sw) << 4)) = make_uint4(c0.x, c0.y, 0, 0);
+                        *reinterpret_cast<uint4 *>(row + ((1 ^ sw) << 4)) = make_uint4(c0.z, c0.w, 0, 0);
+                        *reinterpret_cast<uint4 *>(row + ((2 ^ sw) << 4)) = make_uint4(c1.x, c1.y, 0, 0);
+                        *reinterpret_cast<uint4 *>(row + ((3 ^ sw) << 4)) = make_uint4(c1.z, c1.w, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    mbar_arrive_w(&full[slot]);
                 }
-                uint8_t *bdst = b_ring + slot * b_stage;
-                tma_load_2d_w(bdst, &p.map_b, &full[slot], st * GEMM_KS, t.p0);
-                tma_load_2d_w(bdst + NB * 128, &p.map_b, &full[slot], st * GEMM_KS, p.P_max + t.p0);
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
             }
+            t = tn;
         }
         if (!ok) {
             drain_ring(full, NS, issued, p.wait_limit_ns);
             drain_ring(s_full, 2, s_issued, p.wait_limit_ns);
         }
-    } else if (warp == 1) {
+    } else if (warp == 3) {
+        // --------------------------------------------- B producer (activations)
+        // Per stage one TMA box: the token block's hi rows and then its lo rows.
+        if (lane == 0) tma_prefetch_desc(&p.map_b);
+        int slot = 0;
+        uint32_t ph = 0;
+        long long issued = 0;
+        bool ok = true;
+        const uint32_t b_bytes = (uint32_t)b_stage;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            for (int st = 0; st < n_st; ++st) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                mbar_arrive_expect_tx_w(&full[slot], b_bytes);
+                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], st * GEMM_KS, t.p0, 0);
+                ++issued;
+                if (++slot == NS) { slot = 0; ph ^= 1; }
+            }
+        }
+        if (!ok) drain_ring(full, NS, issued, p.wait_limit_ns);
+    } else if (warp == 1 || (warp == 2 && n_mma_warps == 2)) {
         // ---------------------------------------------------------------- MMA issue
-        int slot = 0, db = 0;
-        uint32_t ph = 0, dph = 0;
+        // MMA warp m takes the stages st = m, m + n_mma_warps, ... of every
+        // work item into its own accumulator pair; stage g of the CTA (counted
+        // over all items) sits in ring slot g % NS with phase parity (g / NS) & 1.
+        const int m = warp - 1;
+        int db = 0, sb = 0;
+        uint32_t dph = 0, sph = 0;
         bool ok = true, issued = false;
+        // ring slot and phase parity of the current item's first stage
+        int islot = 0;
+        uint32_t iph = 0;
+        auto advance = [&](int &sl, uint32_t &par, int by) {
+            sl += by;
+            while (sl >= NS) { sl -= NS; par ^= 1; }
+        };
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
@@ -244,41 +329,54 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             // E8M0 scales, M >> 4; the scale byte of each MMA is set per K block below
             const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
             if (!__all_sync(0xffffffffu, mbar_wait(&d_empty[db], dph ^ 1, wc))) { ok = false; break; }
+            if (SFI && !__all_sync(0xffffffffu, mbar_wait(&f_full[sb], sph, wc))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d_tmem = tmem + (uint32_t)(db * d_cols);
+            const uint32_t d_tmem = tmem + (uint32_t)((m * 2 + db) * d_cols);
+            const uint32_t sf_item = tmem + sf_col0 + (uint32_t)(sb * sfi_cols);
             uint32_t acc = 0;
-            for (int st = 0; st < n_st; ++st) {
+            int slot = islot;
+            uint32_t ph = iph;
+            advance(slot, ph, m);
+            for (int st = m; st < n_st; st += n_mma_warps) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_addr = smem_addr(a_ring + slot * GEMM_A_STAGE);
                 const uint32_t b_addr = smem_addr(b_ring + slot * b_stage);
-                const uint32_t sf = tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * st)
+                                        : tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                const uint32_t sfb = SFI ? sf + 4 : sf + 8;
                 const int nkb = st < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
                 for (int kb = 0; kb < nkb; ++kb) {
                     const uint32_t idesc = idesc0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
                     const uint64_t ad = smem_desc_sw128(a_addr + kb * 32);
-                    mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + kb * 32), idesc, sf, sf + 8, acc);
+                    mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + kb * 32), idesc, sf, sfb, acc);
                     if (!p.stacked)
                         mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + NB * 128 + kb * 32), idesc, sf, sf + 16, 1u);
                     acc = 1;
                 }
                 issued = true;
                 mma_commit_w(&empty[slot]);
-                if (++slot == NS) { slot = 0; ph ^= 1; }
+                advance(slot, ph, n_mma_warps);
             }
             if (!ok) break;
-            mma_commit_w(&d_full[db]);
+            advance(islot, iph, n_st);
+            mma_commit_w(&d_full[m * 2 + db]);
+            if (SFI) mma_commit_w(&f_empty[sb]);
             if (++db == 2) { db = 0; dph ^= 1; }
+            if (++sb == 2) { sb = 0; sph ^= 1; }
         }
         if (!ok && issued) {
-            mma_commit_w(drain_bar);
-            mbar_wait_drain(drain_bar, 0, p.wait_limit_ns);
+            mma_commit_w(&drain_bar[m]);
+            mbar_wait_drain(&drain_bar[m], 0, p.wait_limit_ns);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------ scale-factor warps
-        // Warp q writes TMEM lane quarter q: column c of a region holds, in
-        // lane 32q + i, the four E8M0 bytes (32-blocks 4st..4st+3) of row
-        // 32c + i of the operand.
+        // Warp q writes TMEM lane quarter q.  A stage's scale factors take 4-column
+        // groups: column c of the A group holds, in lane 32q + i, the four E8M0
+        // bytes (32-blocks 4st..4st+3) of weight row 32c + i; column c of the B
+        // group holds token row 32c + i (stacked: rows of [hi | lo]).  Per-item
+        // mode writes every stage of a work item into an item region once;
+        // per-stage mode writes each stage into the slot of its ring stage.
         const int q = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int slot = 0, sb = 0;
@@ -288,6 +386,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            // B scale words of stage st into v: stacked, word c is row 32c + lane of
+            // [hi rows | lo rows]; otherwise words 2c / 2c + 1 are the hi / lo word
+            // of token row 32c + lane.  Rows past the block's tokens get 2^0.
+            auto load_bsf = [&](int st, uint32_t (&v)[SF_WORDS]) {
+                const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
+#pragma unroll
+                for (int i = 0; i < SF_WORDS; ++i) v[i] = 0x7F7F7F7Fu;
+                if (p.stacked) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = 32 * c + lane;
+                        const int plane = r >= NB ? 1 : 0;
+                        const int j = r - plane * NB;
+                        if (c < n_sfb && r < 2 * NB && j < t.n_valid) v[c] = __ldg(bsf + (size_t)plane * p.P_max + j);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < SF_WORDS / 2; ++c) {
+                        const int j = 32 * c + lane;
+                        if (c < n_sfb && j < t.n_valid) {
+                            v[2 * c] = __ldg(bsf + j);
+                            v[2 * c + 1] = __ldg(bsf + p.P_max + j);
+                        }
+                    }
+                }
+            };
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
             const uint8_t *sbase = scale_buf + sb * scale_bytes;
             const uint8_t *srow[4];
@@ -297,77 +421,107 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 srow[c] = sbase + tile_scale_row<MODE>(32 * c + lane) * KB32;
                 row_ok[c] = MODE == MODE_UP || t.mb * GEMM_BM + 32 * c + lane < p.R;
             }
-            for (int st = 0; st < n_st; ++st) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
-                const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
-                // A: four columns
-                {
-                    const int nblk = KB32 - 4 * st;     // 32-blocks of this stage inside K: 2 or >= 4
-                    uint32_t v[4];
+            // A words of stage st: column c
+            auto a_words = [&](int st, uint32_t *v) {
+                const int nblk = KB32 - 4 * st;     // 32-blocks of this stage inside K: 2 or >= 4
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t wv = 0x7F7F7F7Fu;
-                        if (row_ok[c]) {
-                            const uint16_t *s16 = reinterpret_cast<const uint16_t *>(srow[c] + 4 * st);
-                            const uint32_t lo = s16[0];
-                            const uint32_t hi = nblk > 2 ? (uint32_t)s16[1] : 0x7F7Fu;
-                            wv = lo | (hi << 16);
-                        }
-                        v[c] = wv;
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t wv = 0x7F7F7F7Fu;
+                    if (row_ok[c]) {
+                        const uint16_t *s16 = reinterpret_cast<const uint16_t *>(srow[c] + 4 * st);
+                        const uint32_t lo = s16[0];
+                        const uint32_t hi = nblk > 2 ? (uint32_t)s16[1] : 0x7F7Fu;
+                        wv = lo | (hi << 16);
                     }
-                    tmem_st4(sf, v);
+                    v[c] = wv;
                 }
-                // B: hi (and lo) rows of the token block
-                {
-                    const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max;
-                    if (p.stacked) {
-                        for (int c = 0; c < n_sfb; ++c) {
-                            const int r = 32 * c + lane;            // stacked row: hi rows [0, NB), lo rows [NB, 2NB)
+            };
+            if constexpr (SFI) {
+                // the whole item, four stages at a time: 8 columns (A group, B group) per stage
+                if (!__all_sync(0xffffffffu, mbar_wait(&f_empty[sb], sph ^ 1, wc))) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t region = lane_base + sf_col0 + (uint32_t)(sb * sfi_cols);
+                // B words of four stages are loaded while the previous four stages'
+                // columns are stored (two register sets in turn); A words come from
+                // shared memory just before each 8-column store; one wait at the end
+                auto load_b4 = [&](int st0, uint32_t (&b)[4][4]) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int st = min(st0 + i, n_st - 1);
+                        // stacked block: B column c is row 32c + lane of [hi rows | lo rows]
+                        const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int r = 32 * c + lane;
                             const int plane = r >= NB ? 1 : 0;
                             const int j = r - plane * NB;
-                            uint32_t wv = 0x7F7F7F7Fu;
-                            if (r < 2 * NB && j < t.n_valid) wv = bsf[(size_t)plane * p.P_max + t.p0 + j];
-                            tmem_st1(sf + 8 + (uint32_t)c, wv);
-                        }
-                    } else {
-                        for (int c = 0; c < n_sfb; ++c) {
-                            const int j = 32 * c + lane;
-                            uint32_t w0 = 0x7F7F7F7Fu, w1 = 0x7F7F7F7Fu;
-                            if (j < t.n_valid) {
-                                w0 = bsf[t.p0 + j];
-                                w1 = bsf[(size_t)p.P_max + t.p0 + j];
-                            }
-                            tmem_st1(sf + 8 + (uint32_t)c, w0);
-                            tmem_st1(sf + 16 + (uint32_t)c, w1);
+                            b[i][c] = c < n_sfb && r < 2 * NB && j < t.n_valid
+                                          ? __ldg(bsf + (size_t)plane * p.P_max + j) : 0x7F7F7F7Fu;
                         }
                     }
-                }
-                if (st >= n_main) {
-                    // the K tail of tile rows 32q..32q+31: up to 2 x 16 code bytes ->
-                    // the first four 16-byte units of the row (8 code bytes each, the
-                    // rest zero), 128-byte swizzle
-                    const int r = 32 * q + lane;
-                    const int wrow = tile_weight_row<MODE>(r, t.mb, p.F);
-                    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-                    if (wrow < p.R) {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(
-                            p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
-                        c0 = src[0];
-                        c1 = src[1];
+                };
+                auto store4 = [&](int st0, const uint32_t (&b)[4][4]) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (st0 + i < n_st) {
+                            uint32_t v[8];
+                            a_words(st0 + i, v);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) v[4 + c] = b[i][c];
+                            tmem_st8(region + (uint32_t)(GEMM_SFI_COLS * (st0 + i)), v);
+                        }
                     }
-                    uint8_t *row = a_ring + slot * GEMM_A_STAGE + r * 128;
-                    const int sw = r & 7;
-                    *reinterpret_cast<uint4 *>(row + ((0 ^ sw) << 4)) = make_uint4(c0.x, c0.y, 0, 0);
-                    *reinterpret_cast<uint4 *>(row + ((1 ^ sw) << 4)) = make_uint4(c0.z, c0.w, 0, 0);
-                    *reinterpret_cast<uint4 *>(row + ((2 ^ sw) << 4)) = make_uint4(c1.x, c1.y, 0, 0);
-                    *reinterpret_cast<uint4 *>(row + ((3 ^ sw) << 4)) = make_uint4(c1.z, c1.w, 0, 0);
-                    fence_proxy_async_smem();
+                };
+                uint32_t b0[4][4], b1[4][4];
+                load_b4(0, b0);
+                for (int st0 = 0; st0 < n_st; st0 += 8) {
+                    if (st0 + 4 < n_st) load_b4(st0 + 4, b1);
+                    store4(st0, b0);
+                    if (st0 + 8 < n_st) load_b4(st0 + 8, b0);
+                    if (st0 + 4 < n_st) store4(st0 + 4, b1);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                mbar_arrive_w(&full[slot]);
-                if (++slot == NS) { slot = 0; ph ^= 1; }
+                mbar_arrive_w(&f_full[sb]);
+            } else {
+                uint32_t bw[SF_PD][SF_WORDS];
+#pragma unroll
+                for (int i = 0; i < SF_PD; ++i)
+                    if (i < n_st) load_bsf(i, bw[i]);
+                for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
+#pragma unroll
+                    for (int i = 0; i < SF_PD; ++i) {
+                        const int st = st0 + i;
+                        if (st >= n_st) break;
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                        const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                        {
+                            uint32_t v[4];
+                            a_words(st, v);
+                            tmem_st4(sf, v);
+                        }
+                        // B: the hi (and lo) columns of the token block
+                        if (p.stacked) {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                if (c < n_sfb) tmem_st1(sf + 8 + (uint32_t)c, bw[i][c]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < SF_WORDS / 2; ++c)
+                                if (c < n_sfb) {
+                                    tmem_st1(sf + 8 + (uint32_t)c, bw[i][2 * c]);
+                                    tmem_st1(sf + 16 + (uint32_t)c, bw[i][2 * c + 1]);
+                                }
+                        }
+                        tmem_wait_st();
+                        if (st + SF_PD < n_st) load_bsf(st + SF_PD, bw[i]);
+                        tc_fence_before();
+                        __syncwarp();
+                        mbar_arrive_w(&full[slot]);
+                        if (++slot == NS) { slot = 0; ph ^= 1; }
+                    }
+                }
             }
             if (!ok) break;
             __syncwarp();
@@ -399,18 +553,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 __syncwarp();
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
+            if (n_mma_warps == 2 && !__all_sync(0xffffffffu, mbar_wait(&d_full[2 + db], dph, wc))) break;
             tc_fence_after();
-            const uint32_t d_tmem = lane_base + (uint32_t)(db * d_cols);
             for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
                 float acc[16];
-                {
-                    uint32_t v[16];
-                    tmem_ld16(d_tmem + (uint32_t)c0, v);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
-                    if (p.stacked) {
-                        tmem_ld16(d_tmem + (uint32_t)(NB + c0), v);
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                // the sum over the MMA warps' accumulators and, stacked, their hi and lo halves
+                for (int mw = 0; mw < n_mma_warps; ++mw) {
+                    const uint32_t d_tmem = lane_base + (uint32_t)((mw * 2 + db) * d_cols);
+                    for (int half = 0; half < (p.stacked ? 2 : 1); ++half) {
+                        uint32_t v[16];
+                        tmem_ld16(d_tmem + (uint32_t)(half * NB + c0), v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
@@ -510,20 +664,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     }
 }
 
-template __global__ void expert_gemm_kernel<MODE_UP>(const __grid_constant__ GemmParams p);
-template __global__ void expert_gemm_kernel<MODE_DOWN>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_UP, false>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_UP, true>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_DOWN, false>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_DOWN, true>(const __grid_constant__ GemmParams p);
+
+template <int MODE, bool SFI>
+static cudaError_t launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, SFI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    expert_gemm_kernel<MODE, SFI><<<grid, GEMM_THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s) {
-    if (mode == MODE_UP) {
-        cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        expert_gemm_kernel<MODE_UP><<<grid, GEMM_THREADS, smem, s>>>(p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        expert_gemm_kernel<MODE_DOWN><<<grid, GEMM_THREADS, smem, s>>>(p);
-    }
-    return cudaGetLastError();
+    if (mode == MODE_UP)
+        return p.sf_item ? launch_gemm_t<MODE_UP, true>(p, grid, smem, s) : launch_gemm_t<MODE_UP, false>(p, grid, smem, s);
+    return p.sf_item ? launch_gemm_t<MODE_DOWN, true>(p, grid, smem, s) : launch_gemm_t<MODE_DOWN, false>(p, grid, smem, s);
 }
 
 }  // namespace moe

@@ -62,16 +62,18 @@ inline bool encode_a_down(CUtensorMap *m, const void *codes, int E, int d, int K
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Two-term E4M3 B operand u8 [rows][Kpad] (hi plane rows then lo plane rows):
-// box {128 bytes, box_rows}, 128-byte swizzle, zero fill past the last row.
+// Two-term E4M3 B operand u8 [2 planes][rows][Kpad] (the hi plane, then the lo
+// plane, each `rows` rows): a 3-D view {Kpad, rows, 2} whose box {128 bytes,
+// box_rows, 2} brings a token block's hi rows and their lo rows in one copy
+// (hi rows first in shared memory); 128-byte swizzle, zero fill past the last row.
 inline bool encode_bq(CUtensorMap *m, const void *base, int rows, int Kpad, int box_rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)Kpad, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)Kpad};
-    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+    const cuuint64_t dims[3] = {(cuuint64_t)Kpad, (cuuint64_t)rows, 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)Kpad, (cuuint64_t)rows * Kpad};
+    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -112,14 +114,18 @@ inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, in
     p.E = E;
     p.P_max = P_max;
     p.Kf = round_up_128(F);
-    // as many stages as shared memory and TMEM hold
+    // per-item scale factors (and two MMA warps) when a stacked block's item
+    // regions fit in TMEM next to four accumulators
+    const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;
+    p.sf_item = p.stacked && gemm_tmem_cols_item(p.nb_rows, p.stacked, n_st) <= 512 ? 1 : 0;
+    auto fits = [&](int ns) {
+        return gemm_smem_plan(p.K, E, p.nb_rows, ns).total <= GEMM_SMEM_LIMIT &&
+               (p.sf_item || gemm_tmem_cols(p.nb_rows, p.stacked, ns) <= 512);
+    };
+    // as many stages as shared memory (and, per stage, TMEM) hold
     int ns = GEMM_STAGES_MAX;
-    while (ns > 2 && (gemm_smem_plan(p.K, E, p.nb_rows, ns).total > GEMM_SMEM_LIMIT ||
-                      gemm_tmem_cols(p.nb_rows, p.stacked, ns) > 512))
-        --ns;
-    if (gemm_smem_plan(p.K, E, p.nb_rows, ns).total > GEMM_SMEM_LIMIT ||
-        gemm_tmem_cols(p.nb_rows, p.stacked, ns) > 512)
-        return MOE_ERR_ARG;
+    while (ns > 2 && !fits(ns)) --ns;
+    if (!fits(ns)) return MOE_ERR_ARG;
     p.n_stages = ns;
     *smem = gemm_smem_plan(p.K, E, p.nb_rows, ns).total;
     const long long P = (long long)T * top_k;

@@ -55,7 +55,7 @@ struct GemmParams {
     CUtensorMap map_a;          // E2M1 codes, 16 x 4-bit per 16 bytes in shared memory (unpacked TMA type);
                                 //   UP: 5-D {K_main, 16 rows, 2 halves, F/16 groups, E}, box {128, 16, 2, 4, 1}
                                 //   DOWN: 3-D {K_main, d, E}, box {128, 128, 1}
-    CUtensorMap map_b;          // u8 [2 * P_max][Kpad] E4M3 hi plane then lo plane; box {128, nb_rows}
+    CUtensorMap map_b;          // u8 [2][P_max][Kpad] E4M3 hi plane then lo plane; box {128, nb_rows, 2}
     const uint8_t *codes;       // u8 [E][R][K/2] (the K tail is read directly)
     const uint8_t *scales;      // u8 [E][R][K/32]
     const uint16_t *bias;       // bf16 [E][R]
@@ -68,7 +68,10 @@ struct GemmParams {
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= GEMM_NB_MAX)
     int stacked;                // 1: one MMA covers the hi and lo rows (N = 2 nb_rows); 0: one MMA per term
-    int n_stages;               // shared-memory / TMEM scale-factor ring depth
+    int n_stages;               // shared-memory ring depth (and TMEM scale-factor ring depth when !sf_item)
+    int sf_item;                // 1: a work item's scale factors are written to TMEM once, before its first
+                                //    stage, and two MMA warps take alternate stages (decode-sized blocks);
+                                // 0: scale factors per stage in a TMEM ring, one MMA warp
     int P_max;                  // rows of each B plane
     const int *counts, *offsets, *tiles;
     const int *row_token;       // [P]
@@ -100,8 +103,9 @@ struct GemmSmem {
 __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline int gemm_num_barriers(int n_stages) {
-    // stage full/empty, A-scale full/empty, D full/empty, drain, epilogue exchange [2][2]
-    return 2 * n_stages + 4 + 4 + 1 + 4;
+    // stage full/empty [NS], A-scale full/empty [2], D full [2 MMA warps][2], D empty [2],
+    // drain [2], epilogue exchange [2][2], item scale factors full/empty [2]
+    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4;
 }
 
 __host__ __device__ inline int gemm_b_stage_bytes(int nb_rows) { return 2 * nb_rows * 128; }
@@ -122,11 +126,16 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
     return s;
 }
 
-// TMEM columns of the plan: accumulators (2 buffers) first, then the ring of
-// scale-factor slots.
+// TMEM columns of the plan.  Per-stage mode: accumulators (2 buffers), then the
+// ring of scale-factor slots.  Per-item mode: accumulators [2 MMA warps][2
+// buffers], then two item regions of 8 columns per stage (A at +0, B at +4).
+constexpr int GEMM_SFI_COLS = 8;
 __host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 2 * nb_rows : nb_rows; }
 __host__ __device__ inline int gemm_tmem_cols(int nb_rows, int stacked, int n_stages) {
     return 2 * gemm_d_cols(nb_rows, stacked) + GEMM_SF_COLS * n_stages;
+}
+__host__ __device__ inline int gemm_tmem_cols_item(int nb_rows, int stacked, int n_st) {
+    return 4 * gemm_d_cols(nb_rows, stacked) + 2 * GEMM_SFI_COLS * n_st;
 }
 
 }  // namespace moe

@@ -166,7 +166,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nb = token_block_rows(T);
     CUtensorMap map_xq, map_hq;
-    if (!encode_bq(&map_xq, xq, 2 * (int)P, Kd, nb) || !encode_bq(&map_hq, hq, 2 * (int)P, Kf, nb))
+    if (!encode_bq(&map_xq, xq, (int)P, Kd, nb) || !encode_bq(&map_hq, hq, (int)P, Kf, nb))
         return MOE_ERR_CUDA;
     // the error word is the one buffer that must start at zero on every call
     if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
