@@ -195,7 +195,7 @@ MOE_API int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R,
  * Scratch memory comes from one fixed 8 MiB __device__ array inside the
  * library, held on every GPU that loads it until process exit; no context is
  * needed.  Limits: T <= MOE_NOALLOC_MAX_TOKENS and the workspace for the shape
- * (about T*(2d) + T*k*(6d + 2F) bytes, e.g. 6.3 MiB for 64 tokens of the
+ * (about T*(2d + 4E) + T*k*(6d + 2F) bytes, e.g. 6.5 MiB for 64 tokens of the
  * d_model = d_ff = 2880, top-4 layers) must fit in the array; larger requests
  * return MOE_ERR_ARG.  Shape limits otherwise as in moe_init.
  *

@@ -16,8 +16,6 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
-                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
@@ -48,6 +46,8 @@ struct moe_ctx {
     float *rho;
     int *topk_idx;
     float *topk_w;
+    float *logits;          // fp32 [T_max, E] router logits (decode-sized route path)
+    unsigned int *tok_done; // [T_max] per-token CTA counter of that path (zero between calls)
     int *counts, *offsets, *tiles;
     int *row_token;
     float *row_w;
@@ -212,11 +212,12 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
                             P * 4, P * 4, P * 4,
                             2 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
                             2 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
-                            P * s.d_model * 4, 64};
+                            P * s.d_model * 4, 64, T * E * 4, T * 4};
     void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
                       (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xq, (void **)&c->xsf,
-                      (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err};
+                      (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err,
+                      (void **)&c->logits, (void **)&c->tok_done};
     size_t total = 0;
     for (size_t v : sizes) total += round256(v);
     if (cudaMalloc(&c->ws, total) != cudaSuccess) {
@@ -267,6 +268,8 @@ int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale
     p.rho = c->rho;
     p.topk_idx = c->topk_idx;
     p.topk_w = c->topk_w;
+    p.logits = c->logits;
+    p.tok_done = c->tok_done;
     return cuda_status(launch_route(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -288,11 +291,14 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     p.row_w = c->row_w;
     p.pair_row = c->pair_row;
     p.err = c->err;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int rc2 = cuda_status(launch_group(p, st));
-    if (rc2) return rc2;
-    return cuda_status(launch_quant_permute(c->xn16, c->rho, c->row_token, c->xq, c->xsf, p.P,
-                                            c->shape.T_max * c->shape.top_k, c->shape.d_model, c->Kd, st));
+    p.xn16 = c->xn16;
+    p.rho = c->rho;
+    p.xq = c->xq;
+    p.xsf = c->xsf;
+    p.P_max = c->shape.T_max * c->shape.top_k;
+    p.d = c->shape.d_model;
+    p.Kd = c->Kd;
+    return cuda_status(launch_group(p, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,

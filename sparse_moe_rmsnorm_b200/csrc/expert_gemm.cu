@@ -175,14 +175,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         *abort_s = 0;
         fence_barrier_init();
     }
+    if (warp == 2) {
+        tmem_alloc(tmem_base_s, 512);
+        tmem_relinquish();
+    }
+    // the routing arrays and the B operand come from the kernels before this one
+    pdl_wait();
+    pdl_trigger();
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
         counts_s[i] = i < p.E ? p.counts[i] : 0;
         offsets_s[i] = p.offsets[i];
         tiles_s[i] = p.tiles[i];
-    }
-    if (warp == 2) {
-        tmem_alloc(tmem_base_s, 512);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -673,8 +676,7 @@ template <int MODE, bool SFI>
 static cudaError_t launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, SFI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    expert_gemm_kernel<MODE, SFI><<<grid, GEMM_THREADS, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(expert_gemm_kernel<MODE, SFI>, dim3(grid), dim3(GEMM_THREADS), (size_t)smem, s, p);
 }
 
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s) {

@@ -5,8 +5,28 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
 
 namespace moe {
+
+// Launch `kernel` on `s` with programmatic stream serialization: it may begin
+// (and run its prologue) while the previous kernel of the stream finishes;
+// the kernels call pdl_wait() before reading anything a predecessor wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Error bits of the device error word.
 enum : unsigned int {
@@ -27,6 +47,8 @@ struct RouteParams {
     float *rho;                 // fp32 [T]
     int *topk_idx;              // [T, k]
     float *topk_w;              // [T, k]
+    float *logits;              // fp32 [T, E] (decode-sized path: the CTAs' share of each token's logits)
+    unsigned int *tok_done;     // [T] CTAs finished per token (decode-sized path); zero between calls
 };
 
 struct GroupParams {
@@ -40,6 +62,12 @@ struct GroupParams {
     float *row_w;               // [P]
     int *pair_row;              // [P] expert-sorted row of pair (token, slot)
     unsigned int *err;
+    // the expert-sorted two-term E4M3 copy of the normalised tokens (gate/up B operand)
+    const __half *xn16;         // fp16 [T, d]
+    const float *rho;           // [T]
+    uint8_t *xq;                // [2][P_max][Kd]
+    uint32_t *xsf;              // [Kd/128][2][P_max]
+    int P_max, d, Kd;
 };
 
 // Grouped block-scaled GEMM over (expert, 128-row weight block, token block)

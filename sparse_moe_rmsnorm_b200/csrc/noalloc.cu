@@ -29,8 +29,6 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
-cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
-                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
@@ -41,7 +39,7 @@ using namespace moe;
 namespace {
 
 // 8 MiB of scratch: enough for decode-sized batches of the gpt-oss layers
-// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 4.8 MiB).
+// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 6.5 MiB).
 constexpr size_t kScratchBytes = 8u << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -132,7 +130,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     const size_t sizes[] = {(size_t)T * d * 2, (size_t)T * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
                             (size_t)(E + 1) * 4, P * 4, P * 4, P * 4,
                             2 * P * Kd, (size_t)(Kd / 128) * 2 * P * 4, 2 * P * Kf, (size_t)(Kf / 128) * 2 * P * 4,
-                            P * d * 4, 64};
+                            P * d * 4, 64, (size_t)T * E * 4, (size_t)T * 4};
     size_t total = 0;
     for (size_t v : sizes) total += r256(v);
     if (total > kScratchBytes) return MOE_ERR_ARG;
@@ -162,14 +160,18 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     uint32_t *hsf = reinterpret_cast<uint32_t *>(ptrs[13]);
     float *orows = reinterpret_cast<float *>(ptrs[14]);
     unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[15]);
+    float *logits = reinterpret_cast<float *>(ptrs[16]);
+    unsigned int *tok_done = reinterpret_cast<unsigned int *>(ptrs[17]);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nb = token_block_rows(T);
     CUtensorMap map_xq, map_hq;
     if (!encode_bq(&map_xq, xq, (int)P, Kd, nb) || !encode_bq(&map_hq, hq, (int)P, Kf, nb))
         return MOE_ERR_CUDA;
-    // the error word is the one buffer that must start at zero on every call
+    // the error word and the route kernel's per-token counters must start at zero
+    // on every call (the array keeps whatever the previous call, of any shape, left)
     if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(tok_done, 0, (size_t)T * sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
 
     RouteParams rp;
     rp.x = x;
@@ -185,6 +187,8 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     rp.rho = rho;
     rp.topk_idx = topk_idx;
     rp.topk_w = topk_w;
+    rp.logits = logits;
+    rp.tok_done = tok_done;
     if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     GroupParams gp;
@@ -201,9 +205,14 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.row_w = row_w;
     gp.pair_row = pair_row;
     gp.err = err;
+    gp.xn16 = xn16;
+    gp.rho = rho;
+    gp.xq = xq;
+    gp.xsf = xsf;
+    gp.P_max = (int)P;
+    gp.d = d;
+    gp.Kd = Kd;
     if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_quant_permute(xn16, rho, row_token, xq, xsf, (int)P, (int)P, d, Kd, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
 
     rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xq, xsf, counts,
                            offsets, tiles, row_token, row_w, hq, hsf, orows, err, s);

@@ -1,10 +1,12 @@
 // Routing side of the MoE block on sm_100a:
 //   route_kernel     RMSNorm + router logits + top-k + softmax over the chosen,
 //                    plus the fp16 normalised tokens for the experts;
-//   group_kernel     expert histogram, exclusive scan and a stable permutation
-//                    of the (token, expert) pairs into expert-contiguous rows;
-//   quant_permute_kernel  the expert-sorted two-term E4M3 copy of the normalised
-//                    tokens (the gate/up GEMM's B operand);
+//   route_small_kernel  the same for decode-sized batches, a CTA per (token,
+//                    16 experts);
+//   group_permute_kernel  expert histogram, exclusive scan and a stable
+//                    permutation of the (token, expert) pairs into
+//                    expert-contiguous rows, and the expert-sorted two-term E4M3
+//                    copy of the normalised tokens (the gate/up GEMM's B operand);
 //   combine_kernel   y = x + the token's weighted expert rows, in bf16.
 #include <cfloat>
 #include <climits>
@@ -73,6 +75,70 @@ __device__ __forceinline__ void load_bf16_vec(const uint16_t *p, float (&f)[VEC]
     }
 }
 
+// Top-k of one token's E logits (E <= 256) by one warp, then the softmax over
+// the chosen (pnsm.cn overview, section 2.2): k rounds of a warp arg-max on
+// (logit desc, index asc) -- ties go to the lower expert index; a NaN logit
+// ranks below every number, so the k chosen indices are always distinct and
+// in range.  `lg` may be shared or global memory.
+__device__ __forceinline__ void topk_softmax_warp(const float *lg, int E, int k, int t, int *topk_idx, float *topk_w,
+                                                  int lane) {
+    float v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int e = lane + 32 * c;
+        const float l = e < E ? lg[e] : -INFINITY;
+        v[c] = (l != l) ? -INFINITY : l;
+    }
+    unsigned taken = 0;
+    float sel_l[8];
+    int sel_e[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        if (r >= k) break;
+        float bv = -INFINITY;
+        int be = INT_MAX;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane + 32 * c;
+            if (e < E && !((taken >> c) & 1u) && (v[c] > bv || (v[c] == bv && e < be))) {
+                bv = v[c];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (ov > bv || (ov == bv && oe < be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        sel_l[r] = bv;
+        sel_e[r] = be;
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    }
+    if (lane == 0) {
+        const float m = sel_l[0];
+        float wsum = 0.f;
+        float wv[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (r < k) {
+                wv[r] = expf(sel_l[r] - m);
+                wsum += wv[r];
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (r < k) {
+                topk_idx[(size_t)t * k + r] = sel_e[r];
+                topk_w[(size_t)t * k + r] = wv[r] / wsum;
+            }
+        }
+    }
+}
+
 template <int TB, int NW, int EPW, int VEC>
 __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
     extern __shared__ float rsm[];
@@ -84,6 +150,8 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
     const int t0 = blockIdx.x * TB;
     const int ntok = min(TB, p.T - t0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
 
     // ---- RMSNorm
     const int ti = warp / WPT;              // token of this warp
@@ -203,79 +271,254 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
     __syncthreads();
 
     // ---- top-k and softmax, one warp per token
-    for (int i = warp; i < ntok; i += NW) {
-        const int tt = t0 + i;
-        float v[8];
+    for (int i = warp; i < ntok; i += NW) topk_softmax_warp(lg + i * E, E, p.k, t0 + i, p.topk_idx, p.topk_w, lane);
+}
+
+// ------------------------------------------------------ route, decode-sized
+//
+// Grid (token t, group of 16 experts); 16 warps, warp w owns expert 16y + w.
+// Each warp loads its expert's router row into registers before anything
+// else (the loads overlap the RMSNorm), every CTA normalises its token
+// (RMSNorm as above, the same fp32 arithmetic), each warp writes one fp32
+// logit, and the last CTA of the token to finish (a per-token counter, reset
+// by that CTA) takes the top-k and the softmax.  CTA y = 0 writes xn16 / rho.
+constexpr int ROUTE_SMALL_CHUNKS = 12;   // 8-element chunks of a router row per lane: d <= 3072
+
+__global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
+    __shared__ float xs[ROUTE_SMALL_CHUNKS * 256];
+    __shared__ float red[16];
+    __shared__ int is_last;
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d = p.d, E = p.E;
+    const int e = blockIdx.y * 16 + warp;
+    const int nch = d / 8;                   // 8-element chunks of a row
+    uint4 wv[ROUTE_SMALL_CHUNKS];
+#pragma unroll
+    for (int i = 0; i < ROUTE_SMALL_CHUNKS; ++i) {
+        const int c = lane + 32 * i;
+        wv[i] = (e < E && c < nch) ? __ldg(reinterpret_cast<const uint4 *>(p.router_w + (size_t)e * d) + c)
+                                   : make_uint4(0, 0, 0, 0);
+    }
+    // x may be the previous kernel's output: wait for it (the router rows above
+    // are weights, never written by a kernel)
+    pdl_wait();
+    pdl_trigger();
+    // RMSNorm: thread u owns chunks u and u + 512
+    float f[2][8], sc[2][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c = threadIdx.x + 512 * h;
+        if (c < nch) {
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * d) + c), f[h]);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.norm_scale) + c), sc[h]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss += f[h][k] * f[h][k];
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tot += red[i];
+    const float inv_rms = 1.0f / sqrtf(tot / (float)d + p.eps);
+    float amax = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c = threadIdx.x + 512 * h;
+        if (c < nch) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float v = f[h][k] * inv_rms * sc[h][k];
+                f[h][k] = v;
+                xs[8 * c + k] = v;
+                amax = fmaxf(amax, fabsf(v));
+            }
+        }
+    }
+    if (blockIdx.y == 0) {
+        amax = warp_max(amax);
+        __syncthreads();                     // every thread has read red[] above
+        if (lane == 0) red[warp] = amax;
+        __syncthreads();
+        amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, red[i]);
+        float rho = 1.f, inv_rho = 1.f;
+        if (amax > 0.f && amax <= FLT_MAX) {
+            int ex;
+            frexpf(amax, &ex);               // amax in [2^(ex-1), 2^ex)
+            rho = exp2i(ex - 14);
+            inv_rho = exp2i(14 - ex);
+        }
+        if (threadIdx.x == 0) p.rho[t] = rho;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = threadIdx.x + 512 * h;
+            if (c < nch) {
+                uint32_t hw[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const __half2 h2 = __floats2half2_rn(f[h][2 * k] * inv_rho, f[h][2 * k + 1] * inv_rho);
+                    hw[k] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                reinterpret_cast<uint4 *>(p.xn16 + (size_t)t * d)[c] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            }
+        }
+    }
+    __syncthreads();
+    // logit of expert e
+    if (e < E) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < ROUTE_SMALL_CHUNKS; ++i) {
+            const int c = lane + 32 * i;
+            if (c < nch) {
+                float w8[8];
+                bf16x8_to_f32(wv[i], w8);
+                const float4 a = *reinterpret_cast<const float4 *>(xs + 8 * c);
+                const float4 b = *reinterpret_cast<const float4 *>(xs + 8 * c + 4);
+                acc = fmaf(a.x, w8[0], acc);
+                acc = fmaf(a.y, w8[1], acc);
+                acc = fmaf(a.z, w8[2], acc);
+                acc = fmaf(a.w, w8[3], acc);
+                acc = fmaf(b.x, w8[4], acc);
+                acc = fmaf(b.y, w8[5], acc);
+                acc = fmaf(b.z, w8[6], acc);
+                acc = fmaf(b.w, w8[7], acc);
+            }
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) {
+            p.logits[(size_t)t * E + e] = acc + p.router_b[e];
+            __threadfence();
+        }
+    }
+    // the token's last CTA takes the top-k
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&p.tok_done[t], 1u);
+        is_last = prev == gridDim.y - 1;
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (warp == 0) {
+        float lg[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const int e = lane + 32 * c;
-            const float l = e < E ? lg[i * E + e] : -INFINITY;
-            v[c] = (l != l) ? -INFINITY : l;
+            const int ee = lane + 32 * c;
+            lg[c] = ee < E ? __ldcg(p.logits + (size_t)t * E + ee) : 0.f;
         }
-        unsigned taken = 0;
-        float sel_l[8];
-        int sel_e[8];
+        // stage the logits in shared memory for the warp arg-max
+        float *lgs = xs;
+        __syncwarp();
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            if (r >= p.k) break;
-            float bv = -INFINITY;
-            int be = INT_MAX;
+        for (int c = 0; c < 8; ++c)
+            if (lane + 32 * c < E) lgs[lane + 32 * c] = lg[c];
+        __syncwarp();
+        topk_softmax_warp(lgs, E, p.k, t, p.topk_idx, p.topk_w, lane);
+        if (lane == 0) p.tok_done[t] = 0;
+    }
+}
+
+// ------------------------------------------------------- group + permute
+//
+// Grid of G CTAs of 32 warps.  Every CTA computes the whole grouping of the
+// P = T*k pairs (pair i = token i/k, slot i%k) in shared memory: warp w owns
+// a contiguous segment of the pairs; pass 1 counts, per warp and expert, with
+// __match_any_sync; a column scan turns the per-warp counts into each warp's
+// starting position inside every expert's range; pass 2 assigns positions in
+// pair order.  The result is sorted by expert and, within an expert, by token.
+// CTA c then owns the expert-sorted rows [c*R, (c+1)*R): it writes their
+// row_token / row_w / pair_row entries and their B operand row (below).  CTA 0
+// writes counts, offsets and tiles.
+//
+// B operand row r: the normalised activations of token row_token[r],
+// v = xn16 * rho, as two E4M3 terms per 32-element block with E8M0 scale s
+// (the exponent that fits the block maximum to 448):
+//   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)).
+// Out: xq[plane][r][0:Kd] (plane 0 hi, plane 1 lo; columns d..Kd zero) and
+// xsf[g][plane][r] = the scale bytes of the 32-blocks 4g..4g+3 (byte i is
+// block 4g+i).  One warp per row; lane l takes the 32-blocks l, l+32, ...
+constexpr int GROUP_ROWS_MAX = 1024;   // expert-sorted rows per CTA, at most
+
+__device__ __forceinline__ void quant_row(const GroupParams &p, int r, int tok, int lane) {
+    const float sc = p.rho[tok];
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.xn16 + (size_t)tok * p.d);
+    const int nblk = p.d / 32, nblk_pad = p.Kd / 32;
+    for (int b0 = 0; b0 < nblk_pad; b0 += 32) {
+        const int b = b0 + lane;
+        uint32_t s_hi = 127, s_lo = 127;
+        uint32_t qh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ql[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (b < nblk) {
+            float v[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int e = lane + 32 * c;
-                if (e < E && !((taken >> c) & 1u) && (v[c] > bv || (v[c] == bv && e < be))) {
-                    bv = v[c];
-                    be = e;
+            for (int i = 0; i < 4; ++i) {
+                const uint4 u = src[4 * b + i];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t wk = k == 0 ? u.x : (k == 1 ? u.y : (k == 2 ? u.z : u.w));
+                    v[8 * i + 2 * k] = __half2float(__ushort_as_half((unsigned short)(wk & 0xFFFFu))) * sc;
+                    v[8 * i + 2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(wk >> 16))) * sc;
                 }
             }
+            float amax = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (ov > bv || (ov == bv && oe < be)) {
-                    bv = ov;
-                    be = oe;
-                }
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            const int e_hi = e4m3_block_exp(amax);
+            const int e_lo = max(e_hi - 4, -126);
+            const float inv_hi = pow2f(-e_hi), inv_lo = pow2f(-e_lo), mul_hi = pow2f(e_hi);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t h = f32x2_to_e4m3x2(v[2 * i] * inv_hi, v[2 * i + 1] * inv_hi);
+                float d0, d1;
+                e4m3x2_to_f32x2(h, d0, d1);
+                const uint32_t l = f32x2_to_e4m3x2((v[2 * i] - d0 * mul_hi) * inv_lo,
+                                                   (v[2 * i + 1] - d1 * mul_hi) * inv_lo);
+                qh[i >> 1] |= h << (16 * (i & 1));
+                ql[i >> 1] |= l << (16 * (i & 1));
             }
-            sel_l[r] = bv;
-            sel_e[r] = be;
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            s_hi = (uint32_t)(e_hi + 127);
+            s_lo = (uint32_t)(e_lo + 127);
         }
-        if (lane == 0) {
-            const float m = sel_l[0];
-            float wsum = 0.f;
-            float wv[8];
+        if (b < nblk_pad) {
+            uint4 *dh = reinterpret_cast<uint4 *>(p.xq + (size_t)r * p.Kd + 32 * b);
+            uint4 *dl = reinterpret_cast<uint4 *>(p.xq + ((size_t)p.P_max + r) * p.Kd + 32 * b);
+            dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
+            dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
+            dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
+            dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
+        }
+        // the scale bytes of four consecutive blocks (lanes 4m..4m+3) as one word
+        uint32_t wh = s_hi, wl = s_lo;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                if (r < p.k) {
-                    wv[r] = expf(sel_l[r] - m);
-                    wsum += wv[r];
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                if (r < p.k) {
-                    p.topk_idx[(size_t)tt * p.k + r] = sel_e[r];
-                    p.topk_w[(size_t)tt * p.k + r] = wv[r] / wsum;
-                }
-            }
+        for (int i = 1; i < 4; ++i) {
+            wh |= __shfl_down_sync(0xffffffffu, s_hi, i) << (8 * i);
+            wl |= __shfl_down_sync(0xffffffffu, s_lo, i) << (8 * i);
+        }
+        if ((lane & 3) == 0 && b < nblk_pad) {
+            const size_t g = (size_t)(b >> 2);
+            p.xsf[(g * 2) * p.P_max + r] = wh;
+            p.xsf[(g * 2 + 1) * p.P_max + r] = wl;
         }
     }
 }
 
-// ----------------------------------------------------------------- group
-//
-// One CTA of 32 warps.  Warp w owns a contiguous segment of the T*k pairs
-// (pair i = token i/k, slot i%k).  Pass 1 counts, per warp and expert, with
-// __match_any_sync; a column scan turns the per-warp counts into each warp's
-// starting position inside every expert's range; pass 2 assigns positions in
-// pair order.  The result is sorted by expert and, within an expert, by token.
-__global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
+__global__ void __launch_bounds__(1024) group_permute_kernel(const GroupParams p) {
     __shared__ int wcnt[32][257];
     __shared__ int off_s[257];
+    __shared__ int tok_s[GROUP_ROWS_MAX];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E, P = p.P;
+    const int rows_per = (P + gridDim.x - 1) / gridDim.x;
+    const int r0 = blockIdx.x * rows_per, r1 = min(P, r0 + rows_per);
     for (int i = threadIdx.x; i < 32 * 257; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    pdl_wait();
+    pdl_trigger();
     __syncthreads();
     const int seg = (P + 31) / 32;
     const int beg = warp * seg, end = min(P, beg + seg);
@@ -293,7 +536,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
             const int i = base + 32 * r + lane;
             int e = ev[r];
             if (i < end && (e < 0 || e >= E)) {
-                atomicOr(p.err, ERR_ROUTING);
+                if (blockIdx.x == 0) atomicOr(p.err, ERR_ROUTING);
                 e = -1;
             }
             const unsigned m = __match_any_sync(0xffffffffu, e);
@@ -311,7 +554,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
             wcnt[w][e] = s;
             s += c;
         }
-        p.counts[e] = s;
+        if (blockIdx.x == 0) p.counts[e] = s;
         off_s[e] = s;   // total for now
     }
     __syncthreads();
@@ -344,20 +587,22 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
             const int e = lane * 8 + c;
             if (e < E) {
                 off_s[e] = co;
-                p.offsets[e] = co;
-                p.tiles[e] = bo;
+                if (blockIdx.x == 0) {
+                    p.offsets[e] = co;
+                    p.tiles[e] = bo;
+                }
             }
             co += cnt[c];
             bo += blk[c];
         }
-        if (lane == 31) {
+        if (lane == 31 && blockIdx.x == 0) {
             p.offsets[E] = ci;
             p.tiles[E] = bi;
         }
     }
     __syncthreads();
 
-    // pass 2: positions, in pair order within each warp's segment
+    // pass 2: positions, in pair order within each warp's segment; this CTA keeps its rows
     for (int base = beg; base < end; base += 256) {
         int ev[8];
         float wv[8];
@@ -375,95 +620,22 @@ __global__ void __launch_bounds__(1024) group_kernel(const GroupParams p) {
             const unsigned m = __match_any_sync(0xffffffffu, e);
             if (e >= 0) {
                 const int pos = off_s[e] + wcnt[warp][e] + __popc(m & ((1u << lane) - 1u));
-                p.row_token[pos] = i / p.k;
-                p.row_w[pos] = wv[r];
-                p.pair_row[i] = pos;
+                if (pos >= r0 && pos < r1) {
+                    p.row_token[pos] = i / p.k;
+                    p.row_w[pos] = wv[r];
+                    p.pair_row[i] = pos;
+                    tok_s[pos - r0] = i / p.k;
+                }
             }
             __syncwarp();
             if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp][e] += __popc(m);
             __syncwarp();
         }
     }
-}
+    __syncthreads();
 
-// --------------------------------------------------------------- permute + quantise
-//
-// Row r (< P) of the gate/up GEMM's B operand: the normalised activations of
-// token row_token[r], v = xn16 * rho, as two E4M3 terms per 32-element block
-// with E8M0 scale s (the exponent that fits the block maximum to 448):
-//   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)).
-// Out: xq[plane][r][0:Kd] (plane 0 hi, plane 1 lo; columns d..Kd zero) and
-// xsf[g][plane][r] = the scale bytes of the 32-blocks 4g..4g+3 (byte i is
-// block 4g+i).  One warp per row; lane l takes the 32-blocks l, l+32, ...
-__global__ void __launch_bounds__(256, 1) quant_permute_kernel(const __half *__restrict__ xn16,
-                                                            const float *__restrict__ rho,
-                                                            const int *__restrict__ row_token,
-                                                            uint8_t *__restrict__ xq, uint32_t *__restrict__ xsf,
-                                                            int P, int P_max, int d, int Kd) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    const int nblk = d / 32, nblk_pad = Kd / 32;
-    for (int r = warp; r < P; r += nwarps) {
-        const int tok = row_token[r];
-        const float sc = rho[tok];
-        const uint4 *src = reinterpret_cast<const uint4 *>(xn16 + (size_t)tok * d);
-        for (int b0 = 0; b0 < nblk_pad; b0 += 32) {
-            const int b = b0 + lane;
-            uint32_t s_hi = 127, s_lo = 127;
-            uint32_t qh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ql[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (b < nblk) {
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 u = src[4 * b + i];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t wk = k == 0 ? u.x : (k == 1 ? u.y : (k == 2 ? u.z : u.w));
-                        v[8 * i + 2 * k] = __half2float(__ushort_as_half((unsigned short)(wk & 0xFFFFu))) * sc;
-                        v[8 * i + 2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(wk >> 16))) * sc;
-                    }
-                }
-                float amax = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                const int e_hi = e4m3_block_exp(amax);
-                const int e_lo = max(e_hi - 4, -126);
-                const float inv_hi = pow2f(-e_hi), inv_lo = pow2f(-e_lo), mul_hi = pow2f(e_hi);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t h = f32x2_to_e4m3x2(v[2 * i] * inv_hi, v[2 * i + 1] * inv_hi);
-                    float d0, d1;
-                    e4m3x2_to_f32x2(h, d0, d1);
-                    const uint32_t l = f32x2_to_e4m3x2((v[2 * i] - d0 * mul_hi) * inv_lo,
-                                                       (v[2 * i + 1] - d1 * mul_hi) * inv_lo);
-                    qh[i >> 1] |= h << (16 * (i & 1));
-                    ql[i >> 1] |= l << (16 * (i & 1));
-                }
-                s_hi = (uint32_t)(e_hi + 127);
-                s_lo = (uint32_t)(e_lo + 127);
-            }
-            if (b < nblk_pad) {
-                uint4 *dh = reinterpret_cast<uint4 *>(xq + (size_t)r * Kd + 32 * b);
-                uint4 *dl = reinterpret_cast<uint4 *>(xq + ((size_t)P_max + r) * Kd + 32 * b);
-                dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
-                dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
-                dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
-                dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
-            }
-            // the scale bytes of four consecutive blocks (lanes 4m..4m+3) as one word
-            uint32_t wh = s_hi, wl = s_lo;
-#pragma unroll
-            for (int i = 1; i < 4; ++i) {
-                wh |= __shfl_down_sync(0xffffffffu, s_hi, i) << (8 * i);
-                wl |= __shfl_down_sync(0xffffffffu, s_lo, i) << (8 * i);
-            }
-            if ((lane & 3) == 0 && b < nblk_pad) {
-                const size_t g = (size_t)(b >> 2);
-                xsf[(g * 2) * P_max + r] = wh;
-                xsf[(g * 2 + 1) * P_max + r] = wl;
-            }
-        }
-    }
+    // this CTA's rows of the B operand, one warp per row
+    for (int r = r0 + warp; r < r1; r += 32) quant_row(p, r, tok_s[r - r0], lane);
 }
 
 // --------------------------------------------------------------- combine
@@ -477,6 +649,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                                                       int T, int d, int k) {
     const int per_tok = d / 8;
     const long long n = (long long)T * per_tok;
+    pdl_wait();
+    pdl_trigger();
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
         const int t = (int)(i / per_tok), j = (int)(i % per_tok) * 8;
@@ -555,12 +729,15 @@ static cudaError_t launch_route_cfg(const RouteParams &p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(route_kernel<TB, NW, EPW, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    route_kernel<TB, NW, EPW, VEC><<<(p.T + TB - 1) / TB, NW * 32, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(route_kernel<TB, NW, EPW, VEC>, dim3((p.T + TB - 1) / TB), dim3(NW * 32), smem, s, p);
 }
 
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
     if (p.T <= 0) return cudaSuccess;
+    // decode-sized batches: a CTA per (token, 16 experts), router rows held in registers
+    if (p.T <= 512 && p.d <= ROUTE_SMALL_CHUNKS * 256 && p.logits && p.tok_done) {
+        return launch_pdl(route_small_kernel, dim3(p.T, (p.E + 15) / 16), dim3(512), 0, s, p);
+    }
     // few tokens: one token per CTA, 32 warps (latency); many tokens: the
     // router weights are reused across 8 (or 4) tokens of a CTA (throughput)
     if (p.T <= 512 || (size_t)8 * (p.d + p.E) * 4 > 200 * 1024) return launch_route_cfg<1, 32, 8, 8>(p, s);
@@ -569,16 +746,13 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
-    group_kernel<<<1, 1024, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_quant_permute(const __half *xn16, const float *rho, const int *row_token, uint8_t *xq,
-                                 uint32_t *xsf, int P, int P_max, int d, int Kd, cudaStream_t s) {
-    if (P <= 0) return cudaSuccess;
-    const int grid = min((P + 7) / 8, 148 * 8);
-    quant_permute_kernel<<<grid, 256, 0, s>>>(xn16, rho, row_token, xq, xsf, P, P_max, d, Kd);
-    return cudaGetLastError();
+    if (p.P <= 0) return cudaSuccess;
+    // CTAs: one per 8 rows for small batches, one per SM for large ones, and at
+    // most GROUP_ROWS_MAX rows each
+    int grid = (p.P + 7) / 8;
+    if (grid > 148) grid = 148;
+    if ((p.P + grid - 1) / grid > GROUP_ROWS_MAX) grid = (p.P + GROUP_ROWS_MAX - 1) / GROUP_ROWS_MAX;
+    return launch_pdl(group_permute_kernel, dim3(grid), dim3(1024), 0, s, p);
 }
 
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
@@ -586,8 +760,7 @@ cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pai
     const long long n = (long long)T * (d / 8);
     if (n == 0) return cudaSuccess;
     const int grid = (int)min((n + 255) / 256, (long long)148 * 8);
-    combine_kernel<<<grid, 256, 0, s>>>(x, orows, pair_row, y, T, d, k);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, x, orows, pair_row, y, T, d, k);
 }
 
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s) {
