@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NS = p.n_stages;
     const int NB = p.nb_rows;
-    const GemmSmem plan = gemm_smem_plan(p.K, p.E, NB, NS);
+    const GemmSmem plan = gemm_smem_plan(p.K, p.E, NB, NS, SFI ? 1 : 0);
     uint8_t *a_ring = smem + plan.a_off;
     uint8_t *b_ring = smem + plan.b_off;
     const int b_stage = gemm_b_stage_bytes(NB);
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     const int KB32 = p.K / 32;
     const int scale_bytes = align_up(GEMM_BM * KB32, 128);
     float *amax_s = reinterpret_cast<float *>(smem + plan.amax_off);   // [2 groups][2 parities][4 warps][16 columns]
-    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off);  // [8 warps][GEMM_NB_MAX]
+    float *meta_val = reinterpret_cast<float *>(smem + plan.meta_off);  // [8 warps][NB]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bar_off);
     uint64_t *full = bars;
     uint64_t *empty = full + NS;
@@ -137,6 +137,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *ex_bar = drain_bar + 2;       // [2 groups][2 parities]
     uint64_t *f_full = ex_bar + 4;          // [2] a work item's scale factors in TMEM (per-item mode)
     uint64_t *f_empty = f_full + 2;
+    uint64_t *bw_full = f_empty + 2;        // the item's B scale words are staged (per-item mode)
+    uint64_t *bw_empty = bw_full + 1;       // ... and have been read by all four scale-factor warps
+    uint32_t *bw_s = reinterpret_cast<uint32_t *>(smem + plan.bsf_off);   // [stage][4][32]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
@@ -172,6 +175,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             mbar_init(&d_full[i], 1);
             mbar_init(&ex_bar[i], 4);     // the four warps of an epilogue group
         }
+        mbar_init(bw_full, 4);            // the four scale-factor warps
+        mbar_init(bw_empty, 4);
         *abort_s = 0;
         fence_barrier_init();
     }
@@ -197,11 +202,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 
     if (warp == 0) {
         // ------------------------------------------------- A producer (weights)
-        // Per work item the 128 rows' E8M0 bytes (one or two untiled bulk
-        // copies), issued one item ahead so the scale-factor warps can prepare
-        // an item while the MMAs work on the one before; per stage one TMA box
+        // Per work item (per-stage mode) the 128 rows' E8M0 bytes (one or two
+        // untiled bulk copies), issued one item ahead so the scale-factor warps
+        // can prepare an item while the MMAs work on the one before; per stage one TMA box
         // of E2M1 codes (128 rows x 128 K).  The K tail (K not a multiple of
-        // 128) is copied into its stage's slot here, four rows per lane.
+        // 128) is loaded at the start of the item, four rows per lane, and
+        // written into its stage's slot here.
         if (lane == 0 && n_main > 0) tma_prefetch_desc(&p.map_a);
         int slot = 0, sb = 0;
         uint32_t ph = 0, sph = 0;
@@ -229,13 +235,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         Work t;
         if (blockIdx.x < total) {
             work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
-            ok = load_scales(t);
+            if constexpr (!SFI) ok = load_scales(t);     // per-item mode: the scale-factor warps load them
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            uint4 tail[8];                   // the item's K tail codes (rows lane + 32j)
+            auto load_tail = [&]() {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int wrow = tile_weight_row<MODE>(lane + 32 * j, t.mb, p.F);
+                    tail[2 * j] = tail[2 * j + 1] = make_uint4(0, 0, 0, 0);
+                    if (wrow < p.R) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
+                        tail[2 * j] = __ldg(src);
+                        tail[2 * j + 1] = __ldg(src + 1);
+                    }
+                }
+            };
+            // the K tail codes, loaded at the start of the item so that the tail stage
+            // does not wait on global memory
+            if (n_st > n_main) load_tail();
             Work tn;
             if (w + (int)gridDim.x < total) {
                 work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, tn);
-                if (!load_scales(tn)) { ok = false; break; }
+                if constexpr (!SFI) {
+                    if (!load_scales(tn)) { ok = false; break; }
+                }
             }
             for (int st = 0; st < n_st; ++st) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
@@ -251,18 +276,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     // K tail of rows lane + 32j: 2 x 16 code bytes -> the first four
                     // 16-byte units of the row (8 code bytes each, the rest zero),
                     // 128-byte swizzle
-                    uint4 tail[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int wrow = tile_weight_row<MODE>(lane + 32 * j, t.mb, p.F);
-                        tail[2 * j] = tail[2 * j + 1] = make_uint4(0, 0, 0, 0);
-                        if (wrow < p.R) {
-                            const uint4 *src = reinterpret_cast<const uint4 *>(
-                                p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
-                            tail[2 * j] = __ldg(src);
-                            tail[2 * j + 1] = __ldg(src + 1);
-                        }
-                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int r = lane + 32 * j;
@@ -327,10 +340,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
-            const uint32_t n = p.stacked ? (uint32_t)(2 * NB) : (uint32_t)t.n_mma;
+            const bool stacked = SFI || p.stacked;     // per-item mode always stacks hi and lo rows
+            const uint32_t n = stacked ? (uint32_t)(2 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
-            // E8M0 scales, M >> 4; the scale byte of each MMA is set per K block below
+            // E8M0 scales, M >> 4; K block kb of a stage takes scale byte kb (fields at 4 and 29)
             const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
+            uint32_t idesc[4];
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) idesc[kb] = idesc0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
             if (!__all_sync(0xffffffffu, mbar_wait(&d_empty[db], dph ^ 1, wc))) { ok = false; break; }
             if (SFI && !__all_sync(0xffffffffu, mbar_wait(&f_full[sb], sph, wc))) { ok = false; break; }
             tc_fence_after();
@@ -343,20 +360,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             for (int st = m; st < n_st; st += n_mma_warps) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t a_addr = smem_addr(a_ring + slot * GEMM_A_STAGE);
-                const uint32_t b_addr = smem_addr(b_ring + slot * b_stage);
+                // descriptors of the slot's A and B; K block kb starts 32 bytes further
+                // (+2 in the descriptor's address field, which never carries here)
+                const uint64_t ad = smem_desc_sw128(smem_addr(a_ring + slot * GEMM_A_STAGE));
+                const uint64_t bd = smem_desc_sw128(smem_addr(b_ring + slot * b_stage));
+                const uint64_t bd_lo = bd + (uint64_t)(NB * 128 >> 4);
                 const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * st)
                                         : tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
                 const uint32_t sfb = SFI ? sf + 4 : sf + 8;
-                const int nkb = st < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const uint32_t idesc = idesc0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
-                    const uint64_t ad = smem_desc_sw128(a_addr + kb * 32);
-                    mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + kb * 32), idesc, sf, sfb, acc);
-                    if (!p.stacked)
-                        mma_mx_w(d_tmem, ad, smem_desc_sw128(b_addr + NB * 128 + kb * 32), idesc, sf, sf + 16, 1u);
-                    acc = 1;
+                if (st < n_main) {
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, (acc | kb) ? 1u : 0u);
+                        if (!stacked) mma_mx_w(d_tmem, ad + 2 * kb, bd_lo + 2 * kb, idesc[kb], sf, sf + 16, 1u);
+                    }
+                } else {
+                    const int nkb = (p.K - n_main * GEMM_KS) / 32;    // the K tail: 1..3 blocks
+#pragma unroll
+                    for (int kb = 0; kb < 3; ++kb) {
+                        if (kb >= nkb) break;
+                        mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, (acc | kb) ? 1u : 0u);
+                        if (!stacked) mma_mx_w(d_tmem, ad + 2 * kb, bd_lo + 2 * kb, idesc[kb], sf, sf + 16, 1u);
+                    }
                 }
+                acc = 1;
                 issued = true;
                 mma_commit_w(&empty[slot]);
                 advance(slot, ph, n_mma_warps);
@@ -386,6 +413,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         uint32_t ph = 0, sph = 0;
         bool ok = true;
         const int n_sfb = p.stacked ? (2 * NB + 31) / 32 : (NB + 31) / 32;
+        uint32_t bph = 0;                    // phase parity of the staging barriers (one phase per item)
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
@@ -415,8 +443,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     }
                 }
             };
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
-            const uint8_t *sbase = scale_buf + sb * scale_bytes;
+            if constexpr (!SFI) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
+            }
+            const uint8_t *sbase = scale_buf + (SFI ? 0 : sb * scale_bytes);
             const uint8_t *srow[4];
             bool row_ok[4];
 #pragma unroll
@@ -440,53 +470,77 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
             };
             if constexpr (SFI) {
-                // the whole item, four stages at a time: 8 columns (A group, B group) per stage
-                if (!__all_sync(0xffffffffu, mbar_wait(&f_empty[sb], sph ^ 1, wc))) { ok = false; break; }
+                // The whole item.  The four warps load its A scale bytes (one or two
+                // contiguous runs of 16-byte words, a quarter each) and its B scale
+                // words (warp q: stages q, q+4, ...), all loads in flight at once, and
+                // stage them in shared memory for each other; then each warp writes one
+                // 8-column group (A, B) per stage of its lane quarter and waits once.
+                const int sf_tid = 32 * q + lane;
+                const int run_bytes = MODE == MODE_UP ? 64 * KB32 : min(GEMM_BM, p.R - t.mb * GEMM_BM) * KB32;
+                const int n16 = run_bytes / 16;
+                const int n_words = MODE == MODE_UP ? 2 * n16 : n16;
+                const uint4 *run0 = reinterpret_cast<const uint4 *>(
+                    p.scales + ((size_t)t.e * p.R + (MODE == MODE_UP ? t.mb * 64 : t.mb * GEMM_BM)) * KB32);
+                const uint4 *run1 = reinterpret_cast<const uint4 *>(p.scales + ((size_t)t.e * p.R + p.F + t.mb * 64) * KB32);
+                constexpr int SW = (GEMM_SFI_STAGES_MAX * 4 * GEMM_BM / 16 + 127) / 128;   // words per thread, at most
+                uint4 sreg[SW];
+#pragma unroll
+                for (int i = 0; i < SW; ++i) {
+                    const int wi = sf_tid + 128 * i;
+                    sreg[i] = make_uint4(0, 0, 0, 0);
+                    if (wi < n16) sreg[i] = __ldg(run0 + wi);
+                    else if (MODE == MODE_UP && wi < n_words) sreg[i] = __ldg(run1 + (wi - n16));
+                }
+                uint32_t bwr[GEMM_SFI_STAGES_MAX / 4][4];
+#pragma unroll
+                for (int i = 0; i < GEMM_SFI_STAGES_MAX / 4; ++i) {
+                    const int st = q + 4 * i;
+                    // stacked block: B column c is row 32c + lane of [hi rows | lo rows]
+                    const uint32_t *bsf = p.b_sf + (size_t)min(st, n_st - 1) * 2 * p.P_max + t.p0;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = 32 * c + lane;
+                        const int plane = r >= NB ? 1 : 0;
+                        const int j = r - plane * NB;
+                        bwr[i][c] = st < n_st && c < n_sfb && r < 2 * NB && j < t.n_valid
+                                        ? __ldg(bsf + (size_t)plane * p.P_max + j) : 0x7F7F7F7Fu;
+                    }
+                }
+                // the staging buffer is free once all four warps have read the last item's words
+                if (!__all_sync(0xffffffffu, mbar_wait(bw_empty, bph ^ 1, wc))) { ok = false; break; }
+#pragma unroll
+                for (int i = 0; i < GEMM_SFI_STAGES_MAX / 4; ++i) {
+                    const int st = q + 4 * i;
+                    if (st < n_st) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) bw_s[(st * 4 + c) * 32 + lane] = bwr[i][c];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < SW; ++i) {
+                    const int wi = sf_tid + 128 * i;
+                    if (wi < n_words) reinterpret_cast<uint4 *>(scale_buf)[wi] = sreg[i];
+                }
+                __syncwarp();
+                mbar_arrive_w(bw_full);
+                if (!__all_sync(0xffffffffu, mbar_wait(f_empty + sb, sph ^ 1, wc))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(bw_full, bph, wc))) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t region = lane_base + sf_col0 + (uint32_t)(sb * sfi_cols);
-                // B words of four stages are loaded while the previous four stages'
-                // columns are stored (two register sets in turn); A words come from
-                // shared memory just before each 8-column store; one wait at the end
-                auto load_b4 = [&](int st0, uint32_t (&b)[4][4]) {
+                for (int st = 0; st < n_st; ++st) {
+                    uint32_t v[8];
+                    a_words(st, v);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int st = min(st0 + i, n_st - 1);
-                        // stacked block: B column c is row 32c + lane of [hi rows | lo rows]
-                        const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int r = 32 * c + lane;
-                            const int plane = r >= NB ? 1 : 0;
-                            const int j = r - plane * NB;
-                            b[i][c] = c < n_sfb && r < 2 * NB && j < t.n_valid
-                                          ? __ldg(bsf + (size_t)plane * p.P_max + j) : 0x7F7F7F7Fu;
-                        }
-                    }
-                };
-                auto store4 = [&](int st0, const uint32_t (&b)[4][4]) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (st0 + i < n_st) {
-                            uint32_t v[8];
-                            a_words(st0 + i, v);
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) v[4 + c] = b[i][c];
-                            tmem_st8(region + (uint32_t)(GEMM_SFI_COLS * (st0 + i)), v);
-                        }
-                    }
-                };
-                uint32_t b0[4][4], b1[4][4];
-                load_b4(0, b0);
-                for (int st0 = 0; st0 < n_st; st0 += 8) {
-                    if (st0 + 4 < n_st) load_b4(st0 + 4, b1);
-                    store4(st0, b0);
-                    if (st0 + 8 < n_st) load_b4(st0 + 8, b0);
-                    if (st0 + 4 < n_st) store4(st0 + 4, b1);
+                    for (int c = 0; c < 4; ++c) v[4 + c] = bw_s[(st * 4 + c) * 32 + lane];
+                    tmem_st8(region + (uint32_t)(GEMM_SFI_COLS * st), v);
                 }
+                __syncwarp();
+                mbar_arrive_w(bw_empty);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 mbar_arrive_w(&f_full[sb]);
+                bph ^= 1;
             } else {
                 uint32_t bw[SF_PD][SF_WORDS];
 #pragma unroll
@@ -527,8 +581,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
             }
             if (!ok) break;
-            __syncwarp();
-            mbar_arrive_w(&s_empty[sb]);
+            if constexpr (!SFI) {
+                __syncwarp();
+                mbar_arrive_w(&s_empty[sb]);
+            }
             if (++sb == 2) { sb = 0; sph ^= 1; }
         }
     } else if (warp >= 8) {
@@ -539,7 +595,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const int eg = (warp - 8) >> 2;
         const int tl = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        float *mval = meta_val + (warp - 8) * GEMM_NB_MAX;
+        float *mval = meta_val + (warp - 8) * NB;
         int db = 0;
         uint32_t dph = 0;
         bool ok = true;

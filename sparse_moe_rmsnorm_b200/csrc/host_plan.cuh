@@ -117,9 +117,10 @@ inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, in
     // per-item scale factors (and two MMA warps) when a stacked block's item
     // regions fit in TMEM next to four accumulators
     const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;
-    p.sf_item = p.stacked && gemm_tmem_cols_item(p.nb_rows, p.stacked, n_st) <= 512 ? 1 : 0;
+    p.sf_item = p.stacked && n_st <= GEMM_SFI_STAGES_MAX &&
+                gemm_tmem_cols_item(p.nb_rows, p.stacked, n_st) <= 512 ? 1 : 0;
     auto fits = [&](int ns) {
-        return gemm_smem_plan(p.K, E, p.nb_rows, ns).total <= GEMM_SMEM_LIMIT &&
+        return gemm_smem_plan(p.K, E, p.nb_rows, ns, p.sf_item).total <= GEMM_SMEM_LIMIT &&
                (p.sf_item || gemm_tmem_cols(p.nb_rows, p.stacked, ns) <= 512);
     };
     // as many stages as shared memory (and, per stage, TMEM) hold
@@ -127,7 +128,7 @@ inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, in
     while (ns > 2 && !fits(ns)) --ns;
     if (!fits(ns)) return MOE_ERR_ARG;
     p.n_stages = ns;
-    *smem = gemm_smem_plan(p.K, E, p.nb_rows, ns).total;
+    *smem = gemm_smem_plan(p.K, E, p.nb_rows, ns, p.sf_item).total;
     const long long P = (long long)T * top_k;
     const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
     const long long max_work = (long long)p.MB * max_blocks;

@@ -125,28 +125,35 @@ constexpr int GEMM_SMEM_LIMIT = 227 * 1024;
 
 // Shared-memory plan of the GEMM kernel (all offsets from a 1024-aligned base).
 struct GemmSmem {
-    int a_off, b_off, scale_off, amax_off, meta_off, bar_off, misc_off, total;
+    int a_off, b_off, scale_off, amax_off, meta_off, bsf_off, bar_off, misc_off, total;
 };
+
+// Per-item mode: the B scale words of one work item, staged in shared memory
+// for the scale-factor warps ([stage][4 columns][32 lanes] words).
+constexpr int GEMM_SFI_STAGES_MAX = 24;
+constexpr int GEMM_SFI_BSF_BYTES = GEMM_SFI_STAGES_MAX * 4 * 32 * 4;
 
 __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline int gemm_num_barriers(int n_stages) {
     // stage full/empty [NS], A-scale full/empty [2], D full [2 MMA warps][2], D empty [2],
-    // drain [2], epilogue exchange [2][2], item scale factors full/empty [2]
-    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4;
+    // drain [2], epilogue exchange [2][2], item scale factors full/empty [2], staged B words full/empty
+    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2;
 }
 
 __host__ __device__ inline int gemm_b_stage_bytes(int nb_rows) { return 2 * nb_rows * 128; }
 
-__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int n_stages) {
+__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int n_stages, int sf_item) {
     GemmSmem s;
     s.a_off = 0;
     s.b_off = n_stages * GEMM_A_STAGE;
     s.scale_off = s.b_off + n_stages * gemm_b_stage_bytes(nb_rows);
     const int scale_bytes = align_up(GEMM_BM * (K / 32), 128);
-    s.amax_off = s.scale_off + 2 * scale_bytes;
+    // A scale bytes: double-buffered per-stage mode (bulk copies one item ahead), one buffer per-item mode
+    s.amax_off = s.scale_off + (sf_item ? 1 : 2) * scale_bytes;
     s.meta_off = s.amax_off + 2 * 2 * 4 * 16 * 4;                 // [2 groups][2 parities][4 warps][16 columns] fp32
-    s.bar_off = s.meta_off + 8 * GEMM_NB_MAX * 4;                  // per epilogue warp: one value per column
+    s.bsf_off = s.meta_off + align_up(8 * nb_rows * 4, 16);        // per epilogue warp: one value per column
+    s.bar_off = s.bsf_off + (sf_item ? GEMM_SFI_BSF_BYTES : 0);
     s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_stages) * 8, 16);
     // misc: tmem base, abort flag, then counts/offsets/tiles caches
     s.total = s.misc_off + 16 + 3 * (E + 1) * 4;
