@@ -78,17 +78,66 @@ def committed_traffic(key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clocks and clock-event (throttle) reasons sampled while running (read only).
 
+    NVML is polled from a thread every millisecond, so that even a timed region
+    of a few milliseconds gets samples; nvidia-smi (every 200 ms) is the fallback
+    when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
+        self.samples = []          # (sm_mhz, sm_max_mhz, [reason names])
         self.proc = None
+        self.thread = None
+        self.nvml = None
+        self.handle = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.gpu)
+        try:
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _sample(self):
+        nv, h = self.nvml, self.handle
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((float(sm), float(self.max_mhz),
+                                 [n for n, attr in self.REASONS if getattr(nv, attr, 0) and (r & getattr(nv, attr))]))
+        except Exception:
+            pass
+
+    def _poll(self):
+        while not self.stop.is_set():
+            self._sample()
+            self.stop.wait(0.001)
 
     def __enter__(self):
+        import threading
+        try:
+            self.nvml, self.handle = self._nvml_handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+            self._sample()           # one reading as the timed region starts, one as it ends
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
@@ -98,7 +147,11 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.samples = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            self._sample()
+            return False
         if self.proc is None:
             return False
         self.proc.terminate()
@@ -107,22 +160,21 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        names = [n for n, _ in self.REASONS]
         for line in out.splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                self.samples.append((float(parts[1]), float(parts[2]),
+                                     [names[i] for i in range(4) if parts[5 + i].lower() == "active"]))
         return False
 
     def summary(self):
-        s = getattr(self, "samples", [])
+        s = self.samples
         if not s:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(p[1]) for p in s if p[1].replace(".", "").isdigit()]
-        mx = [float(p[2]) for p in s if p[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for p in s for i in range(4) if p[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(s)}
+        return {"sm_mhz": statistics.median(x[0] for x in s), "sm_max_mhz": max(x[1] for x in s),
+                "reasons": sorted({r for x in s for r in x[2]}), "samples": len(s),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def workload_config(name: str, T: int):
