@@ -443,14 +443,15 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
 //   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)).
 // Out: xq[plane][r][0:Kd] (plane 0 hi, plane 1 lo; columns d..Kd zero) and
 // xsf[g][plane][r] = the scale bytes of the 32-blocks 4g..4g+3 (byte i is
-// block 4g+i).  One warp per row; lane l takes the 32-blocks l, l+32, ...
+// block 4g+i).  A warp takes 32 consecutive 32-blocks of a row, one per lane.
 constexpr int GROUP_ROWS_MAX = 1024;   // expert-sorted rows per CTA, at most
 
-__device__ __forceinline__ void quant_row(const GroupParams &p, int r, int tok, int lane) {
+// Blocks b0 + lane (lane < 32) of expert-sorted row r, token tok.
+__device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int tok, int b0, int lane) {
     const float sc = p.rho[tok];
     const uint4 *src = reinterpret_cast<const uint4 *>(p.xn16 + (size_t)tok * p.d);
     const int nblk = p.d / 32, nblk_pad = p.Kd / 32;
-    for (int b0 = 0; b0 < nblk_pad; b0 += 32) {
+    {
         const int b = b0 + lane;
         uint32_t s_hi = 127, s_lo = 127;
         uint32_t qh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ql[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -635,7 +636,13 @@ __global__ void __launch_bounds__(1024) group_permute_kernel(const GroupParams p
     __syncthreads();
 
     // this CTA's rows of the B operand, one warp per row
-    for (int r = r0 + warp; r < r1; r += 32) quant_row(p, r, tok_s[r - r0], lane);
+    // this CTA's rows of the B operand: one warp per (row, 32 blocks of 32 elements), so
+    // that a row's loads are spread over warps rather than chained in one
+    const int parts = (p.Kd / 32 + 31) / 32;
+    for (int u = warp; u < (r1 - r0) * parts; u += 32) {
+        const int rr = u / parts;
+        quant_row_part(p, r0 + rr, tok_s[rr], (u - rr * parts) * 32, lane);
+    }
 }
 
 // --------------------------------------------------------------- combine
