@@ -270,6 +270,8 @@ int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale
     p.topk_w = c->topk_w;
     p.logits = c->logits;
     p.tok_done = c->tok_done;
+    p.err = c->err;
+    p.wait_limit_ns = c->wait_limit_ns;
     return cuda_status(launch_route(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -33,7 +33,8 @@ enum : unsigned int {
     ERR_WAIT_UP = 1u,      // a bounded wait ran out in the gate/up GEMM
     ERR_WAIT_DOWN = 2u,    // ... in the down GEMM
     ERR_WAIT_SELFTEST = 4u,
-    ERR_ROUTING = 8u       // an expert index out of range reached the grouping
+    ERR_ROUTING = 8u,      // an expert index out of range reached the grouping
+    ERR_WAIT_ROUTE = 16u   // a bounded wait ran out in the tensor-core router
 };
 
 struct RouteParams {
@@ -49,6 +50,8 @@ struct RouteParams {
     float *topk_w;              // [T, k]
     float *logits;              // fp32 [T, E] (decode-sized path: the CTAs' share of each token's logits)
     unsigned int *tok_done;     // [T] CTAs finished per token (decode-sized path); zero between calls
+    unsigned int *err;          // device error word (bounded waits of the tensor-core router)
+    unsigned long long wait_limit_ns;
 };
 
 struct GroupParams {

@@ -1,6 +1,7 @@
 // Routing side of the MoE block on sm_100a:
 //   route_kernel     RMSNorm + router logits + top-k + softmax over the chosen,
 //                    plus the fp16 normalised tokens for the experts;
+//   route_tc_kernel  the same for large batches, the router on tensor cores;
 //   route_small_kernel  the same for decode-sized batches, a CTA per (token,
 //                    16 experts);
 //   group_permute_kernel  expert histogram, exclusive scan and a stable
@@ -425,6 +426,329 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
     }
 }
 
+// ---------------------------------------- route, large batches (tensor cores)
+//
+// A CTA takes 128 tokens (the MMA's M) and all E experts (N = E padded to a
+// multiple of 16).  Per token, logit_e = (1/rms) * sum_j (x_j scale_j) W_r[e, j]
+// + b_e: xn . W_r[e] + b_e ("gpt-oss-20B" hub page, sections 3.2 and 3.4) with
+// the factor 1/rms taken out of the sum.  x_j scale_j, the product of two bf16
+// numbers, has at most 16 significant bits and is split exactly into bf16
+// hi + lo; two kind::f16 MMAs (hi . W, lo . W) per K step sum the exact
+// products in fp32 in the tensor core.  Eight producer warps copy 64-wide K
+// chunks of x and W_r ahead (cp.async), stage them (A hi, A lo, B = W_r rows;
+// 128-byte swizzled K-major) in a ring and
+// accumulate each token's sum of squares and max |x_j scale_j|; one warp
+// issues the MMAs; then four warps read the logits from TMEM (lane = token),
+// scale by 1/rms, add the bias and take the top-k (ties to the lower index,
+// NaN below every number) and the softmax in registers; last, xn16 = xn / rho
+// from a second read of the CTA's rows.
+constexpr int RT_TOK = 128;
+constexpr int RT_KC = 64;
+constexpr int RT_THREADS = 288;          // 8 producer warps + 1 MMA warp
+constexpr int RT_DEPTH = 4;              // K chunks of x and W_r in flight per producer thread
+
+__host__ __device__ inline int rt_npad(int E) { return E < 16 ? 16 : (E + 15) / 16 * 16; }
+__host__ __device__ inline int rt_stage_bytes(int npad) { return 2 * RT_TOK * 128 + npad * 128; }
+// The K chunks are spread over n_acc accumulators (contiguous groups), summed in
+// fp32 in the epilogue: the tensor core's accumulation over many MMAs is less
+// exact than fp32 additions, and a routing decision needs the logits to ~1e-5.
+__host__ __device__ inline int rt_n_acc(int npad) { return npad <= 64 ? 8 : 0; }
+__host__ __device__ inline int rt_tmem_cols(int npad) {
+    int c = 32;
+    while (c < rt_n_acc(npad) * npad) c <<= 1;
+    return c;
+}
+
+__global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RouteParams p, int npad, int nst) {
+    extern __shared__ uint8_t rt_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_raw) + 1023) & ~uintptr_t(1023));
+    const int stage_bytes = rt_stage_bytes(npad);
+    float *ss_s = reinterpret_cast<float *>(sm + nst * stage_bytes + RT_DEPTH * (RT_TOK + npad) * 128);   // [128]
+    float *mx_s = ss_s + RT_TOK;                                      // [128] max |x s|
+    uint64_t *full = reinterpret_cast<uint64_t *>(mx_s + RT_TOK);     // [nst]
+    uint64_t *empty = full + nst;                                     // [nst]
+    uint64_t *done = empty + nst;
+    uint32_t *tmem_s = reinterpret_cast<uint32_t *>(done + 1);
+    volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_s + 1);
+    // the RMSNorm scale row, bf16 [d], 16-byte aligned (it is read and written as uint4)
+    uint16_t *sc_s = reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(tmem_s + 2) + 15) & ~uintptr_t(15));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * RT_TOK;
+    const int ntok = min(RT_TOK, p.T - t0);
+    const int d = p.d, E = p.E, nk = d / RT_KC;
+    const int tcols = rt_tmem_cols(npad);
+    const int n_acc = min(rt_n_acc(npad), nk);       // accumulators in use
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nst; ++i) {
+            mbar_init(&full[i], 8);       // the eight producer warps
+            mbar_init(&empty[i], 1);      // MMA commit
+        }
+        mbar_init(done, 1);
+        *abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_s, tcols);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i < d / 8; i += RT_THREADS)
+        reinterpret_cast<uint4 *>(sc_s)[i] = __ldg(reinterpret_cast<const uint4 *>(p.norm_scale) + i);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_s;
+    const WaitCtl wc{abort_s, p.err, (unsigned)ERR_WAIT_ROUTE, p.wait_limit_ns};
+    // x may be the previous kernel's output
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp < 8) {
+        // ------------------------------------------------------------- producers
+        // Thread: 16-byte chunk c of rows rb + 32q (q < 4) of x, and chunks tid + 256q of
+        // W_r.  Each thread copies its own chunks RT_DEPTH K chunks ahead into a raw
+        // staging ring (cp.async, zero fill past the rows / experts) and later converts
+        // exactly those, so no other thread's copies are waited for.
+        const int c = threadIdx.x & 7;
+        const int rb = threadIdx.x >> 3;
+        const int nbt = npad * 8;                    // 16-byte chunks of B per K chunk
+        float ss[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {0.f, 0.f, 0.f, 0.f};
+        uint8_t *raw0 = sm + nst * stage_bytes;      // RT_DEPTH raw slots: x [128][128 B], W [npad][128 B]
+        const int raw_bytes = (RT_TOK + npad) * 128;
+        auto issue = [&](int kc) {
+            if (kc < nk) {
+                uint8_t *raw = raw0 + (kc % RT_DEPTH) * raw_bytes;
+                const int k0 = kc * RT_KC;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = rb + 32 * q;
+                    cp_async16(raw + r * 128 + 16 * c, p.x + (size_t)(t0 + min(r, ntok - 1)) * d + k0 + 8 * c,
+                               r < ntok ? 16u : 0u);
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int task = threadIdx.x + 256 * q;
+                    if (task < nbt) {
+                        const int e = task >> 3, cc = task & 7;
+                        cp_async16(raw + (RT_TOK + e) * 128 + 16 * cc, p.router_w + (size_t)min(e, E - 1) * d + k0 + 8 * cc,
+                                   e < E ? 16u : 0u);
+                    }
+                }
+            }
+            cp_async_commit();                       // (an empty group past the last chunk)
+        };
+#pragma unroll
+        for (int i = 0; i < RT_DEPTH - 1; ++i) issue(i);
+        int slot = 0;
+        uint32_t ph = 0;
+        for (int kc = 0; kc < nk; ++kc) {
+            issue(kc + RT_DEPTH - 1);
+            cp_async_wait<RT_DEPTH - 1>();           // this thread's copies of chunk kc have landed
+            const uint8_t *raw = raw0 + (kc % RT_DEPTH) * raw_bytes;
+            const uint4 sr = *reinterpret_cast<const uint4 *>(sc_s + kc * RT_KC + 8 * c);
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) break;
+            uint8_t *a_hi = sm + slot * stage_bytes;
+            uint8_t *a_lo = a_hi + RT_TOK * 128;
+            uint8_t *bs = a_lo + RT_TOK * 128;
+            float s8[8];
+            bf16x8_to_f32(sr, s8);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = rb + 32 * q;
+                float f[8];
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(raw + r * 128 + 16 * c), f);
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float p0 = f[2 * i] * s8[2 * i], p1 = f[2 * i + 1] * s8[2 * i + 1];
+                    ss[q] += f[2 * i] * f[2 * i] + f[2 * i + 1] * f[2 * i + 1];
+                    mx[q] = fmaxf(mx[q], fmaxf(fabsf(p0), fabsf(p1)));
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    const float2 hf = __bfloat1622float2(h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                    hw[i] = *reinterpret_cast<const uint32_t *>(&h2);
+                    lw[i] = *reinterpret_cast<const uint32_t *>(&l2);
+                }
+                const int off = r * 128 + ((c ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4 *>(a_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(a_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int task = threadIdx.x + 256 * q;
+                if (task < nbt) {
+                    const int e = task >> 3, cc = task & 7;
+                    *reinterpret_cast<uint4 *>(bs + e * 128 + ((cc ^ (e & 7)) << 4)) =
+                        *reinterpret_cast<const uint4 *>(raw + (RT_TOK + e) * 128 + 16 * cc);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            mbar_arrive_w(&full[slot]);
+            if (++slot == nst) { slot = 0; ph ^= 1; }
+        }
+        cp_async_wait<0>();
+        // the row statistics: the eight threads of a row are consecutive lanes
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float a = ss[q], m = mx[q];
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            }
+            if (c == 0) {
+                ss_s[rb + 32 * q] = a;
+                mx_s[rb + 32 * q] = m;
+            }
+        }
+    } else {
+        // --------------------------------------------------------------- MMA issue
+        // kind::f16: D f32 (1 << 4), A bf16 (1 << 7), B bf16 (1 << 10), K-major, N >> 3, M >> 4
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(npad >> 3) << 17) |
+                               ((uint32_t)(RT_TOK >> 4) << 24);
+        int slot = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int kc = 0; kc < nk; ++kc) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
+            tc_fence_after();
+            uint8_t *a_hi = sm + slot * stage_bytes;
+            const uint64_t dh = smem_desc_sw128(smem_addr(a_hi));
+            const uint64_t dl = smem_desc_sw128(smem_addr(a_hi + RT_TOK * 128));
+            const uint64_t db = smem_desc_sw128(smem_addr(a_hi + 2 * RT_TOK * 128));
+            // accumulator a takes chunks [a nk / n_acc, (a + 1) nk / n_acc)
+            const int a = kc * n_acc / nk;
+            const bool first = kc == 0 || (kc - 1) * n_acc / nk != a;
+            const uint32_t dacc = tmem + (uint32_t)(a * npad);
+#pragma unroll
+            for (int ks = 0; ks < RT_KC / 16; ++ks) {      // K = 16 per MMA: 32 bytes of a row
+                mma_f16_ss_w(dacc, dh + 2 * ks, db + 2 * ks, idesc, (first && ks == 0) ? 0u : 1u);
+                mma_f16_ss_w(dacc, dl + 2 * ks, db + 2 * ks, idesc, 1u);
+            }
+            mma_commit_w(&empty[slot]);
+            if (++slot == nst) { slot = 0; ph ^= 1; }
+        }
+        // arrives once every MMA issued above has completed (also on the abort path,
+        // where the epilogue sees the abort and skips the logits)
+        mma_commit_w(done);
+        if (!ok) {
+            const uint64_t start = globaltimer_ns();
+            while (!mbar_try_wait(done, 0) && globaltimer_ns() - start < p.wait_limit_ns) {
+            }
+        }
+    }
+    __syncthreads();                               // row statistics in shared memory
+
+    if (warp < 4) {
+        // ---------------------------------------------------- logits, top-k, softmax
+        const int row = 32 * warp + lane;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, wc));
+        tc_fence_after();
+        if (ok) {
+            const float r = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);
+            float bl[8];
+            int be[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                bl[i] = -INFINITY;
+                be[i] = -1;                        // empty
+            }
+            const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+            for (int c0 = 0; c0 < npad; c0 += 16) {
+                float sum[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+                for (int a = 0; a < n_acc; ++a) {
+                    uint32_t v[16];
+                    tmem_ld16(lane_base + (uint32_t)(a * npad + c0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(v[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    int e = c0 + i;
+                    if (e < E) {
+                        float l = sum[i] * r + p.router_b[e];
+                        if (l != l) l = -INFINITY;
+                        // sorted insertion: a later (higher) index never passes an equal logit
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (j < p.k && e >= 0 && (be[j] < 0 || l > bl[j])) {
+                                const float tl = bl[j];
+                                const int te = be[j];
+                                bl[j] = l;
+                                be[j] = e;
+                                l = tl;
+                                e = te;
+                            }
+                        }
+                    }
+                }
+            }
+            if (row < ntok) {
+                const int t = t0 + row;
+                float wsum = 0.f, wv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j < p.k) {
+                        wv[j] = expf(bl[j] - bl[0]);
+                        wsum += wv[j];
+                    }
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j < p.k) {
+                        p.topk_idx[(size_t)t * p.k + j] = be[j];
+                        p.topk_w[(size_t)t * p.k + j] = wv[j] / wsum;
+                    }
+            }
+        }
+    }
+    // xn16 = xn / rho, rho a power of two with max|xn| / rho in [2^13, 2^14); the
+    // per-row factors first, then every (row, 8-element chunk) with loads in flight
+    if (threadIdx.x < RT_TOK) {
+        const int row = threadIdx.x;
+        const float r = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);
+        const float amax = mx_s[row] * r;
+        float rho = 1.f, inv_rho = 1.f;
+        if (amax > 0.f && amax <= FLT_MAX) {
+            int ex;
+            frexpf(amax, &ex);                     // amax in [2^(ex-1), 2^ex)
+            rho = exp2i(ex - 14);
+            inv_rho = exp2i(14 - ex);
+        }
+        if (row < ntok) p.rho[t0 + row] = rho;
+        ss_s[row] = r;                             // reused: 1/rms
+        mx_s[row] = inv_rho;                       // reused: 1/rho
+    }
+    __syncthreads();
+    {
+        const int nch = d / 8;
+        const int total = ntok * nch;
+#pragma unroll 2
+        for (int i = threadIdx.x; i < total; i += RT_THREADS) {
+            const int row = i / nch, cc = i - row * nch;
+            const float r = ss_s[row], ir = mx_s[row];
+            float f[8], sc[8];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + row) * d) + cc), f);
+            bf16x8_to_f32(reinterpret_cast<const uint4 *>(sc_s)[cc], sc);
+            uint32_t hw[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __half2 h2 = __floats2half2_rn(f[2 * q] * r * sc[2 * q] * ir, f[2 * q + 1] * r * sc[2 * q + 1] * ir);
+                hw[q] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            reinterpret_cast<uint4 *>(p.xn16 + (size_t)(t0 + row) * d)[cc] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, (uint32_t)tcols);
+    }
+}
+
 // ------------------------------------------------------- group + permute
 //
 // Grid of G CTAs of 32 warps.  Every CTA computes the whole grouping of the
@@ -745,8 +1069,25 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
     if (p.T <= 512 && p.d <= ROUTE_SMALL_CHUNKS * 256 && p.logits && p.tok_done) {
         return launch_pdl(route_small_kernel, dim3(p.T, (p.E + 15) / 16), dim3(512), 0, s, p);
     }
-    // few tokens: one token per CTA, 32 warps (latency); many tokens: the
-    // router weights are reused across 8 (or 4) tokens of a CTA (throughput)
+    // large batches: the tensor-core router, 128 tokens per CTA (from 4096 tokens,
+    // where its grid covers enough SMs to beat the CUDA-core router below)
+    if (p.T >= 4096 && p.err && rt_n_acc(rt_npad(p.E)) > 0) {
+        const int npad = rt_npad(p.E);
+        const int sb = rt_stage_bytes(npad);
+        const int fixed = RT_DEPTH * (RT_TOK + npad) * 128 + 2 * RT_TOK * 4 + 16 * 8 + 64 + 2 * p.d + 1024;
+        // (raw ring, statistics, barriers, the scale row, alignment slack)
+        int nst = (220 * 1024 - fixed) / sb;
+        if (nst > 4) nst = 4;
+        if (nst >= 2) {
+            const int smem = nst * sb + fixed;
+            cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            return launch_pdl(route_tc_kernel, dim3((p.T + RT_TOK - 1) / RT_TOK), dim3(RT_THREADS), (size_t)smem, s,
+                              p, npad, nst);
+        }
+    }
+    // otherwise: one token per CTA, 32 warps (few tokens); the router weights
+    // reused across 8 (or 4) tokens of a CTA (many tokens)
     if (p.T <= 512 || (size_t)8 * (p.d + p.E) * 4 > 200 * 1024) return launch_route_cfg<1, 32, 8, 8>(p, s);
     if (p.E <= 128) return launch_route_cfg<8, 16, 8, 4>(p, s);
     return launch_route_cfg<4, 32, 8, 4>(p, s);

@@ -139,7 +139,10 @@ def _assert_same_e4m3(got, want, what):
     assert same.all(), what
 
 
-@pytest.mark.parametrize("T,d,E,k", [(16, 128, 8, 4), (37, 2880, 32, 4), (600, 2880, 128, 4), (2100, 256, 64, 8)])
+# decode-sized (a CTA per token and 16 experts), the CUDA-core router (T 513..4095) and the
+# tensor-core router (T >= 4096), including E not a multiple of 16 and a ragged last token block
+@pytest.mark.parametrize("T,d,E,k", [(16, 128, 8, 4), (37, 2880, 32, 4), (600, 2880, 128, 4), (2100, 256, 64, 8),
+                                     (4200, 256, 40, 8), (4096, 2880, 32, 4)])
 def test_route_stage(T, d, E, k):
     inp = custom_layer(T=T, d=d, F=64, E=E, k=k, seed=T)
     w = moe.MoEWeights.from_numpy(inp)
