@@ -304,11 +304,16 @@ def run_ours(args, rank, world, local_rank):
     up_events = []
 
     def step(timed=False):
-        """One step: the block on every layer, through the five stage calls moe_forward is made
-        of (so that the gate/up GEMM can be bracketed by events on the launching stream)."""
+        """One step: the block on every layer.  timed=False: moe_forward (the public call);
+        timed=True: the five stage calls moe_forward is made of, with the gate/up GEMM
+        bracketed by events on the launching stream."""
         cur = x
         for l, w in enumerate(weights):
             out = bufs[l % 2]
+            if not timed:
+                m.forward(cur, w, y=out)
+                cur = out
+                continue
             moe.moe_route(m.ctx, T, cur, w.norm_scale, w.router_w, w.router_b, cfg.k)
             moe.moe_group(m.ctx, T, cfg.k)
             if timed:
@@ -337,12 +342,16 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clocks:
         ev0.record(stream)
         for _ in range(args.steps):
-            step(timed=True)
+            step()
         ev1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    # ---- the dominant kernel: K more steps, its launches bracketed by events
+    for _ in range(args.steps):
+        step(timed=True)
+    torch.cuda.synchronize()
     up_ms_live = sum(a.elapsed_time(b) for a, b in up_events) / max(len(up_events), 1)
     ms_per_step = ms_total / args.steps
     value = job_tokens_per_s(ms_total, T, args.steps, world)
