@@ -234,6 +234,7 @@ SHAPES = [
     dict(T=300, d=128, F=192, E=2, k=1),         # n_e > 192: several token blocks per expert
     dict(T=700, d=320, F=640, E=8, k=4),         # token blocks of 192, ragged tails
     dict(T=50, d=2880, F=2880, E=32, k=4),
+    dict(T=24, d=384, F=256, E=32, k=4),         # about 3 tokens per expert
 ]
 
 
@@ -281,7 +282,8 @@ def _np_swiglu(gate, lin):
     return g / (1.0 + np.exp(-1.702 * g)) * (u + 1.0)
 
 
-@pytest.mark.parametrize("T,d,F,E,k", [(16, 128, 128, 8, 4), (50, 2880, 2880, 32, 4), (300, 192, 320, 4, 2)])
+@pytest.mark.parametrize("T,d,F,E,k", [(16, 128, 128, 8, 4), (50, 2880, 2880, 32, 4), (300, 192, 320, 4, 2),
+                                         (24, 256, 320, 32, 4)])
 def test_up_stage_h_encoding(T, d, F, E, k):
     """The gate/up GEMM + SwiGLU epilogue against float64 on the same (decoded) operands: h, read back
     from its two-term E4M3 encoding, within the encoding's rounding of the float64 value (2^-9 of the
@@ -321,6 +323,14 @@ def test_up_stage_h_encoding(T, d, F, E, k):
     print("h max err / block max", float(np.max(err / np.maximum(blk_max, 1e-30))))
     assert np.all(err <= bound)
     m.close()
+
+
+def test_decode_blocks_several_per_expert():
+    """Decode-sized token blocks when the router sends most tokens to a few experts: those experts
+    take several blocks each, the last one ragged."""
+    inp = custom_layer(T=48, d=512, F=384, E=64, k=4, seed=21)
+    inp["router_b"][:8] += 4.0
+    check(inp, 4, label="skewed decode blocks")
 
 
 def test_tied_logits_pick_lower_index():
