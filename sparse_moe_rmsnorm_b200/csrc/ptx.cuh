@@ -59,6 +59,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete may
+// sleep in the barrier unit, up to `hint_ns`, until the phase completes,
+// instead of polling (polling warps take issue slots and shared-memory
+// pipe cycles from the producer and MMA warps of the same SM).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t MBAR_SUSPEND_HINT_NS = 1000000;   // 1 ms per sleep; the wait limit is checked after each
+
 // Shared state of the bounded waits of one CTA.  `abort` lives in shared
 // memory: once any thread's wait runs out, every other wait in the CTA gives
 // up at its next poll.
@@ -73,19 +89,14 @@ struct WaitCtl {
 // CTA has aborted or this wait ran out (which aborts the CTA).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t start = 0;
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, MBAR_SUSPEND_HINT_NS)) return true;
         if (*w.abort) return false;
-        if ((it & 63u) == 0) {
-            uint64_t now = globaltimer_ns();
-            if (start == 0) {
-                start = now;
-            } else if (now - start > w.limit_ns) {
-                *w.abort = 1;
-                atomicOr(w.err, w.err_bit);
-                return false;
-            }
+        if (globaltimer_ns() - start > w.limit_ns) {
+            *w.abort = 1;
+            atomicOr(w.err, w.err_bit);
+            return false;
         }
     }
 }
