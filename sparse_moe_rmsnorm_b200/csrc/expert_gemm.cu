@@ -414,13 +414,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         bool ok = true;
         const int n_sfb = p.stacked ? (2 * NB + 31) / 32 : (NB + 31) / 32;
         uint32_t bph = 0;                    // phase parity of the staging barriers (one phase per item)
-        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-            Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
-            // B scale words of stage st into v: stacked, word c is row 32c + lane of
-            // [hi rows | lo rows]; otherwise words 2c / 2c + 1 are the hi / lo word
-            // of token row 32c + lane.  Rows past the block's tokens get 2^0.
-            auto load_bsf = [&](int st, uint32_t (&v)[SF_WORDS]) {
+        // B scale words of stage st of item t into v: stacked, word c is row 32c + lane of
+        // [hi rows | lo rows]; otherwise words 2c / 2c + 1 are the hi / lo word
+        // of token row 32c + lane.  Rows past the block's tokens get 2^0.
+        auto load_bsf = [&](const Work &t, int st, uint32_t (&v)[SF_WORDS]) {
                 const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
 #pragma unroll
                 for (int i = 0; i < SF_WORDS; ++i) v[i] = 0x7F7F7F7Fu;
@@ -442,7 +439,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         }
                     }
                 }
-            };
+        };
+        // per-stage mode: stage st's B words sit in bw[st % SF_PD], loaded SF_PD stages
+        // ahead; the slots an item's last stages free take the next item's first stages
+        uint32_t bw[SF_PD][SF_WORDS];
+        if constexpr (!SFI) {
+            if (blockIdx.x < total) {
+                Work t0;
+                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t0);
+#pragma unroll
+                for (int i = 0; i < SF_PD; ++i)
+                    if (i < n_st) load_bsf(t0, i, bw[i]);
+            }
+        }
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Work t;
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
             if constexpr (!SFI) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
             }
@@ -542,10 +554,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 mbar_arrive_w(&f_full[sb]);
                 bph ^= 1;
             } else {
-                uint32_t bw[SF_PD][SF_WORDS];
-#pragma unroll
-                for (int i = 0; i < SF_PD; ++i)
-                    if (i < n_st) load_bsf(i, bw[i]);
+                Work tn;
+                const bool has_next = w + (int)gridDim.x < total;
+                if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, tn);
                 for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
 #pragma unroll
                     for (int i = 0; i < SF_PD; ++i) {
@@ -572,7 +583,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                                 }
                         }
                         tmem_wait_st();
-                        if (st + SF_PD < n_st) load_bsf(st + SF_PD, bw[i]);
+                        if (st + SF_PD < n_st) load_bsf(t, st + SF_PD, bw[i]);
+                        else if (has_next && i < n_st) load_bsf(tn, i, bw[i]);
                         tc_fence_before();
                         __syncwarp();
                         mbar_arrive_w(&full[slot]);
