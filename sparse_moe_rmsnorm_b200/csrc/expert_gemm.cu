@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const int n_sfb = p.stacked ? (2 * NB + 31) / 32 : (NB + 31) / 32;
         uint32_t bph = 0;                    // phase parity of the staging barriers (one phase per item)
         // B scale words of stage st of item t into v: stacked, word c is row 32c + lane of
-        // [hi rows | lo rows]; otherwise words 2c / 2c + 1 are the hi / lo word
+        // [hi rows | lo rows]; otherwise words c / 6 + c are the hi / lo word
         // of token row 32c + lane.  Rows past the block's tokens get 2^0.
         auto load_bsf = [&](const Work &t, int st, uint32_t (&v)[SF_WORDS]) {
                 const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
@@ -434,8 +434,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     for (int c = 0; c < SF_WORDS / 2; ++c) {
                         const int j = 32 * c + lane;
                         if (c < n_sfb && j < t.n_valid) {
-                            v[2 * c] = __ldg(bsf + j);
-                            v[2 * c + 1] = __ldg(bsf + p.P_max + j);
+                            v[c] = __ldg(bsf + j);
+                            v[SF_WORDS / 2 + c] = __ldg(bsf + p.P_max + j);
                         }
                     }
                 }
@@ -569,18 +569,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                             a_words(st, v);
                             tmem_st4(sf, v);
                         }
-                        // B: the hi (and lo) columns of the token block
+                        // B: the hi (and lo) columns of the token block, one store per
+                        // 4- or 8-column group (columns past the block's hold 2^0)
+                        // (hi words in bw[i][0..5], lo words in bw[i][6..11]; columns 14 and
+                        // 15 take two lo words, past any block's hi columns)
+                        const uint32_t *b = bw[i];
                         if (p.stacked) {
-#pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                if (c < n_sfb) tmem_st1(sf + 8 + (uint32_t)c, bw[i][c]);
+                            tmem_st4v(sf + 8, b[0], b[1], b[2], b[3]);
                         } else {
-#pragma unroll
-                            for (int c = 0; c < SF_WORDS / 2; ++c)
-                                if (c < n_sfb) {
-                                    tmem_st1(sf + 8 + (uint32_t)c, bw[i][2 * c]);
-                                    tmem_st1(sf + 16 + (uint32_t)c, bw[i][2 * c + 1]);
-                                }
+                            tmem_st8v(sf + 8, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7]);
+                            tmem_st4v(sf + 16, b[6], b[7], b[8], b[9]);
+                            tmem_st2v(sf + 20, b[10], b[11]);
                         }
                         tmem_wait_st();
                         if (st + SF_PD < n_st) load_bsf(t, st + SF_PD, bw[i]);
