@@ -10,7 +10,8 @@
 //     thread touches a weight element: the tensor core applies the E8M0 block
 //     scales itself ("MXFP4": 32 elements share one power of two, pnsm.cn
 //     overview sections 1 and 4).  A K tail of 64 (K = 2880 = 22.5 x 128) is
-//     copied and unpacked by the scale-factor warps.
+//     loaded by the A producer with plain loads at the item's start and written
+//     into its stage's slot in the unpacked layout.
 //   B (activations, N = tokens): two E4M3 terms, hi = e4m3(v / 2^s) and
 //     lo = e4m3((v - hi 2^s) / 2^(s-4)), per 32-element block with E8M0 scale
 //     s chosen so the block maximum fits 448.  hi + lo keeps about 8
@@ -18,10 +19,11 @@
 //     and lo rows of a token block sit one after the other in the B ring; small
 //     blocks feed both in one MMA (N = 2 x rows, the epilogue adds the halves),
 //     large ones in two MMAs into the same accumulator.
-//   Scale factors: per stage the scale-factor warps write A's and B's E8M0
-//     bytes into a TMEM slot, one 32-bit column per 32 rows, the byte index
-//     being the 32-block within the stage, replicated in all four lane
-//     quarters (the layout the block-scaled MMA reads).
+//   Scale factors: the scale-factor warps write A's and B's E8M0 bytes into
+//     TMEM, one 32-bit column per 32 rows, the byte index being the 32-block
+//     within the stage, replicated in all four lane quarters (the layout the
+//     block-scaled MMA reads): per stage into a slot of a ring, or per work
+//     item into one of two item regions.
 // Gate/up epilogue: z = D + b13, clamped SwiGLU
 //   h = min(g,7) * sigmoid(1.702 min(g,7)) * (clamp(u,-7,7) + 1)
 //   ("gpt-oss-20B" hub page, section 3.3).  Each 128-row weight block holds 64
@@ -34,12 +36,13 @@
 //   combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
 //
 // Warp roles (512 threads): 0 TMA producer of A (weights), 3 TMA producer of
-// B (activations), 1 MMA issue, 2 TMEM allocation, 4-7 scale-factor warps (one
-// per TMEM lane quarter), 8-11 and 12-15 two epilogue groups taking 16-column
-// chunks in turn.  Producers and MMA run as whole converged warps, one elected
-// lane issuing.  Every mbarrier wait is
-// bounded (WaitCtl); when one runs out the CTA stops issuing work, drains its
-// copies and MMAs in flight, frees TMEM and returns with the error latched.
+// B (activations), 1 MMA issue, 2 TMEM allocation and (per-item scale factors)
+// the second MMA warp, 4-7 scale-factor warps (one per TMEM lane quarter),
+// 8-11 and 12-15 two epilogue groups taking 16-column chunks in turn.
+// Producers and MMA run as whole converged warps, one elected lane issuing.
+// Every mbarrier wait is bounded (WaitCtl); when one runs out the CTA stops
+// issuing work, drains its copies and MMAs in flight, frees TMEM and returns
+// with the error latched.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
