@@ -187,13 +187,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         tmem_alloc(tmem_base_s, 512);
         tmem_relinquish();
     }
-    // the routing arrays and the B operand come from the kernels before this one
-    pdl_wait();
+    // The routing arrays come from the group kernel and the B operand from the
+    // kernel before this one.  The gate/up GEMM follows the group kernel and
+    // waits for it here.  The down GEMM follows the gate/up GEMM, which starts
+    // its dependents only once it has itself waited for the group kernel: so
+    // the down GEMM reads the routing arrays (from L2) at once, and only its
+    // B producer and the loads of B scale words wait for the gate/up GEMM.
+    // Its weight copies and weight scales start while the gate/up GEMM's last
+    // CTAs finish.
+    if constexpr (MODE == MODE_UP) pdl_wait();
     pdl_trigger();
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
-        counts_s[i] = i < p.E ? p.counts[i] : 0;
-        offsets_s[i] = p.offsets[i];
-        tiles_s[i] = p.tiles[i];
+        counts_s[i] = i < p.E ? __ldcg(p.counts + i) : 0;
+        offsets_s[i] = __ldcg(p.offsets + i);
+        tiles_s[i] = __ldcg(p.tiles + i);
     }
     tc_fence_before();
     __syncthreads();
@@ -307,6 +314,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // --------------------------------------------- B producer (activations)
         // Per stage one TMA box: the token block's hi rows and then its lo rows.
         if (lane == 0) tma_prefetch_desc(&p.map_b);
+        if constexpr (MODE == MODE_DOWN) pdl_wait();     // h comes from the gate/up GEMM
         int slot = 0;
         uint32_t ph = 0;
         long long issued = 0;
@@ -447,6 +455,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // ahead; the slots an item's last stages free take the next item's first stages
         uint32_t bw[SF_PD][SF_WORDS];
         if constexpr (!SFI) {
+            if constexpr (MODE == MODE_DOWN) pdl_wait();     // h's scales come from the gate/up GEMM
             if (blockIdx.x < total) {
                 Work t0;
                 work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t0);
@@ -506,6 +515,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     if (wi < n16) sreg[i] = __ldg(run0 + wi);
                     else if (MODE == MODE_UP && wi < n_words) sreg[i] = __ldg(run1 + (wi - n16));
                 }
+                if constexpr (MODE == MODE_DOWN) pdl_wait();   // h's scales come from the gate/up GEMM
                 uint32_t bwr[GEMM_SFI_STAGES_MAX / 4][4];
 #pragma unroll
                 for (int i = 0; i < GEMM_SFI_STAGES_MAX / 4; ++i) {
