@@ -123,7 +123,10 @@ MOE_API int moe_forward(moe_ctx_t *ctx, int T,
  *                    fixed order, so results are reproducible run to run.
  * They exist for per-stage timing and tests; intermediate results stay in the
  * context's workspace (see moe_copy_workspace).  moe_finalize needs the same
- * x that moe_route was given. */
+ * x that moe_route was given.  moe_expert_down reads the routing arrays before
+ * it waits for the kernel before it: call it right after moe_expert_up (a call
+ * in another order computes nothing useful, but every row index it uses stays
+ * inside the workspace). */
 MOE_API int moe_route(moe_ctx_t *ctx, int T, const uint16_t *x, const uint16_t *norm_scale,
               const uint16_t *router_w, const float *router_b, int top_k, void *stream);
 MOE_API int moe_group(moe_ctx_t *ctx, int T, int top_k, void *stream);

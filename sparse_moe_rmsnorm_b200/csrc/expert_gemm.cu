@@ -56,7 +56,7 @@ struct Work {
 };
 
 __device__ __forceinline__ void work_of(int w, const int *tiles_s, const int *counts_s, const int *offsets_s, int E,
-                                        int MB, int nb_rows, Work &t) {
+                                        int MB, int nb_rows, int P_max, Work &t) {
     // the last expert e with MB * tiles[e] <= w has at least one token block
     int lo = 0, hi = E - 1;
     while (lo < hi) {
@@ -71,7 +71,10 @@ __device__ __forceinline__ void work_of(int w, const int *tiles_s, const int *co
     const int nb = local - t.mb * nblk;
     t.p0 = offsets_s[e] + nb * nb_rows;
     t.n_valid = min(nb_rows, counts_s[e] - nb * nb_rows);
-    t.n_mma = (t.n_valid + 15) & ~15;
+    // never past the row buffers, even for routing arrays that do not match (the down
+    // GEMM reads them before its dependency wait; see the kernel's prologue)
+    t.n_valid = max(0, min(t.n_valid, P_max - t.p0));
+    t.n_mma = max(16, (t.n_valid + 15) & ~15);     // a valid MMA width (16..nb_rows) in any case
 }
 
 __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         };
         Work t;
         if (blockIdx.x < total) {
-            work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             if constexpr (!SFI) ok = load_scales(t);     // per-item mode: the scale-factor warps load them
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (n_st > n_main) load_tail();
             Work tn;
             if (w + (int)gridDim.x < total) {
-                work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, tn);
+                work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
                 if constexpr (!SFI) {
                     if (!load_scales(tn)) { ok = false; break; }
                 }
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             for (int st = 0; st < n_st; ++st) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                 mbar_arrive_expect_tx_w(&full[slot], b_bytes);
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         };
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             const bool stacked = SFI || p.stacked;     // per-item mode always stacks hi and lo rows
             const uint32_t n = stacked ? (uint32_t)(2 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
@@ -458,7 +461,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if constexpr (MODE == MODE_DOWN) pdl_wait();     // h's scales come from the gate/up GEMM
             if (blockIdx.x < total) {
                 Work t0;
-                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t0);
+                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t0);
 #pragma unroll
                 for (int i = 0; i < SF_PD; ++i)
                     if (i < n_st) load_bsf(t0, i, bw[i]);
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             if constexpr (!SFI) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
             }
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             } else {
                 Work tn;
                 const bool has_next = w + (int)gridDim.x < total;
-                if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, tn);
+                if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
                 for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
 #pragma unroll
                     for (int i = 0; i < SF_PD; ++i) {
@@ -627,7 +630,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         uint32_t ex_ph = 0;                  // bit i: phase parity of exchange buffer i
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, t);
+            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             const int wrow = tile_weight_row<MODE>(tl, t.mb, p.F);
             const bool row_valid = wrow < p.R;
             const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + wrow]) : 0.f;
