@@ -980,15 +980,33 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                                                       int T, int d, int k) {
     const int per_tok = d / 8;
     const long long n = (long long)T * per_tok;
+    // x (the block's input) and pair_row (from the group kernel, which finished before
+    // the GEMMs started) are final before this kernel launches: the first unit's
+    // loads of them go out before the wait for the down GEMM's rows
+    long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    uint4 xv = make_uint4(0, 0, 0, 0);
+    int prow[8];
+    if (i < n) {
+        const int t = (int)(i / per_tok), j = (int)(i % per_tok) * 8;
+        xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * d + j);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) prow[s] = s < k ? __ldcg(pair_row + (size_t)t * k + s) : 0;
+    }
     pdl_wait();
     pdl_trigger();
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-         i += (long long)gridDim.x * blockDim.x) {
+    for (bool first = true; i < n; i += (long long)gridDim.x * blockDim.x, first = false) {
         const int t = (int)(i / per_tok), j = (int)(i % per_tok) * 8;
         float acc[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(x + (size_t)t * d + j), acc);
-        for (int s = 0; s < k; ++s) {
-            const float4 *o = reinterpret_cast<const float4 *>(orows + (size_t)pair_row[(size_t)t * k + s] * d + j);
+        if (!first) {
+            xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * d + j);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) prow[s] = s < k ? pair_row[(size_t)t * k + s] : 0;
+        }
+        bf16x8_to_f32(xv, acc);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            if (s >= k) break;
+            const float4 *o = reinterpret_cast<const float4 *>(orows + (size_t)prow[s] * d + j);
             const float4 a = o[0], b = o[1];
             acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
             acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
