@@ -188,6 +188,18 @@ MOE_API int moe_selftest_wait_timeout(moe_ctx_t *ctx, void *stream);
  * grouped GEMMs hand the codes and scales to the tensor core as they are. */
 MOE_API int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, void *stream);
 
+/* The launch plan of one grouped-GEMM stage, computed on the host alone (no
+ * device call), as the library makes it for a call: mode 0 (gate/up) or 1
+ * (down), T tokens, top_k, the layer shape, P_max workspace rows (>= T*top_k)
+ * and num_sms SMs.  Writes out[0..9] = {token rows per work item, hi and lo
+ * rows stacked in one MMA (0/1), shared-memory ring stages, per-item scale
+ * factors (0/1), grid size, dynamic shared memory bytes, TMEM columns used,
+ * full 128-wide K stages, K stages, weight-row blocks per expert}.  Shape
+ * limits as moe_init; returns MOE_ERR_ARG for bad arguments or a plan that
+ * does not fit.  For tests of the planner. */
+MOE_API int moe_debug_plan(int mode, int T, int top_k, int d_model, int d_ff, int n_experts, int P_max, int num_sms,
+                           int *out);
+
 /* The whole block (as moe_forward) without any device allocation, for callers
  * that cannot call cudaMalloc: code running inside a CUDA graph capture that
  * forbids allocation, frameworks whose allocator owns all device memory, or

@@ -22,7 +22,7 @@ __all__ = [
     "MoEError", "MoEShape", "MoEWeights", "MoE", "lib", "library_path",
     "moe_init", "moe_destroy", "moe_forward", "moe_route", "moe_group", "moe_expert_up", "moe_expert_down",
     "moe_finalize", "moe_copy_workspace", "moe_sync_status", "moe_set_wait_limit_ns",
-    "moe_selftest_wait_timeout", "moe_debug_decode", "moe_strerror", "moe_version", "WS",
+    "moe_selftest_wait_timeout", "moe_debug_decode", "moe_debug_plan", "moe_strerror", "moe_version", "WS",
     "moe_forward_noalloc", "MOE_NOALLOC_MAX_TOKENS",
 ]
 
@@ -72,6 +72,7 @@ _SIGS = {
     "moe_debug_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_void_p, ctypes.c_void_p]),
     "moe_forward_noalloc": (ctypes.c_int, [ctypes.c_int] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 12),
+    "moe_debug_plan": (ctypes.c_int, [ctypes.c_int] * 8 + [ctypes.c_void_p]),
     "moe_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_version": (ctypes.c_char_p, []),
 }
@@ -197,6 +198,19 @@ def moe_selftest_wait_timeout(ctx, stream=None) -> None:
 def moe_debug_decode(codes, scales, R, K, out, stream=None) -> None:
     _check(lib().moe_debug_decode(_ptr(codes), _ptr(scales), int(R), int(K), _ptr(out), _stream(stream)),
            "moe_debug_decode")
+
+
+PLAN_FIELDS = ("nb_rows", "stacked", "n_stages", "sf_item", "grid", "smem", "tmem_cols", "k_full_stages",
+               "k_stages", "row_blocks")
+
+
+def moe_debug_plan(mode: int, T: int, top_k: int, d_model: int, d_ff: int, n_experts: int, P_max: int,
+                   num_sms: int) -> Dict[str, int]:
+    """The grouped-GEMM launch plan of one stage (mode 0 gate/up, 1 down), computed on the host."""
+    out = (ctypes.c_int * len(PLAN_FIELDS))()
+    _check(lib().moe_debug_plan(int(mode), int(T), int(top_k), int(d_model), int(d_ff), int(n_experts), int(P_max),
+                                int(num_sms), out), "moe_debug_plan")
+    return dict(zip(PLAN_FIELDS, list(out)))
 
 
 # ------------------------------------------------------------- torch layer

@@ -397,4 +397,28 @@ int moe_debug_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, 
     return cuda_status(launch_decode(codes, scales, R, K, out, static_cast<cudaStream_t>(stream)));
 }
 
+int moe_debug_plan(int mode, int T, int top_k, int d, int F, int E, int P_max, int num_sms, int *out) {
+    if (!out || (mode != MODE_UP && mode != MODE_DOWN) || T < 1 || num_sms < 1) return MOE_ERR_ARG;
+    if (d < 64 || d > 6144 || d % 64 || F < 64 || F > 6144 || F % 64) return MOE_ERR_ARG;
+    if (E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return MOE_ERR_ARG;
+    if ((long long)T * top_k > P_max || P_max > (1 << 30)) return MOE_ERR_ARG;
+    GemmParams p;
+    memset(&p, 0, sizeof p);
+    int grid = 0, smem = 0;
+    const int rc = plan_gemm(p, mode, T, top_k, d, F, E, P_max, num_sms, &grid, &smem);
+    if (rc) return rc;
+    const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;
+    out[0] = p.nb_rows;
+    out[1] = p.stacked;
+    out[2] = p.n_stages;
+    out[3] = p.sf_item;
+    out[4] = grid;
+    out[5] = smem;
+    out[6] = p.sf_item ? gemm_tmem_cols_item(p.nb_rows, p.stacked, n_st) : gemm_tmem_cols(p.nb_rows, p.stacked, p.n_stages);
+    out[7] = p.K_main / GEMM_KS;
+    out[8] = n_st;
+    out[9] = p.MB;
+    return MOE_OK;
+}
+
 }  // extern "C"

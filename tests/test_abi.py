@@ -65,3 +65,43 @@ def test_stage_calls_reject_null_context(lib):
     assert lib.moe_group(None, 4, 4, None) == moe.MOE_ERR_ARG
     assert lib.moe_expert_up(None, 4, 4, None, None, None, None) == moe.MOE_ERR_ARG
     assert lib.moe_copy_workspace(None, 0, None, 0, None) == moe.MOE_ERR_ARG
+
+
+# (T, d, F, E, k) of the benchmark workloads; decode-sized batches use stacked
+# 16-row token blocks with per-item scale factors, the others 192-row blocks
+PLAN_CASES = {
+    "tiny": (16, 128, 128, 8, 4, "decode"),
+    "decode20b": (32, 2880, 2880, 32, 4, "decode"),
+    "decode120b": (64, 2880, 2880, 128, 4, "decode"),
+    "prefill20b": (8192, 2880, 2880, 32, 4, "large"),
+    "stack20b": (2048, 2880, 2880, 32, 4, "large"),
+    "single token": (1, 2880, 2880, 32, 4, "decode"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLAN_CASES))
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemm_launch_plan_fits_the_sm(lib, name, mode):
+    """The host planner's choices, without a GPU: within 227 KB of shared memory and 512 TMEM columns,
+    a persistent grid of at most one CTA per SM, the K stages and weight-row blocks of the shape."""
+    T, d, F, E, k, kind = PLAN_CASES[name]
+    pl = moe.moe_debug_plan(mode, T, k, d, F, E, T * k, 148)
+    K = d if mode == 0 else F
+    assert pl["smem"] <= 227 * 1024 and pl["tmem_cols"] <= 512
+    assert 2 <= pl["n_stages"] <= 12 and 1 <= pl["grid"] <= 148
+    assert pl["k_stages"] == -(-K // 128) and pl["k_full_stages"] == K // 128
+    assert pl["row_blocks"] == (F // 64 if mode == 0 else -(-d // 128))
+    if kind == "decode":
+        assert (pl["nb_rows"], pl["stacked"], pl["sf_item"]) == (16, 1, 1)
+    else:
+        assert (pl["nb_rows"], pl["stacked"], pl["sf_item"]) == (192, 0, 0)
+        assert pl["n_stages"] == 3            # 16 KB of codes + 48 KB of two-term tokens per stage
+
+
+def test_gemm_launch_plan_rejects_bad_arguments(lib):
+    out = (ctypes.c_int * 10)()
+    assert lib.moe_debug_plan(2, 32, 4, 2880, 2880, 32, 128, 148, out) == moe.MOE_ERR_ARG     # mode
+    assert lib.moe_debug_plan(0, 32, 4, 2880, 2880, 32, 127, 148, out) == moe.MOE_ERR_ARG     # P_max < T k
+    assert lib.moe_debug_plan(0, 32, 4, 100, 2880, 32, 128, 148, out) == moe.MOE_ERR_ARG      # d
+    assert lib.moe_debug_plan(0, 32, 9, 2880, 2880, 32, 288, 148, out) == moe.MOE_ERR_ARG     # top_k
+    assert lib.moe_debug_plan(0, 32, 4, 2880, 2880, 32, 128, 148, None) == moe.MOE_ERR_ARG
