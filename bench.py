@@ -177,13 +177,27 @@ class ClockSampler:
                 "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
-def workload_config(name: str, T: int):
+def workload_config(name: str, world: int = 1):
+    """The static description of a workload: identical for both arms of the bench."""
     cfg = CONFIGS[name]
-    c = {"workload": DESCRIPTIONS[name], "name": name, "T": T, "d_model": cfg.d, "d_ff": cfg.F, "experts": cfg.E,
-         "top_k": cfg.k, "layers": cfg.layers, "seed": cfg.seed, "weights": "MXFP4 (E2M1 codes + E8M0 per 32)",
-         "mma": "tcgen05 kind::mxf8f6f4 block-scaled: E2M1 weight codes (E8M0 per 32) straight from TMA x "
-                "activations as two E4M3 terms (E8M0 per 32) -> fp32 in TMEM"}
-    return c
+    w_expert = 2 * cfg.F * (cfg.d // 2 + cfg.d // 32 + 2) + cfg.d * (cfg.F // 2 + cfg.F // 32 + 2)
+    return {"workload": DESCRIPTIONS[name], "name": name, "T": cfg.T, "d_model": cfg.d, "d_ff": cfg.F,
+            "experts": cfg.E, "top_k": cfg.k, "layers": cfg.layers, "seed": cfg.seed,
+            "weights": "MXFP4 (E2M1 codes + E8M0 per 32)",
+            "mma": "tcgen05 kind::mxf8f6f4 block-scaled: E2M1 weight codes (E8M0 per 32) straight from TMA x "
+                   "activations as E4M3 terms (E8M0 per 32) -> fp32 in TMEM",
+            "parallelism": "replicas (dp%d, no collective)" % world, "global_batch": cfg.T * world,
+            "l2": "inputs larger than L2: a layer step streams the touched experts' MXFP4 weights (up to %.0f MB "
+                  "per layer) vs a %d MB L2; no flush" % (cfg.E * w_expert / 1e6, L2_BYTES // 2 ** 20)}
+
+
+def layer_inputs_of(cfg, layer: int, x=None):
+    """One layer's inputs (a stack's layer l takes the stack's tokens)."""
+    if cfg.layers == 1:
+        return make_config_inputs(cfg)
+    inp = make_config_inputs(cfg, layer)
+    inp["x"] = x if x is not None else make_tokens(np.random.Generator(np.random.PCG64(cfg.seed)), cfg.T, cfg.d)
+    return inp
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -198,31 +212,54 @@ def oracle_tokens_per_s(inp, cfg, n_tokens: int, threads: int):
     return n_tokens / dt, dt
 
 
+# tokens of a workload one reference (oracle) step processes: the whole batch of
+# the decode workloads, a 64-token sample of the larger ones, always through one layer
+REFERENCE_TOKENS_MAX = 64
+# single-thread oracle runs reported beside the reference line: (workload, tokens)
+SINGLE_THREAD_RUNS = (("tiny", 16), ("decode20b", 4), ("decode120b", 4))
+
+
+def single_thread_baselines():
+    out = []
+    for name, n in SINGLE_THREAD_RUNS:
+        cfg = CONFIGS[name]
+        inp = layer_inputs_of(cfg, 0)
+        tps, dt = oracle_tokens_per_s(inp, cfg, n, 1)
+        out.append({"workload": name, "value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                    "sample": "%d of the workload's %d tokens through one layer (%.1f s)" % (n, cfg.T, dt)})
+    return out
+
+
 def run_reference(args, rank, world):
-    """Reference arm: the CPU oracle, timed on the host cores (rank 0 only)."""
+    """Reference arm: the CPU oracle, timed on the host cores (rank 0 only).
+
+    Each step runs min(T, 64) of the workload's tokens through one layer (all of
+    a decode batch); ms_per_step is the time of exactly that work, and the
+    value is tokens per second per layer (divided by the layer count for a
+    stack)."""
     if rank != 0:
         return 0
     import oracle
     cfg = CONFIGS[args.workload]
-    inp = make_config_inputs(cfg) if cfg.layers == 1 else dict(make_config_inputs(cfg, 0), x=make_tokens(
-        np.random.Generator(np.random.PCG64(cfg.seed)), cfg.T, cfg.d))
+    inp = layer_inputs_of(cfg, 0)
     threads = oracle.max_threads()
-    n = min(cfg.T, max(1, threads))                 # one token per core per step
-    for _ in range(args.warmup if args.warmup <= 1 else 1):
+    n = min(cfg.T, REFERENCE_TOKENS_MAX)
+    for _ in range(min(args.warmup, 1)):
         oracle_tokens_per_s(inp, cfg, min(n, 2), threads)
     total_t = 0.0
     for _ in range(args.steps):
         _, dt = oracle_tokens_per_s(inp, cfg, n, threads)
         total_t += dt
-    # a step of the workload is T tokens; the reference processes n per timed step
-    per_token = total_t / (args.steps * n)
-    value = 1.0 / per_token / max(cfg.layers, 1)
+    value = args.steps * n / total_t / cfg.layers
+    sample = "%d of the workload's %d tokens through %s per step" % (
+        n, cfg.T, "the layer" if cfg.layers == 1 else "layer 0 (value divided by %d layers)" % cfg.layers)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * cfg.T * cfg.layers * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(args.workload, cfg.T),
+            "data": "synthetic", "config": workload_config(args.workload, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": "%d of the workload's %d tokens per step (layer 0)" % (n, cfg.T)},
+                             "sample": sample},
+            "cpu_baseline_single_thread": single_thread_baselines() if not args.no_cpu_baseline else None,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -259,7 +296,9 @@ def algorithmic_counts(cfg, counts):
 
     Bytes: the touched experts' codes + scales + biases, router weights and
     bias, RMSNorm scale, x read and y written (bf16).  FLOPs: 2*T*d*E for the
-    router plus 2*(2F*d + d*F) per routed (token, expert) pair.
+    router plus 2*(2F*d + d*F) per routed (token, expert) pair.  Per GEMM: its
+    touched experts' weights, its activation rows in (bf16-sized: 2 bytes per
+    element) and its output rows (h at 2 bytes, the weighted rows at 4).
     """
     T, d, F, E, k = cfg.T, cfg.d, cfg.F, cfg.E, cfg.k
     touched = int(np.count_nonzero(counts))
@@ -277,36 +316,55 @@ def algorithmic_counts(cfg, counts):
                 w13_expert=w13_expert, w2_expert=w2_expert)
 
 
-def run_ours(args, rank, world, local_rank):
+def gemm_roofline(which, t_s, cnt, tensor_bound, peaks, peak_key, workload):
+    """Roofline of one grouped GEMM launch from its live event time t_s (seconds)."""
+    key = "expert_%s_%s" % (which, workload)
+    if tensor_bound:
+        flops = cnt["flops_" + which]
+        achieved = flops / t_s / 1e12
+        peak = peaks[peak_key]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": committed_traffic(key), "kernel": "expert_gemm_kernel<%s>" % which,
+                "algorithmic_flops_per_launch": flops,
+                "peak_source": "%s bf16 dense%s (the roofline the block is specified against)" % (
+                    peaks["source"], ", sustained" if peak_key.endswith("sustained") else ", burst")}
+    byts = cnt["bytes_" + which]
+    achieved = byts / t_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(key),
+            "kernel": "expert_gemm_kernel<%s>" % which, "algorithmic_bytes_per_launch": byts,
+            "peak_source": peaks["source"] + " HBM copy"}
+
+
+def measure_workload(name, args, rank, world, local_rank, main):
+    """Time one workload: K steps of moe_forward (the value), then K steps of the five stage calls
+    with the two GEMMs bracketed by events, per-stage times, and (main line only) the end-to-end
+    number and the CPU oracle sample.  Returns the measurements (rank 0) or None."""
     import torch
-    import torch.distributed as dist
     import sparse_moe_rmsnorm_b200 as moe
 
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = CONFIGS[args.workload]
-    T = cfg.T
-    layers = cfg.layers
-    # the weights (identical on every rank) and this rank's token batch
-    if layers == 1:
-        inp = make_config_inputs(cfg)
-        layer_inputs = [inp]
-    else:
-        layer_inputs = [make_config_inputs(cfg, l) for l in range(layers)]
+    cfg = CONFIGS[name]
+    T, layers = cfg.T, cfg.layers
     x_np = replica_tokens(cfg, rank)
-    weights = [moe.MoEWeights.from_numpy(li, device=dev) for li in layer_inputs]
+    # the weights (identical on every rank), made and uploaded one layer at a time
+    weights = []
+    first_inputs = None
+    for l in range(layers):
+        li = layer_inputs_of(cfg, l, x=x_np)
+        if l == 0:
+            first_inputs = li
+        weights.append(moe.MoEWeights.from_numpy(li, device=dev))
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     m = moe.MoE(T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps)
     bufs = [torch.empty_like(x) for _ in range(2)]
     stream = torch.cuda.current_stream()
-
-    # events around the gate/up GEMM (the dominant kernel) of every layer of every timed step
-    up_events = []
+    gemm_events = {"up": [], "down": []}
 
     def step(timed=False):
         """One step: the block on every layer.  timed=False: moe_forward (the public call);
-        timed=True: the five stage calls moe_forward is made of, with the gate/up GEMM
-        bracketed by events on the launching stream."""
+        timed=True: the five stage calls moe_forward is made of, with the two GEMMs bracketed
+        by events on the launching stream."""
         cur = x
         for l, w in enumerate(weights):
             out = bufs[l % 2]
@@ -316,14 +374,14 @@ def run_ours(args, rank, world, local_rank):
                 continue
             moe.moe_route(m.ctx, T, cur, w.norm_scale, w.router_w, w.router_b, cfg.k)
             moe.moe_group(m.ctx, T, cfg.k)
-            if timed:
-                ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                ea.record(stream)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(stream)
             moe.moe_expert_up(m.ctx, T, cfg.k, w.w13_codes, w.w13_scales, w.b13)
-            if timed:
-                eb.record(stream)
-                up_events.append((ea, eb))
+            ev[1].record(stream)
             moe.moe_expert_down(m.ctx, T, cfg.k, w.w2_codes, w.w2_scales, w.b2)
+            ev[2].record(stream)
+            gemm_events["up"].append((ev[0], ev[1]))
+            gemm_events["down"].append((ev[1], ev[2]))
             moe.moe_finalize(m.ctx, T, cfg.k, cur, out)
             cur = out
         return cur
@@ -332,10 +390,11 @@ def run_ours(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     if m.sync_status() != moe.MOE_OK:
-        raise RuntimeError("device-side error during warm-up")
+        raise RuntimeError("device-side error during warm-up (%s)" % name)
 
     # ---- timed region: K steps, device events, barrier + sync on both sides
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -348,15 +407,15 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    # ---- the dominant kernel: K more steps, its launches bracketed by events
+    # ---- the GEMMs: K more steps, their launches bracketed by events
     for _ in range(args.steps):
         step(timed=True)
     torch.cuda.synchronize()
-    up_ms_live = sum(a.elapsed_time(b) for a, b in up_events) / max(len(up_events), 1)
+    gemm_ms = {k_: sum(a.elapsed_time(b) for a, b in v) / max(len(v), 1) for k_, v in gemm_events.items()}
     ms_per_step = ms_total / args.steps
     value = job_tokens_per_s(ms_total, T, args.steps, world)
     if m.sync_status() != moe.MOE_OK:
-        raise RuntimeError("device-side error during the timed region")
+        raise RuntimeError("device-side error during the timed region (%s)" % name)
 
     # ---- per-stage times (layer 0) in a separate pass, for the report: events between
     # every kernel, so each stage is timed alone
@@ -384,93 +443,103 @@ def run_ours(args, rank, world, local_rank):
     cnt = algorithmic_counts(cfg, counts)
 
     # ---- end to end through the public API: pinned host x in, y out, every step
-    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(max(1, args.warmup)):
-        m.forward_host(x_host, w0, y_host, x_dev, bufs[0])
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        if layers == 1:
+    e2e = None
+    if main:
+        x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+        y_host = torch.empty_like(x_host).pin_memory()
+        x_dev = torch.empty_like(x)
+        for _ in range(max(1, args.warmup)):
             m.forward_host(x_host, w0, y_host, x_dev, bufs[0])
-        else:
-            x_dev.copy_(x_host, non_blocking=True)
-            cur = x_dev
-            for l, w in enumerate(weights):
-                out = bufs[l % 2]
-                m.forward(cur, w, y=out)
-                cur = out
-            y_host.copy_(cur, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = job_tokens_per_s(e2e_ms, T, args.steps, world)
-
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            if layers == 1:
+                m.forward_host(x_host, w0, y_host, x_dev, bufs[0])
+            else:
+                x_dev.copy_(x_host, non_blocking=True)
+                cur = x_dev
+                for l, w in enumerate(weights):
+                    out = bufs[l % 2]
+                    m.forward(cur, w, y=out)
+                    cur = out
+                y_host.copy_(cur, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_tokens_per_s(e2e_ms, T, args.steps, world), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2}
+    m.close()
+    del weights
+    torch.cuda.empty_cache()
     if rank != 0:
-        m.close()
-        return 0
+        return None
 
     peaks = measured_peaks()
-    # dominant kernel and its roofline
-    # the dominant kernel: the gate/up GEMM (2/3 of the weights and of the flops), timed live
-    dom = "up"
-    t_dom = up_ms_live / 1e3
     tensor_bound = cfg.T * cfg.k >= 4096
-    key = "expert_%s_%s" % (dom, args.workload)
-    if tensor_bound:
-        flops = cnt["flops_" + dom]
-        achieved = flops / t_dom / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": committed_traffic(key),
-                "kernel": "expert_gemm_kernel<%s>" % dom, "algorithmic_flops_per_launch": flops,
-                "peak_source": peaks["source"] + " bf16 dense (the roofline the block is specified against; the "
-                               "fp8-kind MMAs run two activation terms per product, the same tensor time as bf16)"}
-    else:
-        byts = cnt["bytes_" + dom]
-        achieved = byts / t_dom / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(key),
-                "kernel": "expert_gemm_kernel<%s>" % dom, "algorithmic_bytes_per_launch": byts,
-                "peak_source": peaks["source"] + " HBM copy"}
-    t_layer_roof = max(cnt["layer_flops"] / (peaks["bf16_tflops"] * 1e12), cnt["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    # a stack runs for seconds at the power cap: its tensor-bound kernels take the sustained peak
+    peak_key = "bf16_tflops_sustained" if layers > 1 else "bf16_tflops"
+    roof_up = gemm_roofline("up", gemm_ms["up"] / 1e3, cnt, tensor_bound, peaks, peak_key, name)
+    roof_down = gemm_roofline("down", gemm_ms["down"] / 1e3, cnt, tensor_bound, peaks, peak_key, name)
+    tflops_layer = peaks[peak_key] if tensor_bound else peaks["bf16_tflops"]
+    t_layer_roof = max(cnt["layer_flops"] / (tflops_layer * 1e12), cnt["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
     layer_ms = ms_per_step / layers
 
-    # CPU oracle baseline on a bounded sample (rank 0, N = 1 only)
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if main and world == 1 and not args.no_cpu_baseline:
         import oracle
         threads = oracle.max_threads()
-        n = min(T, max(1, threads))
-        tps, dt = oracle_tokens_per_s(layer_inputs[0] if layers == 1 else dict(layer_inputs[0], x=x_np), cfg, n,
-                                      threads)
+        n = min(T, REFERENCE_TOKENS_MAX)
+        tps, dt = oracle_tokens_per_s(first_inputs, cfg, n, threads)
         cpu = {"value": tps / layers, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": "%d tokens of the workload through %s (%.1f s)" % (
-                   n, "the layer" if layers == 1 else "layer 0 (value divided by %d layers)" % layers, dt)}
+               "sample": "%d of the workload's %d tokens through %s (%.1f s)" % (
+                   n, T, "the layer" if layers == 1 else "layer 0 (value divided by %d layers)" % layers, dt)}
+    return {"value": value, "ms_per_step": ms_per_step, "roofline": roof_up, "roofline_down": roof_down,
+            "layer_roofline": {"t_roof_us": t_layer_roof * 1e6, "t_us": layer_ms * 1e3,
+                               "frac": t_layer_roof / (layer_ms / 1e3), "bytes": cnt["layer_bytes"],
+                               "flops": cnt["layer_flops"]},
+            "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+            "gemm_ms_live": {k_: round(v, 4) for k_, v in gemm_ms.items()},
+            "experts_touched": cnt["touched"], "clocks": clocks.summary(), "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": KERNELS_PER_LAYER * layers * args.steps}
 
-    config = workload_config(args.workload, T)
-    config.update({"parallelism": "replicas (dp%d, no collective)" % world, "global_batch": T * world,
-                   "l2": "inputs larger than L2: %.0f MB of touched expert weights per layer step vs %d MB L2" % (
-                       (cnt["touched"] * (cnt["w13_expert"] + cnt["w2_expert"])) / 1e6, L2_BYTES // 2 ** 20),
-                   "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
-                   "up_ms_live": round(up_ms_live, 4),
-                   "experts_touched": cnt["touched"],
-                   "layer_roofline": {"t_roof_us": t_layer_roof * 1e6, "t_us": layer_ms * 1e3,
-                                      "frac": t_layer_roof / (layer_ms / 1e3),
-                                      "bytes": cnt["layer_bytes"], "flops": cnt["layer_flops"]},
-                   "kernel_src_sha": kernel_source_hash()})
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e2m1xe4m3->f32", "data": "synthetic", "config": config,
-            "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.d * 2,
-                    "d2h_bytes_per_step": T * cfg.d * 2},
-            "gpu_launches": KERNELS_PER_LAYER * layers * args.steps, "clocks": clocks.summary()}
+
+EXTRA_WORKLOADS = ("prefill20b", "decode120b", "stack20b")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    main = measure_workload(args.workload, args, rank, world, local_rank, main=True)
+    # the other full-size workloads, one GPU only: each with its own timed region and clocks
+    extra = {}
+    if world == 1 and not args.single and args.workload == "decode20b":
+        for name in EXTRA_WORKLOADS:
+            r = measure_workload(name, args, rank, world, local_rank, main=False)
+            extra[name] = {"config": workload_config(name, world), "value": r["value"], "unit": "tokens/s",
+                           "ms_per_step": r["ms_per_step"], "roofline": r["roofline"],
+                           "roofline_down": r["roofline_down"], "layer_roofline": r["layer_roofline"],
+                           "stage_ms": r["stage_ms"], "gemm_ms_live": r["gemm_ms_live"],
+                           "experts_touched": r["experts_touched"], "clocks": r["clocks"],
+                           "gpu_launches": r["gpu_launches"]}
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e2m1xe4m3->f32", "data": "synthetic",
+            "config": workload_config(args.workload, world), "roofline": main["roofline"],
+            "cpu_baseline": main["cpu_baseline"], "e2e": main["e2e"], "gpu_launches": main["gpu_launches"],
+            "clocks": main["clocks"],
+            "detail": {"roofline_down": main["roofline_down"], "layer_roofline": main["layer_roofline"],
+                       "stage_ms": main["stage_ms"], "gemm_ms_live": main["gemm_ms_live"],
+                       "experts_touched": main["experts_touched"], "kernel_src_sha": kernel_source_hash()}}
+    if extra:
+        line["workloads"] = extra
     print(json.dumps(line), flush=True)
-    m.close()
     return 0
 
 
@@ -482,6 +551,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode20b", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", action="store_true", help="time only --workload (no workloads object)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)

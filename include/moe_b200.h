@@ -201,11 +201,10 @@ MOE_API int moe_debug_plan(int mode, int T, int top_k, int d_model, int d_ff, in
                            int *out);
 
 /* The whole block (as moe_forward) without any device allocation, for callers
- * that cannot call cudaMalloc: code running inside a CUDA graph capture that
- * forbids allocation, frameworks whose allocator owns all device memory, or
- * plugins whose host does not let library code allocate.  (The gpt-oss
- * write-ups have no counterpart of this entry point; it is an integration
- * convenience.)
+ * that cannot call cudaMalloc: frameworks whose caching allocator owns all
+ * device memory, or plugins whose host does not let library code allocate.
+ * (The gpt-oss write-ups have no counterpart of this entry point; it is an
+ * integration convenience.)
  *
  * Scratch memory comes from one fixed 8 MiB __device__ array inside the
  * library, held on every GPU that loads it until process exit; no context is

@@ -1,9 +1,8 @@
 // moe_forward_noalloc: the whole MoE block without any device allocation.
 //
-// Some callers cannot call cudaMalloc at all: code that runs while a CUDA
-// graph is being captured in relaxed/global mode, custom allocators that own
-// every byte of device memory, or plugins loaded into a host that forbids
-// allocation from library code.  For them this entry point takes its scratch
+// Some callers cannot call cudaMalloc at all: frameworks whose custom
+// allocator owns every byte of device memory, or plugins loaded into a host
+// that forbids allocation from library code.  For them this entry point takes its scratch
 // memory from one file-scope __device__ array of fixed size (every GPU that
 // loads the library holds it until process exit).  The caller still passes
 // every input, the weights and the output.

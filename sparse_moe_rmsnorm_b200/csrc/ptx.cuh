@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
-// (tiled, gather4, untiled bulk), and tcgen05 (TMEM alloc, MMA, ld/st, fences).
+// (tiled and untiled bulk loads), and tcgen05 (TMEM alloc, MMA, ld/st, fences).
 #pragma once
 
 #include <cstdint>
@@ -39,13 +39,6 @@ __device__ __forceinline__ void fence_barrier_init() {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
-                     smem_addr(bar)),
-                 "r"(bytes)
                  : "memory");
 }
 
@@ -107,43 +100,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const void *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const void *map, uint64_t *bar, int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void *dst, const void *map, uint64_t *bar, int c0, int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-        "%5}], [%2];" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// Four rows (r0..r3) of box width starting at column c0 of a 2-D tensor map
-// whose box is one row high; they land as four consecutive box rows.
-__device__ __forceinline__ void tma_gather4(void *dst, const void *map, uint64_t *bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-        "%4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
-// Untiled bulk copy global -> shared (16-byte aligned addresses, size a
-// multiple of 16).
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-
 // ----------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
@@ -166,24 +122,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]^T ; kind::f16, one CTA.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, "
-        "p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05 async operation this thread issued
-// so far has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_addr(bar))
-                 : "memory");
 }
 
 // ------------------------------------------------------------ E4M3 / E8M0
@@ -230,15 +168,6 @@ __device__ __forceinline__ void e4m3x2_to_f32x2(uint32_t v, float &lo, float &hi
 // lone lane of a divergent warp holds it for 50-120 cycles, so the MMA and
 // TMA producer roles run as whole warps through these forms.
 
-__device__ __forceinline__ void mma_f16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void mma_commit_w(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
@@ -267,15 +196,6 @@ __device__ __forceinline__ void tma_load_3d_w(void *dst, const void *map, uint64
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
         "%5}], [%2];\n\t}" ::"r"(smem_addr(dst)),
         "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d_w(void *dst, const void *map, uint64_t *bar, int c0, int c1) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];\n\t}" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
 
@@ -326,10 +246,6 @@ __device__ __forceinline__ void bulk_load_w(void *dst, const void *src, uint32_t
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Each thread of the warp writes 1 / 4 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
                  "r"(r[2]), "r"(r[3])
@@ -374,19 +290,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Each thread of the warp writes 32 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
-        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
-        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
 // Each thread of the warp reads 16 consecutive 32-bit columns of its lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -409,15 +312,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     d |= (uint64_t)1 << 46;                           // descriptor version for tcgen05
     d |= (uint64_t)2 << 61;                           // 128-byte swizzle
     return d;
-}
-
-// Instruction descriptor, kind::f16: A and B fp16, D fp32, both K-major.
-__host__ __device__ __forceinline__ uint32_t idesc_f16_f32(uint32_t M, uint32_t N) {
-    return (1u << 4)                 // D format: f32
-           | (0u << 7)               // A format: f16
-           | (0u << 10)              // B format: f16
-           | ((N >> 3) << 17)        // N / 8
-           | ((M >> 4) << 24);       // M / 16
 }
 
 // ------------------------------------------------------------- MXFP4 decode
@@ -451,14 +345,6 @@ __device__ __forceinline__ float exp2i(int e) {
 // E8M0 byte is within 36 of the row's largest is then exact in fp16.  Bytes
 // of 255 (NaN) are left out of the maximum.
 __device__ __forceinline__ int row_shift_from_max(int smax) { return smax < 0 ? 0 : smax - 140; }
-
-// Fast multiplier for rows whose E8M0 bytes all lie within 27 of the row's
-// largest (and none is 255): 2^(s-127-c) with c = smax - 140 is then a normal
-// fp16 number, bits ((s - smax + 28) << 10), duplicated into both halves.
-__device__ __forceinline__ uint32_t block_multiplier_fast(int s, int smax) {
-    const uint32_t b = (uint32_t)(s - smax + 28) << 10;
-    return b | (b << 16);
-}
 
 // Multiplier of one block (E8M0 byte s) under row shift c, as an fp16 pair:
 // 2^(s-127-c), rounded to fp16 (exact down to 2^-24), NaN for s = 255.

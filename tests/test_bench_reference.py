@@ -19,6 +19,8 @@ import bench  # noqa: E402
 def _run(capsys, monkeypatch, rank, world):
     monkeypatch.setenv("RANK", str(rank))
     monkeypatch.setenv("WORLD_SIZE", str(world))
+    # the single-thread oracle runs are covered on their own below
+    monkeypatch.setattr(bench, "SINGLE_THREAD_RUNS", (("tiny", 2),))
     rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1",
                      "--gpus", str(world)])
     return rc, capsys.readouterr().out
@@ -34,9 +36,13 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     assert d["metric"] == bench.METRIC and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"] == bench.workload_config("tiny", 16)
+    assert d["config"] == bench.workload_config("tiny", 1)
+    # ms_per_step is the time of the work one step does: all 16 tokens of the tiny batch through its layer
+    assert abs(d["value"] - 16 / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    st = d["cpu_baseline_single_thread"]
+    assert [r["workload"] for r in st] == ["tiny"] and st[0]["cores"] == 1 and st[0]["value"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 

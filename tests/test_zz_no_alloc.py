@@ -1,20 +1,21 @@
-"""The allocation-free entry point against the regular one.
+"""The allocation-free entry point against the regular one and against the oracle.
 
-Some callers cannot allocate device memory (a CUDA graph being captured in a
-mode that forbids allocation, a framework whose allocator owns all device
-memory, a plugin host that forbids it).  moe_forward_noalloc serves them from a
-fixed scratch array inside the library.  This file is collected last so that a
-run stopping at its first failure has run every other test already; it passes
-alone in a fresh process and after the other tests.
+Some callers cannot allocate device memory: a framework whose caching
+allocator owns all of it, or a plugin host that does not let library code call
+cudaMalloc.  moe_forward_noalloc serves them from a fixed scratch array inside
+the library.  This file is collected last so that a run stopping at its first
+failure has run every other test already; it passes alone in a fresh process
+and after the other tests.
 """
 import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")
 
+import oracle
 import sparse_moe_rmsnorm_b200 as moe
 from moe_inputs import CONFIGS, custom_layer, make_config_inputs
-from _parity import MAX_REL, MEAN_REL
+from _parity import MAX_REL, MEAN_REL, excluded_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -23,30 +24,54 @@ def _bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def _close(a, b):
-    a = a.float().cpu().numpy().astype(np.float64)
-    b = b.float().cpu().numpy().astype(np.float64)
-    diff = np.abs(a - b)
-    return diff.max() <= MAX_REL * np.abs(b).max() and diff.sum() <= MEAN_REL * np.abs(b).sum()
+def _noalloc(cfg, x, w):
+    y = torch.full_like(x, float("nan"))
+    moe.moe_forward_noalloc(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps, x, w.router_w, w.router_b, w.w13_codes,
+                            w.w13_scales, w.b13, w.w2_codes, w.w2_scales, w.b2, w.norm_scale, y)
+    torch.cuda.synchronize()
+    return y
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode20b"])
-def test_noalloc_matches_regular_entry_point_twice(name):
-    cfg = CONFIGS[name]
+def test_noalloc_equals_regular_entry_point_bitwise():
+    """Both paths run the same kernels on the same launch plan (P_max = T * k) and combine in a fixed
+    order, so their outputs agree bit for bit.  The calls go large, small, large: a stale count,
+    offset or tile left in the shared scratch by a larger call would show."""
+    cases = {}
+    for name in ("decode20b", "tiny"):
+        cfg = CONFIGS[name]
+        inp = make_config_inputs(cfg)
+        w = moe.MoEWeights.from_numpy(inp)
+        x = _bf16(inp["x"])
+        ctx = moe.MoE(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps)
+        y_ref = ctx.forward(x, w)
+        torch.cuda.synchronize()
+        assert ctx.sync_status() == moe.MOE_OK
+        ctx.close()
+        cases[name] = (cfg, x, w, y_ref)
+    for name in ("decode20b", "tiny", "decode20b", "decode20b"):
+        cfg, x, w, y_ref = cases[name]
+        y = _noalloc(cfg, x, w)
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), name
+
+
+def test_noalloc_largest_shape_against_oracle():
+    """Its documented maximum: 64 tokens of the 128-expert layer (d_model = d_ff = 2880, top-4),
+    against the CPU oracle within the block's stated tolerances (tokens whose 4th/5th router
+    logits are closer than 1e-4 are left out and counted)."""
+    cfg = CONFIGS["decode120b"]
+    assert cfg.T == moe.MOE_NOALLOC_MAX_TOKENS
     inp = make_config_inputs(cfg)
     w = moe.MoEWeights.from_numpy(inp)
     x = _bf16(inp["x"])
-    ctx = moe.MoE(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps)
-    y_ref = ctx.forward(x, w)
-    torch.cuda.synchronize()
-    assert ctx.sync_status() == moe.MOE_OK
-    ctx.close()
-    for _ in range(2):
-        y = torch.full_like(x, float("nan"))
-        moe.moe_forward_noalloc(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k, cfg.eps, x, w.router_w, w.router_b,
-                                w.w13_codes, w.w13_scales, w.b13, w.w2_codes, w.w2_scales, w.b2, w.norm_scale, y)
-        torch.cuda.synchronize()
-        assert _close(y, y_ref)
+    y = _noalloc(cfg, x, w).float().cpu().numpy().astype(np.float64)
+    ref = oracle.moe_forward(inp, cfg.k, cfg.eps)
+    keep = ~excluded_tokens(ref["logits"], cfg.k)
+    assert keep.sum() >= cfg.T - 2
+    diff = np.abs(y[keep] - ref["y"][keep])
+    max_rel = diff.max() / np.abs(ref["y"][keep]).max()
+    mean_rel = diff.sum() / np.abs(ref["y"][keep]).sum()
+    print("noalloc decode120b: max_rel %.3g mean_rel %.3g, %d excluded" % (max_rel, mean_rel, (~keep).sum()))
+    assert max_rel <= MAX_REL and mean_rel <= MEAN_REL
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
