@@ -85,7 +85,7 @@ typedef struct moe_ctx moe_ctx_t;
 /* Create a context for `shape` on the current CUDA device.  Allocates the
  * device workspace sized for shape->T_max (routing arrays, the fp16 normalised
  * activations, the expert-sorted activations and the SwiGLU output h in the
- * two-term E4M3 form the block-scaled expert GEMMs read, and the fp32
+ * E4M3 terms the block-scaled expert GEMMs read, and the fp32
  * weighted expert rows [T_max*k, d]).  The context owns the workspace; free it with
  * moe_destroy.  Returns MOE_ERR_ARG for an invalid shape, MOE_ERR_UNSUPPORTED
  * off B200, MOE_ERR_NOMEM when the workspace does not fit. */
@@ -147,16 +147,18 @@ enum {
     MOE_WS_OFFSETS = 5,  /* int32 [E+1]   exclusive prefix of counts              */
     MOE_WS_ROW_TOKEN = 6,/* int32 [T*k]   token of each expert-sorted row         */
     MOE_WS_ROW_W = 7,    /* fp32 [T*k]    routing weight of each expert-sorted row */
-    MOE_WS_H = 8,        /* u8 [2, T_max*k, Kf] SwiGLU output h of the expert-sorted rows as
-                            E4M3 hi (plane 0) and lo (plane 1) terms: h ~ hi 2^s + lo 2^(s-4) with
-                            s the block's scale in MOE_WS_HSF; Kf = d_ff rounded up to 128      */
+    MOE_WS_H = 8,        /* u8 [3, T_max*k, Kf] SwiGLU output h of the expert-sorted rows as
+                            E4M3 hi, lo and lo2 terms (planes 0, 1, 2): h ~ hi 2^s + lo 2^(s-4)
+                            + lo2 2^s with s the block's scale in MOE_WS_HSF; Kf = d_ff rounded
+                            up to 128                                                          */
     MOE_WS_OUT_ROWS = 9, /* fp32 [T*k, d] w * (W2 h + b2), expert-sorted rows      */
     MOE_WS_TILES = 10,   /* int32 [E+1]   exclusive prefix of token blocks        */
     MOE_WS_PAIR_ROW = 11,/* int32 [T*k]   expert-sorted row of pair (token, slot) */
-    MOE_WS_XPERM = 12,   /* u8 [2, T_max*k, Kd] normalised tokens in expert-sorted order, E4M3
-                            hi and lo planes as MOE_WS_H; Kd = d_model rounded up to 128      */
+    MOE_WS_XPERM = 12,   /* u8 [3, T_max*k, Kd] normalised tokens in expert-sorted order, E4M3
+                            hi, lo and lo2 planes as MOE_WS_H; Kd = d_model rounded up to 128 */
     MOE_WS_XSF = 13,     /* u32 [Kd/128, 2, T_max*k] E8M0 scales of MOE_WS_XPERM: word (g, plane,
-                            row), byte i = the scale of 32-block 4g+i                          */
+                            row), byte i = the scale of 32-block 4g+i; plane 0 scales the hi and
+                            the lo2 terms, plane 1 the lo term                                 */
     MOE_WS_HSF = 14      /* u32 [Kf/128, 2, T_max*k] E8M0 scales of MOE_WS_H, same layout      */
 };
 
@@ -209,8 +211,8 @@ MOE_API int moe_debug_plan(int mode, int T, int top_k, int d_model, int d_ff, in
  * Scratch memory comes from one fixed 8 MiB __device__ array inside the
  * library, held on every GPU that loads it until process exit; no context is
  * needed.  Limits: T <= MOE_NOALLOC_MAX_TOKENS and the workspace for the shape
- * (about T*(2d + 4E) + T*k*(6d + 2F) bytes, e.g. 6.5 MiB for 64 tokens of the
- * d_model = d_ff = 2880, top-4 layers) must fit in the array; larger requests
+ * (about T*(2d + 4E) + T*k*(7d + 3F) bytes, e.g. 7.6 MiB for 64 tokens of the
+ * d_model = d_ff = 2880, top-4, 128-expert layer) must fit in the array; larger requests
  * return MOE_ERR_ARG.  Shape limits otherwise as in moe_init.
  *
  * The first call on a device looks up the array's device address

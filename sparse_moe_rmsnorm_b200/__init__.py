@@ -316,9 +316,9 @@ class MoE:
     def workspace(self, name: str, T: int, top_k: Optional[int] = None, stream=None):
         """A device copy of one workspace buffer for the first T tokens.
 
-        The two-term E4M3 operands (``xperm``, ``h``) and their scale words
-        (``xsf``, ``hsf``) are returned whole, sized by T_max:
-        ``xperm`` u8 [2, T_max*k, Kd], ``xsf`` int32 [Kd/128, 2, T_max*k]
+        The E4M3 operands (``xperm``, ``h``: hi, lo and lo2 planes) and their scale
+        words (``xsf``, ``hsf``: hi's, also lo2's, and lo's) are returned whole, sized
+        by T_max: ``xperm`` u8 [3, T_max*k, Kd], ``xsf`` int32 [Kd/128, 2, T_max*k]
         (Kd = d_model rounded up to 128; ``h`` / ``hsf`` likewise with d_ff)."""
         import torch
         k = self.top_k if top_k is None else int(top_k)
@@ -334,8 +334,8 @@ class MoE:
             "row_token": ((P,), torch.int32), "row_w": ((P,), torch.float32),
             "out_rows": ((P, s.d_model), torch.float32),
             "tiles": ((s.n_experts + 1,), torch.int32), "pair_row": ((P,), torch.int32),
-            "xperm": ((2, P_max, Kd), torch.uint8), "xsf": ((Kd // 128, 2, P_max), torch.int32),
-            "h": ((2, P_max, Kf), torch.uint8), "hsf": ((Kf // 128, 2, P_max), torch.int32),
+            "xperm": ((3, P_max, Kd), torch.uint8), "xsf": ((Kd // 128, 2, P_max), torch.int32),
+            "h": ((3, P_max, Kf), torch.uint8), "hsf": ((Kf // 128, 2, P_max), torch.int32),
         }[name]
         out = torch.empty(spec[0], dtype=spec[1], device="cuda")
         moe_copy_workspace(self.ctx, WS[name], out, out.numel() * out.element_size(), stream)

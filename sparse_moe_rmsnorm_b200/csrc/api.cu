@@ -52,9 +52,9 @@ struct moe_ctx {
     int *row_token;
     float *row_w;
     int *pair_row;
-    uint8_t *xq;            // gate/up B: two E4M3 planes [2][P_max][Kd] of the expert-sorted tokens
-    uint32_t *xsf;          // their E8M0 scales [Kd/128][2][P_max]
-    uint8_t *hq;            // down B: two E4M3 planes [2][P_max][Kf] of h
+    uint8_t *xq;            // gate/up B: three E4M3 planes [3][P_max][Kd] of the expert-sorted tokens
+    uint32_t *xsf;          // their E8M0 scales [Kd/128][2][P_max] (hi/lo2, lo)
+    uint8_t *hq;            // down B: three E4M3 planes [3][P_max][Kf] of h
     uint32_t *hsf;          // [Kf/128][2][P_max]
     float *orows;           // weighted expert output per expert-sorted row
     unsigned int *err;
@@ -88,11 +88,11 @@ Buf ws_buffer(moe_ctx *c, int which) {
         case MOE_WS_OFFSETS: return {c->offsets, (E + 1) * 4};
         case MOE_WS_ROW_TOKEN: return {c->row_token, P * 4};
         case MOE_WS_ROW_W: return {c->row_w, P * 4};
-        case MOE_WS_H: return {c->hq, 2 * P * c->Kf};
+        case MOE_WS_H: return {c->hq, 3 * P * c->Kf};
         case MOE_WS_OUT_ROWS: return {c->orows, P * s.d_model * 4};
         case MOE_WS_TILES: return {c->tiles, (E + 1) * 4};
         case MOE_WS_PAIR_ROW: return {c->pair_row, P * 4};
-        case MOE_WS_XPERM: return {c->xq, 2 * P * c->Kd};
+        case MOE_WS_XPERM: return {c->xq, 3 * P * c->Kd};
         case MOE_WS_XSF: return {c->xsf, (size_t)(c->Kd / 128) * 2 * P * 4};
         case MOE_WS_HSF: return {c->hsf, (size_t)(c->Kf / 128) * 2 * P * 4};
         default: return {nullptr, 0};
@@ -125,7 +125,8 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
             c->w13_ptr = codes;
         }
         if (!c->have_xq[bi]) {
-            if (!encode_bq(&c->map_xq[bi], c->xq, P_max, c->Kd, p.nb_rows)) return MOE_ERR_CUDA;
+            if (!encode_bq(&c->map_xq[bi], c->xq, P_max, c->Kd, p.nb_rows, gemm_b_planes(p.stacked)))
+                return MOE_ERR_CUDA;
             c->have_xq[bi] = true;
         }
         p.map_a = c->map_w13;
@@ -139,7 +140,8 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
             c->w2_ptr = codes;
         }
         if (!c->have_hq[bi]) {
-            if (!encode_bq(&c->map_hq[bi], c->hq, P_max, c->Kf, p.nb_rows)) return MOE_ERR_CUDA;
+            if (!encode_bq(&c->map_hq[bi], c->hq, P_max, c->Kf, p.nb_rows, gemm_b_planes(p.stacked)))
+                return MOE_ERR_CUDA;
             c->have_hq[bi] = true;
         }
         p.map_a = c->map_w2;
@@ -210,8 +212,8 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
     const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
     const size_t sizes[] = {T * s.d_model * 2, T * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
                             P * 4, P * 4, P * 4,
-                            2 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
-                            2 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
+                            3 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
+                            3 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
                             P * s.d_model * 4, 64, T * E * 4, T * 4};
     void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,

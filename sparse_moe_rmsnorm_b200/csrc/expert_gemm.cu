@@ -12,13 +12,17 @@
 //     overview sections 1 and 4).  A K tail of 64 (K = 2880 = 22.5 x 128) is
 //     loaded by the A producer with plain loads at the item's start and written
 //     into its stage's slot in the unpacked layout.
-//   B (activations, N = tokens): two E4M3 terms, hi = e4m3(v / 2^s) and
-//     lo = e4m3((v - hi 2^s) / 2^(s-4)), per 32-element block with E8M0 scale
-//     s chosen so the block maximum fits 448.  hi + lo keeps about 8
-//     significant bits of every element (the precision of bf16).  The hi rows
-//     and lo rows of a token block sit one after the other in the B ring; small
-//     blocks feed both in one MMA (N = 2 x rows, the epilogue adds the halves),
-//     large ones in two MMAs into the same accumulator.
+//   B (activations, N = tokens): E4M3 terms per 32-element block with E8M0
+//     scale s chosen so the block maximum fits 448: hi = e4m3(v / 2^s),
+//     lo = e4m3((v - hi 2^s) / 2^(s-4)) and lo2 = e4m3((v - hi 2^s - lo
+//     2^(s-4)) / 2^s).  hi + lo keep about 8 significant bits of every element
+//     (the precision of bf16), the three terms about 12 (that of the fp16
+//     normalised tokens).  lo2 uses hi's scale byte, so its MMA reads hi's
+//     scale column.  Small (decode-sized) blocks stack a token block's hi, lo
+//     and lo2 rows in one MMA (N = 3 x rows, the epilogue adds the thirds).
+//     Large blocks run one MMA over hi and one over lo per K block into the
+//     same accumulator; a work item whose weights reach the E8M0 byte
+//     LO2_SCALE_MIN then takes a second pass over K with the lo2 rows.
 //   Scale factors: the scale-factor warps write A's and B's E8M0 bytes into
 //     TMEM, one 32-bit column per 32 rows, the byte index being the 32-block
 //     within the stage, replicated in all four lane quarters (the layout the
@@ -29,8 +33,8 @@
 //   ("gpt-oss-20B" hub page, section 3.3).  Each 128-row weight block holds 64
 //   gate rows and their 64 linear rows, interleaved in groups of 16 by the
 //   tensor map, so each pair meets in one warp.  h is written directly as the
-//   down GEMM's two-term B: the block maxima over 32 consecutive h rows are
-//   exchanged between the two warps holding them.
+//   down GEMM's B (three E4M3 planes): the block maxima over 32 consecutive h
+//   rows are exchanged between the two warps holding them.
 // Down epilogue: o = w_token * (D + b2) written to the pair's expert-sorted
 //   row; the combine kernel adds a token's rows to its residual (weighted
 //   combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
@@ -39,6 +43,11 @@
 // B (activations), 1 MMA issue, 2 TMEM allocation and (per-item scale factors)
 // the second MMA warp, 4-7 scale-factor warps (one per TMEM lane quarter),
 // 8-11 and 12-15 two epilogue groups taking 16-column chunks in turn.
+// Large blocks: the A producer decides each work item's pass count (one, or
+// two with the lo2 pass) from the item's weight scale bytes, which it stages
+// in shared memory one item ahead, and publishes it to the B producer, the
+// MMA warp and the scale-factor warps through a shared-memory word and an
+// mbarrier.
 // Producers and MMA run as whole converged warps, one elected lane issuing.
 // Every mbarrier wait is bounded (WaitCtl); when one runs out the CTA stops
 // issuing work, drains its copies and MMAs in flight, frees TMEM and returns
@@ -123,10 +132,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NS = p.n_stages;
     const int NB = p.nb_rows;
-    const GemmSmem plan = gemm_smem_plan(p.K, p.E, NB, NS, SFI ? 1 : 0);
+    const GemmSmem plan = gemm_smem_plan(p.K, p.E, NB, p.stacked, NS, SFI ? 1 : 0);
     uint8_t *a_ring = smem + plan.a_off;
     uint8_t *b_ring = smem + plan.b_off;
-    const int b_stage = gemm_b_stage_bytes(NB);
+    const int b_stage = gemm_b_stage_bytes(NB, p.stacked);
     uint8_t *scale_buf = smem + plan.scale_off;
     const int KB32 = p.K / 32;
     const int scale_bytes = align_up(GEMM_BM * KB32, 128);
@@ -145,9 +154,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *f_empty = f_full + 2;
     uint64_t *bw_full = f_empty + 2;        // the item's B scale words are staged (per-item mode)
     uint64_t *bw_empty = bw_full + 1;       // ... and have been read by all four scale-factor warps
+    uint64_t *info_full = bw_empty + 1;     // [2] the pass count of the item using scale buffer i is published
     uint32_t *bw_s = reinterpret_cast<uint32_t *>(smem + plan.bsf_off);   // [stage][4][32]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
+    volatile int *npass_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 8);   // [2] per scale buffer
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
     int *offsets_s = counts_s + (p.E + 1);
     int *tiles_s = offsets_s + (p.E + 1);
@@ -159,8 +170,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     // MMA warps: two taking alternate stages in per-item mode (the second only
     // when an item has more than one stage), one otherwise
     const int n_mma_warps = SFI && n_st > 1 ? 2 : 1;
+    // accumulator buffers per MMA warp: two (the epilogue drains one while the MMAs
+    // fill the other), one in per-item mode, where the two MMA warps' accumulators
+    // and the two item regions of scale factors fill TMEM
+    constexpr int n_dbuf = SFI ? 1 : 2;
     // TMEM columns: accumulators first, then the scale factors
-    const uint32_t sf_col0 = (uint32_t)((SFI ? 4 : 2) * d_cols);
+    const uint32_t sf_col0 = (uint32_t)(2 * d_cols);
     const int sfi_cols = GEMM_SFI_COLS * n_st;           // one item region (per-item mode)
 
     if (threadIdx.x == 0) {
@@ -171,7 +186,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4);
+            // per-stage mode: the four scale-factor warps, and the B producer and the MMA
+            // warp once they have read the item's pass count
+            mbar_init(&s_empty[i], SFI ? 4 : 6);
+            mbar_init(&info_full[i], 1);
             mbar_init(&d_empty[i], 8);    // every epilogue warp
             mbar_init(&drain_bar[i], 1);
             mbar_init(&f_full[i], 4);     // the four scale-factor warps
@@ -217,15 +235,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // ------------------------------------------------- A producer (weights)
         // Per work item (per-stage mode) the 128 rows' E8M0 bytes (one or two
         // untiled bulk copies), issued one item ahead so the scale-factor warps
-        // can prepare an item while the MMAs work on the one before; per stage one TMA box
-        // of E2M1 codes (128 rows x 128 K).  The K tail (K not a multiple of
-        // 128) is loaded at the start of the item, four rows per lane, and
-        // written into its stage's slot here.
+        // can prepare an item while the MMAs work on the one before; from them the
+        // item's pass count (a lo2 pass when a byte reaches LO2_SCALE_MIN),
+        // published before the item starts.  Per stage one TMA box of E2M1 codes
+        // (128 rows x 128 K), the item's K stages once per pass.  The K tail (K not
+        // a multiple of 128) is loaded at the start of the item, four rows per
+        // lane, and written into its stage's slot here.
         if (lane == 0 && n_main > 0) tma_prefetch_desc(&p.map_a);
         int slot = 0, sb = 0;
         uint32_t ph = 0, sph = 0;
         long long issued = 0, s_issued = 0;
         bool ok = true;
+        // scale-buffer index and phase parity of the item loaded last
+        int ld_buf = 0;
+        uint32_t ld_par = 0;
         auto load_scales = [&](const Work &t) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[sb], sph ^ 1, wc))) return false;
             uint8_t *sdst = scale_buf + sb * scale_bytes;
@@ -242,13 +265,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 bulk_load_w(sdst, p.scales + ((size_t)t.e * p.R + m0) * KB32, bytes, &s_full[sb]);
             }
             ++s_issued;
+            ld_buf = sb;
+            ld_par = sph;
             if (++sb == 2) { sb = 0; sph ^= 1; }
             return true;
         };
+        // The pass count of the item whose scale bytes sit in buffer `buf`: the largest
+        // E8M0 byte of its rows, then published for the other roles.  Returns the count
+        // (0 when a wait ran out).
+        auto publish_passes = [&](const Work &t, int buf, uint32_t par) -> int {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], par, wc))) return 0;
+            const int rows = MODE == MODE_UP ? GEMM_BM : min(GEMM_BM, p.R - t.mb * GEMM_BM);
+            const int n16 = rows * KB32 / 16;
+            const uint4 *src = reinterpret_cast<const uint4 *>(scale_buf + buf * scale_bytes);
+            uint32_t m4 = 0;
+            for (int i = lane; i < n16; i += 32) {
+                const uint4 v = src[i];
+                m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
+            }
+            uint32_t mx = max(max(m4 & 0xFFu, (m4 >> 8) & 0xFFu), max((m4 >> 16) & 0xFFu, m4 >> 24));
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            // (a stacked block's MMA already covers the lo2 rows)
+            const int np = !p.stacked && mx >= (uint32_t)LO2_SCALE_MIN ? 2 : 1;
+            if (lane == 0) npass_s[buf] = np;
+            __syncwarp();
+            mbar_arrive_w(&info_full[buf]);
+            return np;
+        };
         Work t;
+        int t_pass = 1;
         if (blockIdx.x < total) {
             work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            if constexpr (!SFI) ok = load_scales(t);     // per-item mode: the scale-factor warps load them
+            if constexpr (!SFI) {     // per-item mode: the scale-factor warps load the scales
+                ok = load_scales(t);
+                if (ok) t_pass = publish_passes(t, ld_buf, ld_par);
+                ok = ok && t_pass > 0;
+            }
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             uint4 tail[8];                   // the item's K tail codes (rows lane + 32j)
@@ -269,22 +321,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             // does not wait on global memory
             if (n_st > n_main) load_tail();
             Work tn;
-            if (w + (int)gridDim.x < total) {
+            const bool has_next = w + (int)gridDim.x < total;
+            int tn_buf = 0;
+            uint32_t tn_par = 0;
+            if (has_next) {
                 work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
                 if constexpr (!SFI) {
                     if (!load_scales(tn)) { ok = false; break; }
+                    tn_buf = ld_buf;
+                    tn_par = ld_par;
                 }
             }
-            for (int st = 0; st < n_st; ++st) {
+            const int n_it = n_st * t_pass;
+            for (int st = 0; st < n_it; ++st) {
+                const int kst = st < n_st ? st : st - n_st;      // the K stage (the same in both passes)
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                 uint8_t *adst = a_ring + slot * GEMM_A_STAGE;
-                if (st < n_main) {
+                if (kst < n_main) {
                     // the unpacked-type TMA counts the packed bytes: 128 rows x 64
                     mbar_arrive_expect_tx_w(&full[slot], 128u * 64u);
                     if (MODE == MODE_UP)
-                        tma_load_5d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, 0, 0, 4 * t.mb, t.e);
+                        tma_load_5d_w(adst, &p.map_a, &full[slot], kst * GEMM_KS, 0, 0, 4 * t.mb, t.e);
                     else
-                        tma_load_3d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, t.mb * GEMM_BM, t.e);
+                        tma_load_3d_w(adst, &p.map_a, &full[slot], kst * GEMM_KS, t.mb * GEMM_BM, t.e);
                 } else {
                     // K tail of rows lane + 32j: 2 x 16 code bytes -> the first four
                     // 16-byte units of the row (8 code bytes each, the rest zero),
@@ -307,6 +366,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
             }
+            if (!ok) break;
+            if constexpr (!SFI) {
+                if (has_next) {
+                    t_pass = publish_passes(tn, tn_buf, tn_par);
+                    if (t_pass == 0) { ok = false; break; }
+                }
+            }
             t = tn;
         }
         if (!ok) {
@@ -315,21 +381,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
     } else if (warp == 3) {
         // --------------------------------------------- B producer (activations)
-        // Per stage one TMA box: the token block's hi rows and then its lo rows.
+        // Per stage one TMA box: the token block's rows of two planes (hi, lo) or,
+        // stacked, of all three (hi, lo, lo2); in a lo2 pass the box starts at the
+        // lo2 plane (the plane after it lies outside the map and reads as zeros).
         if (lane == 0) tma_prefetch_desc(&p.map_b);
         if constexpr (MODE == MODE_DOWN) pdl_wait();     // h comes from the gate/up GEMM
         int slot = 0;
         uint32_t ph = 0;
+        int ib = 0;                          // scale buffer (and pass-count word) of the item
+        uint32_t iph = 0;
         long long issued = 0;
         bool ok = true;
         const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            for (int st = 0; st < n_st; ++st) {
+            int npass = 1;
+            if constexpr (!SFI) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[ib], iph, wc))) { ok = false; break; }
+                npass = npass_s[ib];
+                __syncwarp();
+                mbar_arrive_w(&s_empty[ib]);
+                if (++ib == 2) { ib = 0; iph ^= 1; }
+            }
+            for (int st = 0; st < n_st * npass; ++st) {
+                const int kst = st < n_st ? st : st - n_st;
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                 mbar_arrive_expect_tx_w(&full[slot], b_bytes);
-                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], st * GEMM_KS, t.p0, 0);
+                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], kst * GEMM_KS, t.p0, st < n_st ? 0 : 2);
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
             }
@@ -338,24 +417,37 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     } else if (warp == 1 || (warp == 2 && n_mma_warps == 2)) {
         // ---------------------------------------------------------------- MMA issue
         // MMA warp m takes the stages st = m, m + n_mma_warps, ... of every
-        // work item into its own accumulator pair; stage g of the CTA (counted
+        // work item into its own accumulator; stage g of the CTA (counted
         // over all items) sits in ring slot g % NS with phase parity (g / NS) & 1.
+        // A lo2 pass (per-stage mode) issues one MMA per K block over the slot's
+        // first plane (lo2) with hi's scale column.
         const int m = warp - 1;
         int db = 0, sb = 0;
         uint32_t dph = 0, sph = 0;
+        int ib = 0;
+        uint32_t iph = 0;
         bool ok = true, issued = false;
         // ring slot and phase parity of the current item's first stage
         int islot = 0;
-        uint32_t iph = 0;
+        uint32_t iph_ring = 0;
         auto advance = [&](int &sl, uint32_t &par, int by) {
             sl += by;
             while (sl >= NS) { sl -= NS; par ^= 1; }
         };
+        const bool stacked = SFI || p.stacked;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            const bool stacked = SFI || p.stacked;     // per-item mode always stacks hi and lo rows
-            const uint32_t n = stacked ? (uint32_t)(2 * NB) : (uint32_t)t.n_mma;
+            int npass = 1;
+            if constexpr (!SFI) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[ib], iph, wc))) { ok = false; break; }
+                npass = npass_s[ib];
+                __syncwarp();
+                mbar_arrive_w(&s_empty[ib]);
+                if (++ib == 2) { ib = 0; iph ^= 1; }
+            }
+            const int n_it = n_st * npass;
+            const uint32_t n = stacked ? (uint32_t)(3 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
             // E8M0 scales, M >> 4; K block kb of a stage takes scale byte kb (fields at 4 and 29)
             const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
@@ -365,13 +457,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (!__all_sync(0xffffffffu, mbar_wait(&d_empty[db], dph ^ 1, wc))) { ok = false; break; }
             if (SFI && !__all_sync(0xffffffffu, mbar_wait(&f_full[sb], sph, wc))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d_tmem = tmem + (uint32_t)((m * 2 + db) * d_cols);
+            const uint32_t d_tmem = tmem + (uint32_t)((m * n_dbuf + db) * d_cols);
             const uint32_t sf_item = tmem + sf_col0 + (uint32_t)(sb * sfi_cols);
             uint32_t acc = 0;
             int slot = islot;
-            uint32_t ph = iph;
+            uint32_t ph = iph_ring;
             advance(slot, ph, m);
-            for (int st = m; st < n_st; st += n_mma_warps) {
+            for (int st = m; st < n_it; st += n_mma_warps) {
+                const bool lo2_pass = st >= n_st;
+                const int kst = lo2_pass ? st - n_st : st;
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
                 tc_fence_after();
                 // descriptors of the slot's A and B; K block kb starts 32 bytes further
@@ -379,17 +473,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 const uint64_t ad = smem_desc_sw128(smem_addr(a_ring + slot * GEMM_A_STAGE));
                 const uint64_t bd = smem_desc_sw128(smem_addr(b_ring + slot * b_stage));
                 const uint64_t bd_lo = bd + (uint64_t)(NB * 128 >> 4);
-                const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * st)
+                const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * kst)
                                         : tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
                 const uint32_t sfb = SFI ? sf + 4 : sf + 8;
-                if (st < n_main) {
+                // K blocks of this stage: 4, or 1..3 in the K tail
+                const int nkb = kst < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
+                if (lo2_pass) {
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)
+                        if (kb < nkb) mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, 1u);
+                } else if (nkb == 4) {
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
                         mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, (acc | kb) ? 1u : 0u);
                         if (!stacked) mma_mx_w(d_tmem, ad + 2 * kb, bd_lo + 2 * kb, idesc[kb], sf, sf + 16, 1u);
                     }
                 } else {
-                    const int nkb = (p.K - n_main * GEMM_KS) / 32;    // the K tail: 1..3 blocks
 #pragma unroll
                     for (int kb = 0; kb < 3; ++kb) {
                         if (kb >= nkb) break;
@@ -403,10 +502,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 advance(slot, ph, n_mma_warps);
             }
             if (!ok) break;
-            advance(islot, iph, n_st);
+            advance(islot, iph_ring, n_it);
             mma_commit_w(&d_full[m * 2 + db]);
             if (SFI) mma_commit_w(&f_empty[sb]);
-            if (++db == 2) { db = 0; dph ^= 1; }
+            if (++db == n_dbuf) { db = 0; dph ^= 1; }
             if (++sb == 2) { sb = 0; sph ^= 1; }
         }
         if (!ok && issued) {
@@ -418,30 +517,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // Warp q writes TMEM lane quarter q.  A stage's scale factors take 4-column
         // groups: column c of the A group holds, in lane 32q + i, the four E8M0
         // bytes (32-blocks 4st..4st+3) of weight row 32c + i; column c of the B
-        // group holds token row 32c + i (stacked: rows of [hi | lo]).  Per-item
-        // mode writes every stage of a work item into an item region once;
-        // per-stage mode writes each stage into the slot of its ring stage.
+        // group holds token row 32c + i (stacked: rows of [hi | lo | lo2], lo2 rows
+        // taking hi's words).  Per-item mode writes every stage of a work item into
+        // an item region once; per-stage mode writes each stage into the slot of its
+        // ring stage (both passes of a lo2 item carry the same words: A's, hi's at
+        // +8 and lo's at +16).
         const int q = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int slot = 0, sb = 0;
         uint32_t ph = 0, sph = 0;
         bool ok = true;
-        const int n_sfb = p.stacked ? (2 * NB + 31) / 32 : (NB + 31) / 32;
+        const int n_sfb = p.stacked ? (3 * NB + 31) / 32 : (NB + 31) / 32;
         uint32_t bph = 0;                    // phase parity of the staging barriers (one phase per item)
-        // B scale words of stage st of item t into v: stacked, word c is row 32c + lane of
-        // [hi rows | lo rows]; otherwise words c / 6 + c are the hi / lo word
+        // B scale words of K stage kst of item t into v: stacked, word c is row 32c + lane of
+        // [hi rows | lo rows | lo2 rows]; otherwise words c and 6 + c are the hi and lo words
         // of token row 32c + lane.  Rows past the block's tokens get 2^0.
-        auto load_bsf = [&](const Work &t, int st, uint32_t (&v)[SF_WORDS]) {
-                const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
+        auto load_bsf = [&](const Work &t, int kst, uint32_t (&v)[SF_WORDS]) {
+                const uint32_t *bsf = p.b_sf + (size_t)kst * 2 * p.P_max + t.p0;
 #pragma unroll
                 for (int i = 0; i < SF_WORDS; ++i) v[i] = 0x7F7F7F7Fu;
                 if (p.stacked) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < SF_WORDS / 2; ++c) {
                         const int r = 32 * c + lane;
-                        const int plane = r >= NB ? 1 : 0;
+                        const int plane = r / NB;
                         const int j = r - plane * NB;
-                        if (c < n_sfb && r < 2 * NB && j < t.n_valid) v[c] = __ldg(bsf + (size_t)plane * p.P_max + j);
+                        if (c < n_sfb && r < 3 * NB && j < t.n_valid)
+                            v[c] = __ldg(bsf + (plane == 1 ? (size_t)p.P_max : 0) + j);
                     }
                 } else {
 #pragma unroll
@@ -454,24 +556,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     }
                 }
         };
-        // per-stage mode: stage st's B words sit in bw[st % SF_PD], loaded SF_PD stages
-        // ahead; the slots an item's last stages free take the next item's first stages
+        // per-stage mode: the item's stage st (counted over both passes) uses bw[st % SF_PD],
+        // loaded SF_PD stages ahead; an item with at least SF_PD stages loads the next item's
+        // first SF_PD stages into the slots its last stages free
         uint32_t bw[SF_PD][SF_WORDS];
+        bool bw_ready = false;               // bw holds the current item's first stages
         if constexpr (!SFI) {
             if constexpr (MODE == MODE_DOWN) pdl_wait();     // h's scales come from the gate/up GEMM
-            if (blockIdx.x < total) {
-                Work t0;
-                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t0);
-#pragma unroll
-                for (int i = 0; i < SF_PD; ++i)
-                    if (i < n_st) load_bsf(t0, i, bw[i]);
-            }
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
+            int npass = 1;
             if constexpr (!SFI) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[sb], sph, wc))) { ok = false; break; }
+                npass = npass_s[sb];
             }
             const uint8_t *sbase = scale_buf + (SFI ? 0 : sb * scale_bytes);
             const uint8_t *srow[4];
@@ -481,14 +581,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 srow[c] = sbase + tile_scale_row<MODE>(32 * c + lane) * KB32;
                 row_ok[c] = MODE == MODE_UP || t.mb * GEMM_BM + 32 * c + lane < p.R;
             }
-            // A words of stage st: column c
-            auto a_words = [&](int st, uint32_t *v) {
-                const int nblk = KB32 - 4 * st;     // 32-blocks of this stage inside K: 2 or >= 4
+            // A words of K stage kst: column c
+            auto a_words = [&](int kst, uint32_t *v) {
+                const int nblk = KB32 - 4 * kst;     // 32-blocks of this stage inside K: 2 or >= 4
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t wv = 0x7F7F7F7Fu;
                     if (row_ok[c]) {
-                        const uint16_t *s16 = reinterpret_cast<const uint16_t *>(srow[c] + 4 * st);
+                        const uint16_t *s16 = reinterpret_cast<const uint16_t *>(srow[c] + 4 * kst);
                         const uint32_t lo = s16[0];
                         const uint32_t hi = nblk > 2 ? (uint32_t)s16[1] : 0x7F7Fu;
                         wv = lo | (hi << 16);
@@ -523,15 +623,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 #pragma unroll
                 for (int i = 0; i < GEMM_SFI_STAGES_MAX / 4; ++i) {
                     const int st = q + 4 * i;
-                    // stacked block: B column c is row 32c + lane of [hi rows | lo rows]
+                    // stacked block: B column c is row 32c + lane of [hi rows | lo rows | lo2 rows]
                     const uint32_t *bsf = p.b_sf + (size_t)min(st, n_st - 1) * 2 * p.P_max + t.p0;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int r = 32 * c + lane;
-                        const int plane = r >= NB ? 1 : 0;
+                        const int plane = r / NB;
                         const int j = r - plane * NB;
-                        bwr[i][c] = st < n_st && c < n_sfb && r < 2 * NB && j < t.n_valid
-                                        ? __ldg(bsf + (size_t)plane * p.P_max + j) : 0x7F7F7F7Fu;
+                        bwr[i][c] = st < n_st && c < n_sfb && r < 3 * NB && j < t.n_valid
+                                        ? __ldg(bsf + (plane == 1 ? (size_t)p.P_max : 0) + j) : 0x7F7F7F7Fu;
                     }
                 }
                 // the staging buffer is free once all four warps have read the last item's words
@@ -570,19 +670,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 mbar_arrive_w(&f_full[sb]);
                 bph ^= 1;
             } else {
+                const int n_it = n_st * npass;
+                if (!bw_ready) {
+#pragma unroll
+                    for (int i = 0; i < SF_PD; ++i) load_bsf(t, i % n_st, bw[i]);
+                }
                 Work tn;
                 const bool has_next = w + (int)gridDim.x < total;
                 if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
-                for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
+                const bool pre_next = has_next && n_it >= SF_PD;
+                for (int st0 = 0; st0 < n_it && ok; st0 += SF_PD) {
 #pragma unroll
                     for (int i = 0; i < SF_PD; ++i) {
                         const int st = st0 + i;
-                        if (st >= n_st) break;
+                        if (st >= n_it) break;
+                        const int kst = st < n_st ? st : st - n_st;
                         if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                         const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
                         {
                             uint32_t v[4];
-                            a_words(st, v);
+                            a_words(kst, v);
                             tmem_st4(sf, v);
                         }
                         // B: the hi (and lo) columns of the token block, one store per
@@ -591,21 +698,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         // 15 take two lo words, past any block's hi columns)
                         const uint32_t *b = bw[i];
                         if (p.stacked) {
-                            tmem_st4v(sf + 8, b[0], b[1], b[2], b[3]);
+                            if (n_sfb <= 4) tmem_st4v(sf + 8, b[0], b[1], b[2], b[3]);
+                            else tmem_st8v(sf + 8, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7]);
                         } else {
                             tmem_st8v(sf + 8, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7]);
                             tmem_st4v(sf + 16, b[6], b[7], b[8], b[9]);
                             tmem_st2v(sf + 20, b[10], b[11]);
                         }
                         tmem_wait_st();
-                        if (st + SF_PD < n_st) load_bsf(t, st + SF_PD, bw[i]);
-                        else if (has_next && i < n_st) load_bsf(tn, i, bw[i]);
+                        if (st + SF_PD < n_it) {
+                            const int kn = st + SF_PD;
+                            load_bsf(t, kn < n_st ? kn : kn - n_st, bw[i]);
+                        } else if (pre_next) {
+                            load_bsf(tn, i % n_st, bw[i]);
+                        }
                         tc_fence_before();
                         __syncwarp();
                         mbar_arrive_w(&full[slot]);
                         if (++slot == NS) { slot = 0; ph ^= 1; }
                     }
                 }
+                bw_ready = pre_next;
             }
             if (!ok) break;
             if constexpr (!SFI) {
@@ -645,10 +758,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 float acc[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-                // the sum over the MMA warps' accumulators and, stacked, their hi and lo halves
+                // the sum over the MMA warps' accumulators and, stacked, their hi, lo and lo2 thirds
                 for (int mw = 0; mw < n_mma_warps; ++mw) {
-                    const uint32_t d_tmem = lane_base + (uint32_t)((mw * 2 + db) * d_cols);
-                    for (int half = 0; half < (p.stacked ? 2 : 1); ++half) {
+                    const uint32_t d_tmem = lane_base + (uint32_t)((mw * n_dbuf + db) * d_cols);
+                    for (int half = 0; half < (p.stacked ? 3 : 1); ++half) {
                         uint32_t v[16];
                         tmem_ld16(d_tmem + (uint32_t)(half * NB + c0), v);
                         tmem_wait_ld();
@@ -709,13 +822,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         const int s_hi = e4m3_block_exp(m[i]);
                         const int s_lo = max(s_hi - 4, -126);
                         const float v = hv[i];
+                        // the three terms; each residual is exact in fp32
                         const uint32_t qh = f32x2_to_e4m3x2(v * pow2f(-s_hi), 0.0f) & 0xFFu;
                         const float res = v - e4m3_to_f32(qh) * pow2f(s_hi);
                         const uint32_t ql = f32x2_to_e4m3x2(res * pow2f(-s_lo), 0.0f) & 0xFFu;
+                        const float res2 = res - e4m3_to_f32(ql) * pow2f(s_lo);
+                        const uint32_t ql2 = f32x2_to_e4m3x2(res2 * pow2f(-s_hi), 0.0f) & 0xFFu;
                         if (col < t.n_valid) {
                             const size_t prow = (size_t)(t.p0 + col);
                             p.h_q[prow * p.Kf + j] = (uint8_t)qh;
                             p.h_q[((size_t)p.P_max + prow) * p.Kf + j] = (uint8_t)ql;
+                            p.h_q[((size_t)2 * p.P_max + prow) * p.Kf + j] = (uint8_t)ql2;
                             if ((q & 1) == 0 && (lane & 15) == 0) {
                                 // one lane per (column, 32-block): the two scale bytes
                                 const size_t wi = (size_t)(fblk >> 2) * 2 * p.P_max;
@@ -738,7 +855,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&d_empty[db]);
-            if (++db == 2) { db = 0; dph ^= 1; }
+            if (++db == n_dbuf) { db = 0; dph ^= 1; }
         }
     }
 

@@ -65,16 +65,17 @@ inline bool encode_a_down(CUtensorMap *m, const void *codes, int E, int d, int K
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Two-term E4M3 B operand u8 [2 planes][rows][Kpad] (the hi plane, then the lo
-// plane, each `rows` rows): a 3-D view {Kpad, rows, 2} whose box {128 bytes,
-// box_rows, 2} brings a token block's hi rows and their lo rows in one copy
-// (hi rows first in shared memory); 128-byte swizzle, zero fill past the last row.
-inline bool encode_bq(CUtensorMap *m, const void *base, int rows, int Kpad, int box_rows) {
+// E4M3 B operand u8 [3 planes][rows][Kpad] (hi, lo and lo2 planes, each `rows`
+// rows): a 3-D view {Kpad, rows, 3} whose box {128 bytes, box_rows, box_planes}
+// brings a token block's rows of box_planes consecutive planes in one copy,
+// plane by plane in shared memory; 128-byte swizzle, zero fill past the last row
+// and past the last plane.
+inline bool encode_bq(CUtensorMap *m, const void *base, int rows, int Kpad, int box_rows, int box_planes) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)Kpad, (cuuint64_t)rows, 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)Kpad, (cuuint64_t)rows, 3};
     const cuuint64_t strides[2] = {(cuuint64_t)Kpad, (cuuint64_t)rows * Kpad};
-    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 2};
+    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, (cuuint32_t)box_planes};
     const cuuint32_t es[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -101,7 +102,7 @@ inline int token_block_rows(int T) {
 inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, int E, int P_max, int num_sms,
                      int *grid, int *smem) {
     p.nb_rows = token_block_rows(T);
-    // small token blocks: one MMA over the hi rows and the lo rows together
+    // small token blocks: one MMA over the hi, lo and lo2 rows together (N = 3 nb_rows <= 192)
     p.stacked = p.nb_rows <= 64 ? 1 : 0;
     if (mode == MODE_UP) {
         p.K = d;
@@ -118,12 +119,13 @@ inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, in
     p.P_max = P_max;
     p.Kf = round_up_128(F);
     // per-item scale factors (and two MMA warps) when a stacked block's item
-    // regions fit in TMEM next to four accumulators
+    // regions fit in TMEM next to the two MMA warps' accumulators
     const int n_st = (p.K + GEMM_KS - 1) / GEMM_KS;
-    p.sf_item = p.stacked && n_st <= GEMM_SFI_STAGES_MAX &&
+    // (an item region's B group holds the scale words of at most 128 stacked rows)
+    p.sf_item = p.stacked && 3 * p.nb_rows <= 128 && n_st <= GEMM_SFI_STAGES_MAX &&
                 gemm_tmem_cols_item(p.nb_rows, p.stacked, n_st) <= 512 ? 1 : 0;
     auto fits = [&](int ns) {
-        return gemm_smem_plan(p.K, E, p.nb_rows, ns, p.sf_item).total <= GEMM_SMEM_LIMIT &&
+        return gemm_smem_plan(p.K, E, p.nb_rows, p.stacked, ns, p.sf_item).total <= GEMM_SMEM_LIMIT &&
                (p.sf_item || gemm_tmem_cols(p.nb_rows, p.stacked, ns) <= 512);
     };
     // as many stages as shared memory (and, per stage, TMEM) hold
@@ -131,7 +133,7 @@ inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, in
     while (ns > 2 && !fits(ns)) --ns;
     if (!fits(ns)) return MOE_ERR_ARG;
     p.n_stages = ns;
-    *smem = gemm_smem_plan(p.K, E, p.nb_rows, ns, p.sf_item).total;
+    *smem = gemm_smem_plan(p.K, E, p.nb_rows, p.stacked, ns, p.sf_item).total;
     const long long P = (long long)T * top_k;
     const long long max_blocks = (P < E ? P : E) + P / p.nb_rows;
     const long long max_work = (long long)p.MB * max_blocks;

@@ -65,28 +65,34 @@ struct GroupParams {
     float *row_w;               // [P]
     int *pair_row;              // [P] expert-sorted row of pair (token, slot)
     unsigned int *err;
-    // the expert-sorted two-term E4M3 copy of the normalised tokens (gate/up B operand)
+    // the expert-sorted E4M3 terms of the normalised tokens (gate/up B operand)
     const __half *xn16;         // fp16 [T, d]
     const float *rho;           // [T]
-    uint8_t *xq;                // [2][P_max][Kd]
-    uint32_t *xsf;              // [Kd/128][2][P_max]
+    uint8_t *xq;                // [3][P_max][Kd]: hi, lo, lo2 planes
+    uint32_t *xsf;              // [Kd/128][2][P_max]: scales of the hi (also lo2) and lo planes
     int P_max, d, Kd;
 };
 
 // Grouped block-scaled GEMM over (expert, 128-row weight block, token block)
 // work items: MXFP4 weights (E2M1 codes, E8M0 block scales) times the
-// activations held as two E4M3 terms (hi + lo, each with its own E8M0 block
-// scales), fp32 accumulation in TMEM.  MODE_UP: rows are the gate/linear pairs
-// of W13, epilogue is the clamped SwiGLU, written as the down GEMM's two-term
-// B.  MODE_DOWN: rows are W2's, epilogue writes the routing-weighted expert
-// output rows.
+// activations held as three E4M3 terms per 32-element block with exponent s:
+//   hi  = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)),
+//   lo2 = e4m3((v - hi 2^s - lo 2^(s-4)) / 2^s)
+// (hi and lo keep about 8 significant bits of v, the three together about 12;
+// lo2 shares hi's scale byte, so an MMA over lo2 rows reads hi's scale
+// column).  fp32 accumulation in TMEM.  Stacked token blocks (decode-sized)
+// always use all three terms in one MMA; large blocks use hi + lo, and add a
+// pass over lo2 for work items whose weights reach E8M0 byte LO2_SCALE_MIN.
+// MODE_UP: rows are the gate/linear pairs of W13, epilogue is the clamped
+// SwiGLU, written as the down GEMM's B.  MODE_DOWN: rows are W2's, epilogue
+// writes the routing-weighted expert output rows.
 enum { MODE_UP = 0, MODE_DOWN = 1 };
 
 struct GemmParams {
     CUtensorMap map_a;          // E2M1 codes, 16 x 4-bit per 16 bytes in shared memory (unpacked TMA type);
                                 //   UP: 5-D {K_main, 16 rows, 2 halves, F/16 groups, E}, box {128, 16, 2, 4, 1}
                                 //   DOWN: 3-D {K_main, d, E}, box {128, 128, 1}
-    CUtensorMap map_b;          // u8 [2][P_max][Kpad] E4M3 hi plane then lo plane; box {128, nb_rows, 2}
+    CUtensorMap map_b;          // u8 [3][P_max][Kpad] E4M3 hi, lo, lo2 planes; box {128, nb_rows, 3 stacked / 2}
     const uint8_t *codes;       // u8 [E][R][K/2] (the K tail is read directly)
     const uint8_t *scales;      // u8 [E][R][K/32]
     const uint16_t *bias;       // bf16 [E][R]
@@ -98,7 +104,7 @@ struct GemmParams {
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= GEMM_NB_MAX)
-    int stacked;                // 1: one MMA covers the hi and lo rows (N = 2 nb_rows); 0: one MMA per term
+    int stacked;                // 1: one MMA covers the hi, lo and lo2 rows (N = 3 nb_rows); 0: one MMA per term
     int n_stages;               // shared-memory ring depth (and TMEM scale-factor ring depth when !sf_item)
     int sf_item;                // 1: a work item's scale factors are written to TMEM once, before its first
                                 //    stage, and two MMA warps take alternate stages (decode-sized blocks);
@@ -107,7 +113,7 @@ struct GemmParams {
     const int *counts, *offsets, *tiles;
     const int *row_token;       // [P]
     const float *row_w;         // [P]
-    // UP output: the down GEMM's B (two E4M3 planes [2][P_max][Kf]) and its scales
+    // UP output: the down GEMM's B (three E4M3 planes [3][P_max][Kf]) and its scales
     uint8_t *h_q;
     uint8_t *h_sf;              // bytes of [Kf/128][2][P_max] words
     int Kf;                     // F rounded up to 128
@@ -124,6 +130,12 @@ constexpr int GEMM_NB_MAX = 192;      // token rows per work item, at most
 constexpr int GEMM_STAGES_MAX = 12;
 constexpr int GEMM_A_STAGE = GEMM_BM * 128;   // unpacked E2M1: one byte per element in shared memory
 constexpr int GEMM_SF_COLS = 24;      // TMEM columns per scale-factor slot: A at +0, B hi at +8, B lo at +16
+// Large token blocks add a pass over the third activation term (lo2) to the work
+// items whose weight rows hold an E8M0 byte of at least this (weights of
+// magnitude 3 or more: 6 * 2^-1).  Below it two terms keep the block well inside
+// its tolerance; above it the pre-activations grow large enough that two-term
+// rounding of the activations moves the clamped SwiGLU's output.
+constexpr int LO2_SCALE_MIN = 126;
 constexpr int GEMM_SMEM_LIMIT = 227 * 1024;
 
 // Shared-memory plan of the GEMM kernel (all offsets from a 1024-aligned base).
@@ -140,17 +152,24 @@ __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a *
 
 __host__ __device__ inline int gemm_num_barriers(int n_stages) {
     // stage full/empty [NS], A-scale full/empty [2], D full [2 MMA warps][2], D empty [2],
-    // drain [2], epilogue exchange [2][2], item scale factors full/empty [2], staged B words full/empty
-    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2;
+    // drain [2], epilogue exchange [2][2], item scale factors full/empty [2], staged B words full/empty,
+    // item pass count published [2]
+    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2 + 2;
 }
 
-__host__ __device__ inline int gemm_b_stage_bytes(int nb_rows) { return 2 * nb_rows * 128; }
+// B ring slot: the token block's hi, lo and lo2 rows (stacked) or two planes (hi and lo, or lo2
+// and an empty plane in a lo2 pass)
+__host__ __device__ inline int gemm_b_planes(int stacked) { return stacked ? 3 : 2; }
+__host__ __device__ inline int gemm_b_stage_bytes(int nb_rows, int stacked) {
+    return gemm_b_planes(stacked) * nb_rows * 128;
+}
 
-__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int n_stages, int sf_item) {
+__host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int stacked, int n_stages,
+                                                   int sf_item) {
     GemmSmem s;
     s.a_off = 0;
     s.b_off = n_stages * GEMM_A_STAGE;
-    s.scale_off = s.b_off + n_stages * gemm_b_stage_bytes(nb_rows);
+    s.scale_off = s.b_off + n_stages * gemm_b_stage_bytes(nb_rows, stacked);
     const int scale_bytes = align_up(GEMM_BM * (K / 32), 128);
     // A scale bytes: double-buffered per-stage mode (bulk copies one item ahead), one buffer per-item mode
     s.amax_off = s.scale_off + (sf_item ? 1 : 2) * scale_bytes;
@@ -158,22 +177,23 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
     s.bsf_off = s.meta_off + align_up(8 * nb_rows * 4, 16);        // per epilogue warp: one value per column
     s.bar_off = s.bsf_off + (sf_item ? GEMM_SFI_BSF_BYTES : 0);
     s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_stages) * 8, 16);
-    // misc: tmem base, abort flag, then counts/offsets/tiles caches
+    // misc: tmem base, abort flag, the lo2 pass flags of the two scale buffers, then
+    // counts/offsets/tiles caches
     s.total = s.misc_off + 16 + 3 * (E + 1) * 4;
     s.total = align_up(s.total, 128) + 1024;  // slack for aligning the base
     return s;
 }
 
 // TMEM columns of the plan.  Per-stage mode: accumulators (2 buffers), then the
-// ring of scale-factor slots.  Per-item mode: accumulators [2 MMA warps][2
-// buffers], then two item regions of 8 columns per stage (A at +0, B at +4).
+// ring of scale-factor slots.  Per-item mode: accumulators [2 MMA warps] (one
+// buffer each), then two item regions of 8 columns per stage (A at +0, B at +4).
 constexpr int GEMM_SFI_COLS = 8;
-__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 2 * nb_rows : nb_rows; }
+__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 3 * nb_rows : nb_rows; }
 __host__ __device__ inline int gemm_tmem_cols(int nb_rows, int stacked, int n_stages) {
     return 2 * gemm_d_cols(nb_rows, stacked) + GEMM_SF_COLS * n_stages;
 }
 __host__ __device__ inline int gemm_tmem_cols_item(int nb_rows, int stacked, int n_st) {
-    return 4 * gemm_d_cols(nb_rows, stacked) + 2 * GEMM_SFI_COLS * n_st;
+    return 2 * gemm_d_cols(nb_rows, stacked) + 2 * GEMM_SFI_COLS * n_st;
 }
 
 }  // namespace moe

@@ -38,7 +38,8 @@ using namespace moe;
 namespace {
 
 // 8 MiB of scratch: enough for decode-sized batches of the gpt-oss layers
-// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 6.5 MiB).
+// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 7.8 MiB with 128
+// experts).
 constexpr size_t kScratchBytes = 8u << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -128,7 +129,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     const int Kd = round_up_128(d), Kf = round_up_128(F);
     const size_t sizes[] = {(size_t)T * d * 2, (size_t)T * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
                             (size_t)(E + 1) * 4, P * 4, P * 4, P * 4,
-                            2 * P * Kd, (size_t)(Kd / 128) * 2 * P * 4, 2 * P * Kf, (size_t)(Kf / 128) * 2 * P * 4,
+                            3 * P * Kd, (size_t)(Kd / 128) * 2 * P * 4, 3 * P * Kf, (size_t)(Kf / 128) * 2 * P * 4,
                             P * d * 4, 64, (size_t)T * E * 4, (size_t)T * 4};
     size_t total = 0;
     for (size_t v : sizes) total += r256(v);
@@ -164,8 +165,9 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nb = token_block_rows(T);
+    const int planes = gemm_b_planes(nb <= 64 ? 1 : 0);
     CUtensorMap map_xq, map_hq;
-    if (!encode_bq(&map_xq, xq, (int)P, Kd, nb) || !encode_bq(&map_hq, hq, (int)P, Kf, nb))
+    if (!encode_bq(&map_xq, xq, (int)P, Kd, nb, planes) || !encode_bq(&map_hq, hq, (int)P, Kf, nb, planes))
         return MOE_ERR_CUDA;
     // the error word and the route kernel's per-token counters must start at zero
     // on every call (the array keeps whatever the previous call, of any shape, left)

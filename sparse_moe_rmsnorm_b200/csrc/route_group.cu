@@ -6,8 +6,8 @@
 //                    16 experts);
 //   group_permute_kernel  expert histogram, exclusive scan and a stable
 //                    permutation of the (token, expert) pairs into
-//                    expert-contiguous rows, and the expert-sorted two-term E4M3
-//                    copy of the normalised tokens (the gate/up GEMM's B operand);
+//                    expert-contiguous rows, and the expert-sorted E4M3 terms
+//                    of the normalised tokens (the gate/up GEMM's B operand);
 //   combine_kernel   y = x + the token's weighted expert rows, in bf16.
 #include <cfloat>
 #include <climits>
@@ -762,12 +762,15 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RoutePara
 // writes counts, offsets and tiles.
 //
 // B operand row r: the normalised activations of token row_token[r],
-// v = xn16 * rho, as two E4M3 terms per 32-element block with E8M0 scale s
+// v = xn16 * rho, as three E4M3 terms per 32-element block with E8M0 scale s
 // (the exponent that fits the block maximum to 448):
-//   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)).
-// Out: xq[plane][r][0:Kd] (plane 0 hi, plane 1 lo; columns d..Kd zero) and
-// xsf[g][plane][r] = the scale bytes of the 32-blocks 4g..4g+3 (byte i is
-// block 4g+i).  A warp takes 32 consecutive 32-blocks of a row, one per lane.
+//   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)),
+//   lo2 = e4m3((v - hi 2^s - lo 2^(s-4)) / 2^s)
+// (every residual is exact in fp32).  Out: xq[plane][r][0:Kd] (planes hi, lo,
+// lo2; columns d..Kd zero) and xsf[g][plane][r] = the scale bytes of the
+// 32-blocks 4g..4g+3 (byte i is block 4g+i) of plane 0 (hi, and lo2, which
+// shares its scale) and plane 1 (lo).  A warp takes 32 consecutive 32-blocks of
+// a row, one per lane.
 constexpr int GROUP_ROWS_MAX = 1024;   // expert-sorted rows per CTA, at most
 
 // Blocks b0 + lane (lane < 32) of expert-sorted row r, token tok.
@@ -779,6 +782,7 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
         const int b = b0 + lane;
         uint32_t s_hi = 127, s_lo = 127;
         uint32_t qh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ql[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        uint32_t ql2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (b < nblk) {
             float v[32];
 #pragma unroll
@@ -796,16 +800,20 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
             for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
             const int e_hi = e4m3_block_exp(amax);
             const int e_lo = max(e_hi - 4, -126);
-            const float inv_hi = pow2f(-e_hi), inv_lo = pow2f(-e_lo), mul_hi = pow2f(e_hi);
+            const float inv_hi = pow2f(-e_hi), inv_lo = pow2f(-e_lo), mul_hi = pow2f(e_hi), mul_lo = pow2f(e_lo);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const uint32_t h = f32x2_to_e4m3x2(v[2 * i] * inv_hi, v[2 * i + 1] * inv_hi);
                 float d0, d1;
                 e4m3x2_to_f32x2(h, d0, d1);
-                const uint32_t l = f32x2_to_e4m3x2((v[2 * i] - d0 * mul_hi) * inv_lo,
-                                                   (v[2 * i + 1] - d1 * mul_hi) * inv_lo);
+                const float r0 = v[2 * i] - d0 * mul_hi, r1 = v[2 * i + 1] - d1 * mul_hi;
+                const uint32_t l = f32x2_to_e4m3x2(r0 * inv_lo, r1 * inv_lo);
+                float l0, l1;
+                e4m3x2_to_f32x2(l, l0, l1);
+                const uint32_t l2 = f32x2_to_e4m3x2((r0 - l0 * mul_lo) * inv_hi, (r1 - l1 * mul_lo) * inv_hi);
                 qh[i >> 1] |= h << (16 * (i & 1));
                 ql[i >> 1] |= l << (16 * (i & 1));
+                ql2[i >> 1] |= l2 << (16 * (i & 1));
             }
             s_hi = (uint32_t)(e_hi + 127);
             s_lo = (uint32_t)(e_lo + 127);
@@ -813,10 +821,13 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
         if (b < nblk_pad) {
             uint4 *dh = reinterpret_cast<uint4 *>(p.xq + (size_t)r * p.Kd + 32 * b);
             uint4 *dl = reinterpret_cast<uint4 *>(p.xq + ((size_t)p.P_max + r) * p.Kd + 32 * b);
+            uint4 *dl2 = reinterpret_cast<uint4 *>(p.xq + ((size_t)2 * p.P_max + r) * p.Kd + 32 * b);
             dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
             dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
             dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
             dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
+            dl2[0] = make_uint4(ql2[0], ql2[1], ql2[2], ql2[3]);
+            dl2[1] = make_uint4(ql2[4], ql2[5], ql2[6], ql2[7]);
         }
         // the scale bytes of four consecutive blocks (lanes 4m..4m+3) as one word
         uint32_t wh = s_hi, wl = s_lo;

@@ -1,4 +1,4 @@
-"""The two-term E4M3 encoding of activations the block-scaled GEMMs read, in plain numpy.
+"""The E4M3 terms of activations the block-scaled GEMMs read, in plain numpy.
 
 This is the definition the device encoders (the permute kernel for the normalised tokens, the
 gate/up epilogue for h) implement, written out for tests: per block of 32 consecutive elements
@@ -6,9 +6,11 @@ of a row, with v the fp32 values,
   s   = x - 8 + [m > 1.75], where max|v| = m * 2^x, 1 <= m < 2, clamped to [-126, 126]
         (the E8M0 exponent that brings the block maximum to at most 448 = 1.75 * 2^8);
   hi  = e4m3(v * 2^-s),   lo = e4m3((v - hi * 2^s) * 2^-s_lo),   s_lo = max(s - 4, -126),
+  lo2 = e4m3((v - hi * 2^s - lo * 2^s_lo) * 2^-s),
 with e4m3() the round-to-nearest-even conversion to OCP E4M3 (bias 7, 3 mantissa bits,
-subnormals below 2^-6, largest finite 448), saturating to +-448.  v is then represented as
-hi * 2^s + lo * 2^s_lo; the scale bytes are s + 127 and s_lo + 127.
+subnormals below 2^-6, largest finite 448), saturating to +-448.  Two terms represent v as
+hi * 2^s + lo * 2^s_lo, three add lo2 * 2^s (lo2 shares hi's scale); the scale bytes are
+s + 127 and s_lo + 127.
 """
 from __future__ import annotations
 
@@ -65,6 +67,30 @@ def encode_two_term(v: np.ndarray):
     res = blk - e4m3_decode(hi) * np.exp2(s)[..., None]
     lo = e4m3_encode(res * np.exp2(-s_lo)[..., None])
     return (hi.reshape(rows, K), lo.reshape(rows, K), (s + 127).astype(np.uint8), (s_lo + 127).astype(np.uint8))
+
+
+def encode_three_term(v: np.ndarray):
+    """v: float32 [rows, K] -> (hi u8, lo u8, lo2 u8, s_hi u8, s_lo u8 [rows, K/32])."""
+    v = np.asarray(v, dtype=np.float32)
+    rows, K = v.shape
+    hi, lo, s_hi, s_lo = encode_two_term(v)
+    blk = v.reshape(rows, K // 32, 32).astype(np.float64)
+    s = s_hi.astype(np.float64) - 127
+    sl = s_lo.astype(np.float64) - 127
+    res = (blk - e4m3_decode(hi.reshape(rows, K // 32, 32)) * np.exp2(s)[..., None]
+           - e4m3_decode(lo.reshape(rows, K // 32, 32)) * np.exp2(sl)[..., None])
+    lo2 = e4m3_encode(res * np.exp2(-s)[..., None])
+    return hi, lo, lo2.reshape(rows, K), s_hi, s_lo
+
+
+def decode_terms(planes, s_hi, s_lo) -> np.ndarray:
+    """Sum of the first len(planes) terms (hi, lo[, lo2]) -> float64 [rows, K]."""
+    rows, K = planes[0].shape
+    scale = (s_hi, s_lo, s_hi)
+    out = np.zeros((rows, K // 32, 32))
+    for q, sc in zip(planes, scale):
+        out += e4m3_decode(q).reshape(rows, K // 32, 32) * np.exp2(sc.astype(np.float64) - 127)[..., None]
+    return out.reshape(rows, K)
 
 
 def decode_two_term(hi, lo, s_hi, s_lo) -> np.ndarray:

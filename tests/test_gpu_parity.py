@@ -14,15 +14,26 @@ import oracle
 import sparse_moe_rmsnorm_b200 as moe
 from moe_inputs import CONFIGS, bf16_bits_to_f32, custom_layer, make_config_inputs
 from _parity import compare_block, excluded_tokens
-from _e4m3 import decode_two_term, encode_two_term, scale_bytes_from_words
+from _e4m3 import decode_terms, encode_three_term, scale_bytes_from_words
 
 pytestmark = pytest.mark.gpu
 
-# Tighter bound on the fp32 accumulator y_acc (before the bf16 output cast).  The expert GEMMs see
-# the activations (normalised tokens, h) as two E4M3 terms per 32-block, at most 2^-9 relative error
-# per element; a float64 emulation of those rounding points gives 1.1e-3 mean relative error on the
-# 2880-wide layers (5e-4 on small ones).  2.5e-3 leaves room for the fp32 accumulation order.
-ACC_MEAN_REL = 2.5e-3
+# Tighter bounds on the fp32 accumulator y_acc (before the bf16 output cast), beside the block's
+# stated 2e-2 max / 5e-3 mean on y.
+#  * Decode-sized batches (T <= 64) reach the tensor core with three E4M3 terms per activation
+#    (about 12 significant bits, the fp16 precision of the normalised tokens): 1e-3.
+#  * Larger batches use two terms (about 8 bits, the precision of bf16) on weights whose E8M0
+#    bytes stay below 126.  The bound there is what bf16 operands -- the precision of the scope
+#    statement's own design, bf16 activations against exactly decoded weights -- give on the
+#    2880-wide layer: a float64 model of nothing but those bf16 roundings measures 2.9e-3 mean
+#    relative error on the accumulator of the decode20b layer, so 2.5e-3 asks the two-term path
+#    to be at least as exact as bf16 operands.
+ACC_MEAN_REL_THREE_TERMS = 1e-3
+ACC_MEAN_REL_TWO_TERMS = 2.5e-3
+
+
+def acc_bound(T):
+    return ACC_MEAN_REL_THREE_TERMS if T <= 64 else ACC_MEAN_REL_TWO_TERMS
 
 
 def _bf16_dev(a):
@@ -52,7 +63,9 @@ def run_block(inp, k, eps=1e-5, T_max=None):
     return out
 
 
-def check(inp, k, eps=1e-5, rows=None, label="", acc_mean_rel=ACC_MEAN_REL):
+def check(inp, k, eps=1e-5, rows=None, label="", acc_mean_rel="auto"):
+    if acc_mean_rel == "auto":
+        acc_mean_rel = acc_bound(inp["x"].shape[0])
     g = run_block(inp, k, eps)
     if rows is None:
         ref = oracle.moe_forward(inp, k, eps)
@@ -60,7 +73,6 @@ def check(inp, k, eps=1e-5, rows=None, label="", acc_mean_rel=ACC_MEAN_REL):
     else:
         ref = oracle.moe_forward(inp, k, eps, x=inp["x"][rows])
         res = compare_block(g["y"][rows], g["idx"][rows], g["w"][rows], ref, k, inp["router_w"].shape[0])
-    # the fp32 accumulator before the bf16 cast: fp16 activations leave ~2e-4 of mean relative error
     if rows is None:
         acc = compare_block(g["yacc"], g["idx"], g["w"], ref, k, inp["router_w"].shape[0])
     else:
@@ -193,12 +205,13 @@ def test_group_stage_invariants(T, E, k):
     # pair_row inverts the permutation
     assert np.array_equal(np.sort(pair_row), np.arange(P))
     assert np.array_equal(row_token[pair_row], np.repeat(np.arange(T), k))
-    # the expert-sorted B operand is exactly the two-term E4M3 encoding of xn16 * rho of each row's token
+    # the expert-sorted B operand is exactly the three-term E4M3 encoding of xn16 * rho of each row's token
     v = (xn16[row_token].astype(np.float32) * rho[row_token][:, None]).astype(np.float32)
-    hi, lo, s_hi, s_lo = encode_two_term(v)
+    hi, lo, lo2, s_hi, s_lo = encode_three_term(v)
     d = v.shape[1]
     _assert_same_e4m3(xq[0, :P, :d], hi, "hi")
     _assert_same_e4m3(xq[1, :P, :d], lo, "lo")
+    _assert_same_e4m3(xq[2, :P, :d], lo2, "lo2")
     assert not xq[:, :P, d:].any()                        # K padding to a multiple of 128
     assert np.array_equal(scale_bytes_from_words(xsf, 0, np.arange(P), d // 32), s_hi)
     assert np.array_equal(scale_bytes_from_words(xsf, 1, np.arange(P), d // 32), s_lo)
@@ -245,35 +258,83 @@ def test_shapes(shape):
     check(custom_layer(**shape, k=k, seed=sum(shape.values())), k, label=str(shape))
 
 
-def test_scale_extremes():
-    """E8M0 exponents far from 127, outside the layers' distribution.
-
-    Exponents 100..136 on every weight; then huge W2 (140..150) behind normal W13, and tiny W13
-    (104..110).  The block scales reach the tensor core unchanged, so extreme exponents cost no
-    precision in the weights; the activations, though, carry 2^-9 relative rounding (two E4M3
-    terms), and with 36 binades of weight scales the few largest blocks dominate sums that partly
-    cancel.  A float64 emulation of the same rounding points gives max 0.068 / mean 0.0028 relative
-    error for the first case, so the max bound here is 0.1 and the accumulator bound is skipped;
-    the indices and the 5e-3 mean bound still hold.  (Huge W13 is left out: it scales the gate
-    pre-activations to ~1e7, where the clamped SwiGLU is a step function of them and any rounding
-    of the activations moves outputs across the step.)"""
-    def loose(inp, label):
-        g = run_block(inp, 2)
-        ref = oracle.moe_forward(inp, 2, 1e-5)
-        res = compare_block(g["y"], g["idx"], g["w"], ref, 2, inp["router_w"].shape[0])
-        print(label, res)
-        assert res["idx_mismatch"] == 0 and res["w_max_err"] < 1e-5, res
-        assert res["max_rel"] <= 0.1 and res["mean_rel"] <= 5e-3, res
-        g["ctx"].close()
-
-    loose(custom_layer(T=24, d=256, F=256, E=4, k=2, seed=5, scale_lo=100, scale_hi=136), "scales 100..136")
+@pytest.mark.parametrize("T", [24, 200])
+def test_scale_extremes(T):
+    """E8M0 exponents far from 127, outside the layers' distribution, at the block's stated
+    tolerances: exponents 100..136 on every weight; then huge W2 (140..150) behind normal W13, and
+    tiny W13 (104..110).  The block scales reach the tensor core unchanged, so extreme exponents
+    cost no precision in the weights.  With weights this large the activations need more than
+    bf16's 8 bits: decode-sized batches (T = 24) always carry three E4M3 terms, and larger ones
+    (T = 200) add the third term on the work items whose weight bytes reach 126."""
+    loose_w = custom_layer(T=T, d=256, F=256, E=4, k=2, seed=5, scale_lo=100, scale_hi=136)
+    check(loose_w, 2, label="scales 100..136")
     rng = np.random.default_rng(7)
-    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=6)
+    inp = custom_layer(T=T, d=256, F=256, E=4, k=2, seed=6)
     inp["w2_scales"] = rng.integers(140, 151, size=inp["w2_scales"].shape, dtype=np.uint8)
     check(inp, 2, label="W2 scales 140..150")
-    inp = custom_layer(T=24, d=256, F=256, E=4, k=2, seed=8)
+    inp = custom_layer(T=T, d=256, F=256, E=4, k=2, seed=8)
     inp["w13_scales"] = rng.integers(104, 111, size=inp["w13_scales"].shape, dtype=np.uint8)
     check(inp, 2, label="W13 scales 104..110")
+
+
+@pytest.mark.parametrize("T", [24, 200])
+def test_mixed_weight_scales_in_one_launch(T):
+    """Experts 0 and 2 with E8M0 bytes 100..136, experts 1 and 3 with the layers' 120..122: in large
+    batches the work items of one launch then take one or two passes over K."""
+    inp = custom_layer(T=T, d=320, F=192, E=4, k=2, seed=31)
+    wide = custom_layer(T=T, d=320, F=192, E=4, k=2, seed=32, scale_lo=100, scale_hi=136)
+    for e in (0, 2):
+        inp["w13_scales"][e] = wide["w13_scales"][e]
+        inp["w2_scales"][e] = wide["w2_scales"][e]
+    check(inp, 2, label="mixed scales T=%d" % T)
+
+
+def swiglu_edge_tokens(inp, k, eps=1e-5):
+    """Tokens whose block output is not determined at the activations' precision (huge W13).
+
+    A token is flagged when, for any of its k experts, a gate pre-activation z lies in
+    (-64 - D, 7 + D) or a linear one in (-7 - D, 7 + D), with D = 2^-10 * sum_j |W_rj xn_j| (oracle
+    values).  D bounds the change of z when every normalised activation is rounded to 11
+    significant bits and then split into three E4M3 terms.  Outside those intervals the clamped
+    SwiGLU is flat in z: min(z, 7) = 7 above 7, g * sigmoid(1.702 g) is below 1e-45 under -64, and
+    clamp(z, -7, 7) is constant outside [-7, 7]."""
+    xn = oracle.rmsnorm(inp["x"], inp["norm_scale"], eps)
+    idx, _ = oracle.topk_softmax(oracle.router(xn, inp["router_w"], inp["router_b"]), k)
+    E = inp["router_w"].shape[0]
+    F = inp["w13_codes"].shape[1] // 2
+    flagged = np.zeros(xn.shape[0], dtype=bool)
+    for e in range(E):
+        t = np.nonzero((idx == e).any(axis=1))[0]
+        if t.size == 0:
+            continue
+        W = oracle.decode_matrix(inp["w13_codes"][e], inp["w13_scales"][e])
+        z = xn[t] @ W.T + bf16_bits_to_f32(inp["b13"][e]).astype(np.float64)
+        D = 2.0 ** -10 * (np.abs(xn[t]) @ np.abs(W).T)
+        g, u, Dg, Du = z[:, :F], z[:, F:], D[:, :F], D[:, F:]
+        edge = ((g > -64 - Dg) & (g < 7 + Dg)).any(axis=1) | ((u > -7 - Du) & (u < 7 + Du)).any(axis=1)
+        flagged[t[edge]] = True
+    return flagged
+
+
+@pytest.mark.parametrize("T", [48, 96])
+def test_huge_w13_outside_the_swiglu_edges(T):
+    """W13 E8M0 bytes 140..146 (weights up to 6 * 2^19): pre-activations reach ~1e6, where the
+    clamped SwiGLU is a step function of them.  Tokens flagged by swiglu_edge_tokens are left out
+    and counted (as tokens with a 4th/5th logit gap below 1e-4 are); every other token must meet
+    the block's stated tolerances."""
+    inp = custom_layer(T=T, d=128, F=64, E=4, k=1, seed=40 + T)
+    inp["w13_scales"] = np.random.default_rng(41).integers(140, 147, size=inp["w13_scales"].shape, dtype=np.uint8)
+    edge = swiglu_edge_tokens(inp, 1)
+    keep = ~edge
+    print("huge W13: %d of %d tokens at a SwiGLU edge" % (edge.sum(), T))
+    assert keep.sum() >= T // 2
+    g = run_block(inp, 1)
+    ref = oracle.moe_forward(inp, 1, 1e-5)
+    sub = {k_: v[keep] for k_, v in ref.items()}
+    res = compare_block(g["y"][keep], g["idx"][keep], g["w"][keep], sub, 1, 4)
+    print(res)
+    assert res["ok"], res
+    g["ctx"].close()
 
 
 def _np_swiglu(gate, lin):
@@ -286,7 +347,7 @@ def _np_swiglu(gate, lin):
                                          (24, 256, 320, 32, 4)])
 def test_up_stage_h_encoding(T, d, F, E, k):
     """The gate/up GEMM + SwiGLU epilogue against float64 on the same (decoded) operands: h, read back
-    from its two-term E4M3 encoding, within the encoding's rounding of the float64 value (2^-9 of the
+    from its three E4M3 terms, within the encoding's rounding of the float64 value (2^-12 of the
     32-block maximum, plus the fp32 accumulation)."""
     inp = custom_layer(T=T, d=d, F=F, E=E, k=k, seed=T + d)
     w = moe.MoEWeights.from_numpy(inp)
@@ -305,10 +366,13 @@ def test_up_stage_h_encoding(T, d, F, E, k):
     hq = m.workspace("h", T).cpu().numpy()
     hsf = m.workspace("hsf", T).cpu().numpy()
     rows = np.arange(P)
-    xb = decode_two_term(xq[0, :P, :d], xq[1, :P, :d], scale_bytes_from_words(xsf, 0, rows, d // 32),
-                         scale_bytes_from_words(xsf, 1, rows, d // 32))
-    h = decode_two_term(hq[0, :P, :F], hq[1, :P, :F], scale_bytes_from_words(hsf, 0, rows, F // 32),
-                        scale_bytes_from_words(hsf, 1, rows, F // 32))
+    # the terms the gate/up GEMM used: three in decode-sized batches, two otherwise (these
+    # weights' E8M0 bytes stay below 126)
+    nt = 3 if T <= 64 else 2
+    xb = decode_terms([xq[i, :P, :d] for i in range(nt)], scale_bytes_from_words(xsf, 0, rows, d // 32),
+                      scale_bytes_from_words(xsf, 1, rows, d // 32))
+    h = decode_terms([hq[i, :P, :F] for i in range(3)], scale_bytes_from_words(hsf, 0, rows, F // 32),
+                     scale_bytes_from_words(hsf, 1, rows, F // 32))
     W13 = oracle.decode_matrix(inp["w13_codes"].reshape(-1, d // 2), inp["w13_scales"].reshape(-1, d // 32))
     W13 = W13.reshape(E, 2 * F, d)
     b13 = bf16_bits_to_f32(inp["b13"]).astype(np.float64)
@@ -319,7 +383,8 @@ def test_up_stage_h_encoding(T, d, F, E, k):
         want[r] = _np_swiglu(z[:, :F], z[:, F:])
     blk_max = np.abs(want).reshape(P, F // 32, 32).max(axis=2, keepdims=True)
     err = np.abs(h - want).reshape(P, F // 32, 32)
-    bound = 2.0 ** -8 * blk_max + 1e-5 * np.abs(want).max()
+    # three terms keep h to 2^-12 of its block maximum (plus the fp32 accumulation of z)
+    bound = 2.0 ** -11 * blk_max + 1e-5 * np.abs(want).max()
     print("h max err / block max", float(np.max(err / np.maximum(blk_max, 1e-30))))
     assert np.all(err <= bound)
     m.close()
