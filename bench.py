@@ -305,7 +305,7 @@ def algorithmic_counts(cfg, counts):
     w13_expert = 2 * F * (d // 2) + 2 * F * (d // 32) + 2 * F * 2
     w2_expert = d * (F // 2) + d * (F // 32) + d * 2
     pairs = T * k
-    bytes_up = touched * w13_expert + T * d * 2 + pairs * F * 2          # weights, xn16 in, h out
+    bytes_up = touched * w13_expert + T * d * 2 + pairs * F * 2          # weights, xn in, h out
     bytes_down = touched * w2_expert + pairs * F * 2 + pairs * d * 4      # weights, h in, weighted rows out
     flops_up = pairs * 2 * (2 * F) * d
     flops_down = pairs * 2 * d * F

@@ -139,8 +139,7 @@ MOE_API int moe_finalize(moe_ctx_t *ctx, int T, int top_k, const uint16_t *x, ui
 
 /* Workspace buffers readable through moe_copy_workspace. */
 enum {
-    MOE_WS_XN16 = 0,     /* fp16 [T, d]   xn / rho_t                              */
-    MOE_WS_RHO = 1,      /* fp32 [T]      per-token power of two rho_t            */
+    MOE_WS_XN = 0,       /* fp32 [T, d]   normalised tokens xn (the experts' input) */
     MOE_WS_TOPK_IDX = 2, /* int32 [T, k]                                         */
     MOE_WS_TOPK_W = 3,   /* fp32 [T, k]                                          */
     MOE_WS_COUNTS = 4,   /* int32 [E]     tokens routed to each expert            */

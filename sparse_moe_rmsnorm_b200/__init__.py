@@ -31,7 +31,7 @@ MOE_NOALLOC_MAX_TOKENS = 64
 MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_NOMEM = 0, -1, -2, -3, -4, -5
 
 # workspace buffer ids of moe_copy_workspace
-WS = dict(xn16=0, rho=1, topk_idx=2, topk_w=3, counts=4, offsets=5, row_token=6, row_w=7, h=8, out_rows=9, tiles=10,
+WS = dict(xn=0, topk_idx=2, topk_w=3, counts=4, offsets=5, row_token=6, row_w=7, h=8, out_rows=9, tiles=10,
           pair_row=11, xperm=12, xsf=13, hsf=14)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -328,7 +328,7 @@ class MoE:
         Kd = (s.d_model + 127) // 128 * 128
         Kf = (s.d_ff + 127) // 128 * 128
         spec = {
-            "xn16": ((T, s.d_model), torch.float16), "rho": ((T,), torch.float32),
+            "xn": ((T, s.d_model), torch.float32),
             "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
             "counts": ((s.n_experts,), torch.int32), "offsets": ((s.n_experts + 1,), torch.int32),
             "row_token": ((P,), torch.int32), "row_w": ((P,), torch.float32),

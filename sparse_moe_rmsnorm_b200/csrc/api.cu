@@ -42,8 +42,7 @@ struct moe_ctx {
     void *ws;
     size_t ws_bytes;
     int Kd, Kf;             // d_model and d_ff rounded up to 128
-    __half *xn16;
-    float *rho;
+    float *xn;              // fp32 [T_max, d] normalised tokens
     int *topk_idx;
     float *topk_w;
     float *logits;          // fp32 [T_max, E] router logits (decode-sized route path)
@@ -80,8 +79,7 @@ Buf ws_buffer(moe_ctx *c, int which) {
     const moe_shape_t &s = c->shape;
     const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
     switch (which) {
-        case MOE_WS_XN16: return {c->xn16, T * s.d_model * 2};
-        case MOE_WS_RHO: return {c->rho, T * 4};
+        case MOE_WS_XN: return {c->xn, T * s.d_model * 4};
         case MOE_WS_TOPK_IDX: return {c->topk_idx, P * 4};
         case MOE_WS_TOPK_W: return {c->topk_w, P * 4};
         case MOE_WS_COUNTS: return {c->counts, E * 4};
@@ -210,12 +208,12 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
     c->Kd = round_up_128(s.d_model);
     c->Kf = round_up_128(s.d_ff);
     const size_t T = (size_t)s.T_max, P = T * s.top_k, E = s.n_experts;
-    const size_t sizes[] = {T * s.d_model * 2, T * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
+    const size_t sizes[] = {T * s.d_model * 4, P * 4, P * 4, E * 4, (E + 1) * 4, (E + 1) * 4,
                             P * 4, P * 4, P * 4,
                             3 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
                             3 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
                             P * s.d_model * 4, 64, T * E * 4, T * 4};
-    void **slots[] = {(void **)&c->xn16, (void **)&c->rho, (void **)&c->topk_idx, (void **)&c->topk_w,
+    void **slots[] = {(void **)&c->xn, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
                       (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xq, (void **)&c->xsf,
                       (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err,
@@ -266,8 +264,7 @@ int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale
     p.E = c->shape.n_experts;
     p.k = top_k;
     p.eps = c->shape.eps;
-    p.xn16 = c->xn16;
-    p.rho = c->rho;
+    p.xn = c->xn;
     p.topk_idx = c->topk_idx;
     p.topk_w = c->topk_w;
     p.logits = c->logits;
@@ -295,8 +292,7 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     p.row_w = c->row_w;
     p.pair_row = c->pair_row;
     p.err = c->err;
-    p.xn16 = c->xn16;
-    p.rho = c->rho;
+    p.xn = c->xn;
     p.xq = c->xq;
     p.xsf = c->xsf;
     p.P_max = c->shape.T_max * c->shape.top_k;

@@ -44,8 +44,7 @@ struct RouteParams {
     const float *router_b;      // fp32 [E]
     int T, d, E, k;
     float eps;
-    __half *xn16;               // fp16 [T, d] = xn / rho
-    float *rho;                 // fp32 [T]
+    float *xn;                  // fp32 [T, d] normalised tokens
     int *topk_idx;              // [T, k]
     float *topk_w;              // [T, k]
     float *logits;              // fp32 [T, E] (decode-sized path: the CTAs' share of each token's logits)
@@ -66,8 +65,7 @@ struct GroupParams {
     int *pair_row;              // [P] expert-sorted row of pair (token, slot)
     unsigned int *err;
     // the expert-sorted E4M3 terms of the normalised tokens (gate/up B operand)
-    const __half *xn16;         // fp16 [T, d]
-    const float *rho;           // [T]
+    const float *xn;            // fp32 [T, d]
     uint8_t *xq;                // [3][P_max][Kd]: hi, lo, lo2 planes
     uint32_t *xsf;              // [Kd/128][2][P_max]: scales of the hi (also lo2) and lo planes
     int P_max, d, Kd;

@@ -127,7 +127,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     // carve the scratch; reject shapes that do not fit
     const size_t P = (size_t)T * k;
     const int Kd = round_up_128(d), Kf = round_up_128(F);
-    const size_t sizes[] = {(size_t)T * d * 2, (size_t)T * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
+    const size_t sizes[] = {(size_t)T * d * 4, P * 4, P * 4, (size_t)E * 4, (size_t)(E + 1) * 4,
                             (size_t)(E + 1) * 4, P * 4, P * 4, P * 4,
                             3 * P * Kd, (size_t)(Kd / 128) * 2 * P * 4, 3 * P * Kf, (size_t)(Kf / 128) * 2 * P * 4,
                             P * d * 4, 64, (size_t)T * E * 4, (size_t)T * 4};
@@ -144,24 +144,23 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
         ptrs[i] = base;
         base += r256(sizes[i]);
     }
-    __half *xn16 = reinterpret_cast<__half *>(ptrs[0]);
-    float *rho = reinterpret_cast<float *>(ptrs[1]);
-    int *topk_idx = reinterpret_cast<int *>(ptrs[2]);
-    float *topk_w = reinterpret_cast<float *>(ptrs[3]);
-    int *counts = reinterpret_cast<int *>(ptrs[4]);
-    int *offsets = reinterpret_cast<int *>(ptrs[5]);
-    int *tiles = reinterpret_cast<int *>(ptrs[6]);
-    int *row_token = reinterpret_cast<int *>(ptrs[7]);
-    float *row_w = reinterpret_cast<float *>(ptrs[8]);
-    int *pair_row = reinterpret_cast<int *>(ptrs[9]);
-    uint8_t *xq = reinterpret_cast<uint8_t *>(ptrs[10]);
-    uint32_t *xsf = reinterpret_cast<uint32_t *>(ptrs[11]);
-    uint8_t *hq = reinterpret_cast<uint8_t *>(ptrs[12]);
-    uint32_t *hsf = reinterpret_cast<uint32_t *>(ptrs[13]);
-    float *orows = reinterpret_cast<float *>(ptrs[14]);
-    unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[15]);
-    float *logits = reinterpret_cast<float *>(ptrs[16]);
-    unsigned int *tok_done = reinterpret_cast<unsigned int *>(ptrs[17]);
+    float *xn = reinterpret_cast<float *>(ptrs[0]);
+    int *topk_idx = reinterpret_cast<int *>(ptrs[1]);
+    float *topk_w = reinterpret_cast<float *>(ptrs[2]);
+    int *counts = reinterpret_cast<int *>(ptrs[3]);
+    int *offsets = reinterpret_cast<int *>(ptrs[4]);
+    int *tiles = reinterpret_cast<int *>(ptrs[5]);
+    int *row_token = reinterpret_cast<int *>(ptrs[6]);
+    float *row_w = reinterpret_cast<float *>(ptrs[7]);
+    int *pair_row = reinterpret_cast<int *>(ptrs[8]);
+    uint8_t *xq = reinterpret_cast<uint8_t *>(ptrs[9]);
+    uint32_t *xsf = reinterpret_cast<uint32_t *>(ptrs[10]);
+    uint8_t *hq = reinterpret_cast<uint8_t *>(ptrs[11]);
+    uint32_t *hsf = reinterpret_cast<uint32_t *>(ptrs[12]);
+    float *orows = reinterpret_cast<float *>(ptrs[13]);
+    unsigned int *err = reinterpret_cast<unsigned int *>(ptrs[14]);
+    float *logits = reinterpret_cast<float *>(ptrs[15]);
+    unsigned int *tok_done = reinterpret_cast<unsigned int *>(ptrs[16]);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nb = token_block_rows(T);
@@ -184,8 +183,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     rp.E = E;
     rp.k = k;
     rp.eps = eps;
-    rp.xn16 = xn16;
-    rp.rho = rho;
+    rp.xn = xn;
     rp.topk_idx = topk_idx;
     rp.topk_w = topk_w;
     rp.logits = logits;
@@ -208,8 +206,7 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.row_w = row_w;
     gp.pair_row = pair_row;
     gp.err = err;
-    gp.xn16 = xn16;
-    gp.rho = rho;
+    gp.xn = xn;
     gp.xq = xq;
     gp.xsf = xsf;
     gp.P_max = (int)P;

@@ -44,9 +44,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
 //
 // One CTA per TB tokens, NW warps; NW / TB warps share each token.
 //   xn = x / sqrt(mean(x^2) + eps) * scale in fp32 ("gpt-oss-20B" hub page,
-//   section 3.2), kept in shared memory for the router; rho = a power of two
-//   with max|xn| / rho in [2^13, 2^14), and xn / rho stored as fp16 (an exact
-//   rescaling, so fp16's range never clips a token).
+//   section 3.2), kept in shared memory for the router and stored (fp32) for
+//   the experts.
 // Router: logit_e = W_r[e] . xn + b_e in fp32 ("gpt-oss-20B" page, 3.4).
 //   Warp w owns experts w, w+NW, ... (at most EPW); the loop runs over
 //   VEC-element chunks of d, holding the TB tokens' chunk in registers while
@@ -180,44 +179,15 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
 #pragma unroll
     for (int i = 0; i < WPT; ++i) tot += red[ti * WPT + i];
     const float inv_rms = 1.0f / sqrtf(tot / (float)d + p.eps);
-    float amax = 0.f;
     if (has_tok) {
+        float *xo = p.xn + (size_t)t * d;
         for (int j = u * 8; j < d; j += WPT * 256) {
             float sc[8];
             bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p.norm_scale + j), sc);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float v = xsr[j + c] * inv_rms * sc[c];
-                xsr[j + c] = v;
-                amax = fmaxf(amax, fabsf(v));
-            }
-        }
-    }
-    amax = warp_max(amax);
-    __syncthreads();
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < WPT; ++i) amax = fmaxf(amax, red[ti * WPT + i]);
-    if (has_tok) {
-        float rho = 1.f, inv_rho = 1.f;
-        if (amax > 0.f && amax <= FLT_MAX) {
-            int ex;
-            frexpf(amax, &ex);          // amax in [2^(ex-1), 2^ex)
-            rho = exp2i(ex - 14);
-            inv_rho = exp2i(14 - ex);
-        }
-        if (u == 0) p.rho[t] = rho;
-        __half *xo = p.xn16 + (size_t)t * d;
-        for (int j = u * 8; j < d; j += WPT * 256) {
-            uint32_t hw[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const __half2 h2 = __floats2half2_rn(xsr[j + 2 * c] * inv_rho, xsr[j + 2 * c + 1] * inv_rho);
-                hw[c] = *reinterpret_cast<const uint32_t *>(&h2);
-            }
-            *reinterpret_cast<uint4 *>(xo + j) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            for (int c = 0; c < 8; ++c) xsr[j + c] = xsr[j + c] * inv_rms * sc[c];
+            reinterpret_cast<float4 *>(xo + j)[0] = make_float4(xsr[j], xsr[j + 1], xsr[j + 2], xsr[j + 3]);
+            reinterpret_cast<float4 *>(xo + j)[1] = make_float4(xsr[j + 4], xsr[j + 5], xsr[j + 6], xsr[j + 7]);
         }
     }
     __syncthreads();
@@ -282,7 +252,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
 // else (the loads overlap the RMSNorm), every CTA normalises its token
 // (RMSNorm as above, the same fp32 arithmetic), each warp writes one fp32
 // logit, and the last CTA of the token to finish (a per-token counter, reset
-// by that CTA) takes the top-k and the softmax.  CTA y = 0 writes xn16 / rho.
+// by that CTA) takes the top-k and the softmax.  CTA y = 0 writes xn.
 constexpr int ROUTE_SMALL_CHUNKS = 12;   // 8-element chunks of a router row per lane: d <= 3072
 
 __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
@@ -325,7 +295,6 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) tot += red[i];
     const float inv_rms = 1.0f / sqrtf(tot / (float)d + p.eps);
-    float amax = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int c = threadIdx.x + 512 * h;
@@ -335,37 +304,11 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
                 const float v = f[h][k] * inv_rms * sc[h][k];
                 f[h][k] = v;
                 xs[8 * c + k] = v;
-                amax = fmaxf(amax, fabsf(v));
             }
-        }
-    }
-    if (blockIdx.y == 0) {
-        amax = warp_max(amax);
-        __syncthreads();                     // every thread has read red[] above
-        if (lane == 0) red[warp] = amax;
-        __syncthreads();
-        amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, red[i]);
-        float rho = 1.f, inv_rho = 1.f;
-        if (amax > 0.f && amax <= FLT_MAX) {
-            int ex;
-            frexpf(amax, &ex);               // amax in [2^(ex-1), 2^ex)
-            rho = exp2i(ex - 14);
-            inv_rho = exp2i(14 - ex);
-        }
-        if (threadIdx.x == 0) p.rho[t] = rho;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = threadIdx.x + 512 * h;
-            if (c < nch) {
-                uint32_t hw[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const __half2 h2 = __floats2half2_rn(f[h][2 * k] * inv_rho, f[h][2 * k + 1] * inv_rho);
-                    hw[k] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                reinterpret_cast<uint4 *>(p.xn16 + (size_t)t * d)[c] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            if (blockIdx.y == 0) {
+                float4 *xo = reinterpret_cast<float4 *>(p.xn + (size_t)t * d + 8 * c);
+                xo[0] = make_float4(f[h][0], f[h][1], f[h][2], f[h][3]);
+                xo[1] = make_float4(f[h][4], f[h][5], f[h][6], f[h][7]);
             }
         }
     }
@@ -440,7 +383,7 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
 // accumulate each token's sum of squares and max |x_j scale_j|; one warp
 // issues the MMAs; then four warps read the logits from TMEM (lane = token),
 // scale by 1/rms, add the bias and take the top-k (ties to the lower index,
-// NaN below every number) and the softmax in registers; last, xn16 = xn / rho
+// NaN below every number) and the softmax in registers; last, xn
 // from a second read of the CTA's rows.
 constexpr int RT_TOK = 128;
 constexpr int RT_KC = 64;
@@ -704,22 +647,11 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RoutePara
             }
         }
     }
-    // xn16 = xn / rho, rho a power of two with max|xn| / rho in [2^13, 2^14); the
-    // per-row factors first, then every (row, 8-element chunk) with loads in flight
+    // xn = x * (1/rms) * scale in fp32: the per-row factors first, then every (row,
+    // 8-element chunk) with loads in flight
     if (threadIdx.x < RT_TOK) {
         const int row = threadIdx.x;
-        const float r = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);
-        const float amax = mx_s[row] * r;
-        float rho = 1.f, inv_rho = 1.f;
-        if (amax > 0.f && amax <= FLT_MAX) {
-            int ex;
-            frexpf(amax, &ex);                     // amax in [2^(ex-1), 2^ex)
-            rho = exp2i(ex - 14);
-            inv_rho = exp2i(14 - ex);
-        }
-        if (row < ntok) p.rho[t0 + row] = rho;
-        ss_s[row] = r;                             // reused: 1/rms
-        mx_s[row] = inv_rho;                       // reused: 1/rho
+        ss_s[row] = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);   // reused: 1/rms
     }
     __syncthreads();
     {
@@ -728,17 +660,13 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RoutePara
 #pragma unroll 2
         for (int i = threadIdx.x; i < total; i += RT_THREADS) {
             const int row = i / nch, cc = i - row * nch;
-            const float r = ss_s[row], ir = mx_s[row];
+            const float r = ss_s[row];
             float f[8], sc[8];
             bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + row) * d) + cc), f);
             bf16x8_to_f32(reinterpret_cast<const uint4 *>(sc_s)[cc], sc);
-            uint32_t hw[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const __half2 h2 = __floats2half2_rn(f[2 * q] * r * sc[2 * q] * ir, f[2 * q + 1] * r * sc[2 * q + 1] * ir);
-                hw[q] = *reinterpret_cast<const uint32_t *>(&h2);
-            }
-            reinterpret_cast<uint4 *>(p.xn16 + (size_t)(t0 + row) * d)[cc] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            float4 *xo = reinterpret_cast<float4 *>(p.xn + (size_t)(t0 + row) * d + 8 * cc);
+            xo[0] = make_float4(f[0] * r * sc[0], f[1] * r * sc[1], f[2] * r * sc[2], f[3] * r * sc[3]);
+            xo[1] = make_float4(f[4] * r * sc[4], f[5] * r * sc[5], f[6] * r * sc[6], f[7] * r * sc[7]);
         }
     }
     tc_fence_before();
@@ -761,8 +689,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RoutePara
 // row_token / row_w / pair_row entries and their B operand row (below).  CTA 0
 // writes counts, offsets and tiles.
 //
-// B operand row r: the normalised activations of token row_token[r],
-// v = xn16 * rho, as three E4M3 terms per 32-element block with E8M0 scale s
+// B operand row r: the normalised activations v = xn (fp32) of token
+// row_token[r], as three E4M3 terms per 32-element block with E8M0 scale s
 // (the exponent that fits the block maximum to 448):
 //   hi = e4m3(v / 2^s),  lo = e4m3((v - hi 2^s) / 2^(s-4)),
 //   lo2 = e4m3((v - hi 2^s - lo 2^(s-4)) / 2^s)
@@ -775,8 +703,7 @@ constexpr int GROUP_ROWS_MAX = 1024;   // expert-sorted rows per CTA, at most
 
 // Blocks b0 + lane (lane < 32) of expert-sorted row r, token tok.
 __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int tok, int b0, int lane) {
-    const float sc = p.rho[tok];
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.xn16 + (size_t)tok * p.d);
+    const float4 *src = reinterpret_cast<const float4 *>(p.xn + (size_t)tok * p.d);
     const int nblk = p.d / 32, nblk_pad = p.Kd / 32;
     {
         const int b = b0 + lane;
@@ -786,14 +713,12 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
         if (b < nblk) {
             float v[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 u = src[4 * b + i];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t wk = k == 0 ? u.x : (k == 1 ? u.y : (k == 2 ? u.z : u.w));
-                    v[8 * i + 2 * k] = __half2float(__ushort_as_half((unsigned short)(wk & 0xFFFFu))) * sc;
-                    v[8 * i + 2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(wk >> 16))) * sc;
-                }
+            for (int i = 0; i < 8; ++i) {
+                const float4 u = src[8 * b + i];
+                v[4 * i] = u.x;
+                v[4 * i + 1] = u.y;
+                v[4 * i + 2] = u.z;
+                v[4 * i + 3] = u.w;
             }
             float amax = 0.f;
 #pragma unroll

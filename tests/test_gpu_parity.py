@@ -163,20 +163,15 @@ def test_route_stage(T, d, E, k):
     moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
     idx = m.workspace("topk_idx", T).cpu().numpy()
     wts = m.workspace("topk_w", T).cpu().numpy()
-    xn16 = m.workspace("xn16", T).float().cpu().numpy().astype(np.float64)
-    rho = m.workspace("rho", T).cpu().numpy().astype(np.float64)
+    xn_gpu = m.workspace("xn", T).cpu().numpy().astype(np.float64)
     xn = oracle.rmsnorm(inp["x"], inp["norm_scale"], 1e-5)
     logits = oracle.router(xn, inp["router_w"], inp["router_b"])
     ref_idx, ref_w = oracle.topk_softmax(logits, k)
     keep = ~excluded_tokens(logits, k)
     assert np.array_equal(idx[keep], ref_idx[keep])
     assert np.max(np.abs(wts[keep] - ref_w[keep])) < 1e-5
-    # rho is a power of two with max|xn|/rho in [2^13, 2^14)
-    m2, e2 = np.frexp(rho)
-    assert np.all(m2 == 0.5)
-    amax = np.abs(xn16).max(axis=1)
-    assert np.all((amax >= 2.0 ** 13 * (1 - 2 ** -10)) & (amax <= 2.0 ** 14))
-    assert np.max(np.abs(xn16 * rho[:, None] - xn) / np.abs(xn).max(axis=1, keepdims=True)) < 6e-4
+    # the normalised tokens in fp32: a few fp32 roundings from the float64 RMSNorm
+    assert np.max(np.abs(xn_gpu - xn) / np.abs(xn).max(axis=1, keepdims=True)) < 2e-6
     m.close()
 
 
@@ -196,8 +191,7 @@ def test_group_stage_invariants(T, E, k):
     row_token = m.workspace("row_token", T).cpu().numpy()
     row_w = m.workspace("row_w", T).cpu().numpy()
     pair_row = m.workspace("pair_row", T).cpu().numpy()
-    xn16 = m.workspace("xn16", T).cpu().numpy()
-    rho = m.workspace("rho", T).cpu().numpy()
+    xn_gpu = m.workspace("xn", T).cpu().numpy()
     xq = m.workspace("xperm", T).cpu().numpy()
     xsf = m.workspace("xsf", T).cpu().numpy()
     P = T * k
@@ -205,8 +199,8 @@ def test_group_stage_invariants(T, E, k):
     # pair_row inverts the permutation
     assert np.array_equal(np.sort(pair_row), np.arange(P))
     assert np.array_equal(row_token[pair_row], np.repeat(np.arange(T), k))
-    # the expert-sorted B operand is exactly the three-term E4M3 encoding of xn16 * rho of each row's token
-    v = (xn16[row_token].astype(np.float32) * rho[row_token][:, None]).astype(np.float32)
+    # the expert-sorted B operand is exactly the three-term E4M3 encoding of each row's token's xn
+    v = xn_gpu[row_token].astype(np.float32)
     hi, lo, lo2, s_hi, s_lo = encode_three_term(v)
     d = v.shape[1]
     _assert_same_e4m3(xq[0, :P, :d], hi, "hi")
@@ -294,8 +288,8 @@ def swiglu_edge_tokens(inp, k, eps=1e-5):
 
     A token is flagged when, for any of its k experts, a gate pre-activation z lies in
     (-64 - D, 7 + D) or a linear one in (-7 - D, 7 + D), with D = 2^-10 * sum_j |W_rj xn_j| (oracle
-    values).  D bounds the change of z when every normalised activation is rounded to 11
-    significant bits and then split into three E4M3 terms.  Outside those intervals the clamped
+    values).  D bounds, generously, the change of z when every normalised activation is split
+    into three E4M3 terms (about 12 significant bits of each element).  Outside those intervals the clamped
     SwiGLU is flat in z: min(z, 7) = 7 above 7, g * sigmoid(1.702 g) is below 1e-45 under -64, and
     clamp(z, -7, 7) is constant outside [-7, 7]."""
     xn = oracle.rmsnorm(inp["x"], inp["norm_scale"], eps)
