@@ -333,6 +333,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
             }
             const int n_it = n_st * t_pass;
+            // the next item's pass count is published a few stages into this item (its
+            // scale bytes have landed by then, and the ring is full, so the wait costs
+            // nothing), well before the other roles reach the item
+            const int pub_st = min(n_it - 1, 2);
+            int next_pass = 1;
             for (int st = 0; st < n_it; ++st) {
                 const int kst = st < n_st ? st : st - n_st;      // the K stage (the same in both passes)
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
@@ -365,14 +370,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
-            }
-            if (!ok) break;
-            if constexpr (!SFI) {
-                if (has_next) {
-                    t_pass = publish_passes(tn, tn_buf, tn_par);
-                    if (t_pass == 0) { ok = false; break; }
+                if constexpr (!SFI) {
+                    if (has_next && st == pub_st) {
+                        next_pass = publish_passes(tn, tn_buf, tn_par);
+                        if (next_pass == 0) { ok = false; break; }
+                    }
                 }
             }
+            if (!ok) break;
+            t_pass = next_pass;
             t = tn;
         }
         if (!ok) {
@@ -754,6 +760,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
             if (n_mma_warps == 2 && !__all_sync(0xffffffffu, mbar_wait(&d_full[2 + db], dph, wc))) break;
             tc_fence_after();
+            // The accumulator goes back to the MMA warps as soon as this warp has read its
+            // last chunk of it, before the chunk's SwiGLU / stores: with one buffer per MMA
+            // warp (per-item mode) the next item's MMAs then wait only for the TMEM reads.
+            bool released = false;
+            auto release = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&d_empty[db]);
+                released = true;
+            };
+            if (16 * eg >= t.n_mma) release();
             for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
                 float acc[16];
 #pragma unroll
@@ -769,6 +786,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
                     }
                 }
+                if (c0 + 32 >= t.n_mma) release();
                 if (MODE == MODE_UP) {
                     // SwiGLU: lanes < 16 hold gate rows, lanes >= 16 the linear rows of the
                     // same h rows; lanes < 16 finish columns 0..7, lanes >= 16 columns 8..15
@@ -852,9 +870,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
             }
             if (!ok) break;
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (!released) release();
             if (++db == n_dbuf) { db = 0; dph ^= 1; }
         }
     }
