@@ -32,8 +32,10 @@ sys.path.insert(0, ROOT)
 from moe_inputs import CONFIGS, make_config_inputs, make_tokens  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
-# kernels of one moe_forward: route, group + permute, gate/up GEMM, down GEMM, combine
-KERNELS_PER_LAYER = 5
+# kernels of one moe_forward: route, group + permute, gate/up GEMM, down GEMM, combine; large
+# batches add the scan of the W2 scale bytes before the gate/up GEMM
+def kernels_per_layer(T: int) -> int:
+    return 5 if T <= 64 else 6
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / bf16 tensor roofline"
 DESCRIPTIONS = {
     "tiny": "tiny MoE layer: T=16, d_model=d_ff=128, E=8, top-4",
@@ -376,7 +378,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
             moe.moe_group(m.ctx, T, cfg.k)
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             ev[0].record(stream)
-            moe.moe_expert_up(m.ctx, T, cfg.k, w.w13_codes, w.w13_scales, w.b13)
+            moe.moe_expert_up(m.ctx, T, cfg.k, w.w13_codes, w.w13_scales, w.b13, w.w2_scales)
             ev[1].record(stream)
             moe.moe_expert_down(m.ctx, T, cfg.k, w.w2_codes, w.w2_scales, w.b2)
             ev[2].record(stream)
@@ -430,7 +432,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
         evs[1].record(stream)
         moe.moe_group(m.ctx, T, cfg.k)
         evs[2].record(stream)
-        moe.moe_expert_up(m.ctx, T, cfg.k, w0.w13_codes, w0.w13_scales, w0.b13)
+        moe.moe_expert_up(m.ctx, T, cfg.k, w0.w13_codes, w0.w13_scales, w0.b13, w0.w2_scales)
         evs[3].record(stream)
         moe.moe_expert_down(m.ctx, T, cfg.k, w0.w2_codes, w0.w2_scales, w0.b2)
         evs[4].record(stream)
@@ -504,7 +506,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "gemm_ms_live": {k_: round(v, 4) for k_, v in gemm_ms.items()},
             "experts_touched": cnt["touched"], "clocks": clocks.summary(), "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": KERNELS_PER_LAYER * layers * args.steps}
+            "gpu_launches": kernels_per_layer(T) * layers * args.steps}
 
 
 EXTRA_WORKLOADS = ("prefill20b", "decode120b", "stack20b")

@@ -118,20 +118,25 @@ MOE_API int moe_forward(moe_ctx_t *ctx, int T,
  *                    of (token, expert) pairs into expert-contiguous rows,
  *                    then the expert-sorted copy of the normalised tokens;
  *   moe_expert_up    gate/up grouped GEMM with the clamped-SwiGLU epilogue;
+ *                    for batches over 64 tokens it first reads both weight
+ *                    tensors' scale bytes (w13_scales, w2_scales) to plan which
+ *                    weight blocks of the two GEMMs take a pass over the third
+ *                    E4M3 activation term (blocks with an E8M0 byte >= 126);
  *   moe_expert_down  down grouped GEMM, each row scaled by its routing weight;
  *   moe_finalize     y = x + the token's weighted expert rows (bf16), in a
  *                    fixed order, so results are reproducible run to run.
  * They exist for per-stage timing and tests; intermediate results stay in the
  * context's workspace (see moe_copy_workspace).  moe_finalize needs the same
- * x that moe_route was given.  moe_expert_down reads the routing arrays before
- * it waits for the kernel before it: call it right after moe_expert_up (a call
+ * x that moe_route was given.  moe_expert_down reads the routing arrays (and,
+ * for batches over 64 tokens, moe_expert_up's pass plan) before it waits for
+ * the kernel before it: call it right after moe_expert_up (a call
  * in another order computes nothing useful, but every row index it uses stays
  * inside the workspace). */
 MOE_API int moe_route(moe_ctx_t *ctx, int T, const uint16_t *x, const uint16_t *norm_scale,
               const uint16_t *router_w, const float *router_b, int top_k, void *stream);
 MOE_API int moe_group(moe_ctx_t *ctx, int T, int top_k, void *stream);
 MOE_API int moe_expert_up(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
-                  const uint16_t *b13, void *stream);
+                  const uint16_t *b13, const uint8_t *w2_scales, void *stream);
 MOE_API int moe_expert_down(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w2_codes, const uint8_t *w2_scales,
                     const uint16_t *b2, void *stream);
 MOE_API int moe_finalize(moe_ctx_t *ctx, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,

@@ -61,7 +61,7 @@ _SIGS = {
                     + [ctypes.c_void_p] * 4),
     "moe_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p]),
     "moe_group": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
-    "moe_expert_up": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
+    "moe_expert_up": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5),
     "moe_expert_down": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
     "moe_finalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5),
     "moe_copy_workspace": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
@@ -154,9 +154,9 @@ def moe_group(ctx, T, top_k, stream=None) -> None:
     _check(lib().moe_group(ctx, int(T), int(top_k), _stream(stream)), "moe_group")
 
 
-def moe_expert_up(ctx, T, top_k, w13_codes, w13_scales, b13, stream=None) -> None:
+def moe_expert_up(ctx, T, top_k, w13_codes, w13_scales, b13, w2_scales, stream=None) -> None:
     _check(lib().moe_expert_up(ctx, int(T), int(top_k), _ptr(w13_codes), _ptr(w13_scales), _ptr(b13),
-                               _stream(stream)), "moe_expert_up")
+                               _ptr(w2_scales), _stream(stream)), "moe_expert_up")
 
 
 def moe_expert_down(ctx, T, top_k, w2_codes, w2_scales, b2, stream=None) -> None:

@@ -21,6 +21,8 @@ cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pai
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
 cudaError_t launch_selftest_wait(unsigned int *err, unsigned long long limit_ns, cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
+cudaError_t launch_pass_plan(const uint8_t *w13_scales, const uint8_t *w2_scales, int E, int d, int F,
+                             uint8_t *up_pass, uint8_t *down_pass, cudaStream_t s);
 }  // namespace moe
 
 using namespace moe;
@@ -56,6 +58,8 @@ struct moe_ctx {
     uint8_t *hq;            // down B: three E4M3 planes [3][P_max][Kf] of h
     uint32_t *hsf;          // [Kf/128][2][P_max]
     float *orows;           // weighted expert output per expert-sorted row
+    uint8_t *up_pass;       // [E][F/64] passes over K of each gate/up weight block (large batches)
+    uint8_t *down_pass;     // [E][DOWN_PASS_STRIDE] ... of each down weight block
     unsigned int *err;
     unsigned long long wait_limit_ns;
     // B tensor maps, one per token-block height (16 * (i + 1) rows), made on first use
@@ -107,7 +111,7 @@ int check_call(moe_ctx *c, int T, int top_k) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
-                const uint16_t *bias, cudaStream_t stream) {
+                const uint16_t *bias, const uint8_t *w2_scales, cudaStream_t stream) {
     const moe_shape_t &s = c->shape;
     GemmParams p;
     memset(&p, 0, sizeof p);
@@ -132,6 +136,15 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
         p.b_sf = c->xsf;
         p.h_q = c->hq;
         p.h_sf = reinterpret_cast<uint8_t *>(c->hsf);
+        // large blocks: the pass table of both GEMMs, from the weights' scale bytes
+        if (!p.stacked) {
+            if (launch_pass_plan(scales, w2_scales, E, d, F, c->up_pass, c->down_pass, stream) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            p.item_pass = c->up_pass;
+            p.item_pass_stride = F / 64;
+            p.down_pass = c->down_pass;
+            p.MB_down = (d + GEMM_BM - 1) / GEMM_BM;
+        }
     } else {
         if (codes != c->w2_ptr) {
             if (p.K_main >= 128 && !encode_a_down(&c->map_w2, codes, E, d, F, p.K_main)) return MOE_ERR_CUDA;
@@ -146,6 +159,10 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
         p.map_b = c->map_hq[bi];
         p.b_sf = c->hsf;
         p.out_rows = c->orows;
+        if (!p.stacked) {                                // written by moe_expert_up's pass plan
+            p.item_pass = c->down_pass;
+            p.item_pass_stride = DOWN_PASS_STRIDE;
+        }
     }
     p.codes = codes;
     p.scales = scales;
@@ -212,12 +229,13 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
                             P * 4, P * 4, P * 4,
                             3 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
                             3 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
-                            P * s.d_model * 4, 64, T * E * 4, T * 4};
+                            P * s.d_model * 4, 64, T * E * 4, T * 4, E * (size_t)(s.d_ff / 64),
+                            E * (size_t)DOWN_PASS_STRIDE};
     void **slots[] = {(void **)&c->xn, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
                       (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xq, (void **)&c->xsf,
                       (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err,
-                      (void **)&c->logits, (void **)&c->tok_done};
+                      (void **)&c->logits, (void **)&c->tok_done, (void **)&c->up_pass, (void **)&c->down_pass};
     size_t total = 0;
     for (size_t v : sizes) total += round256(v);
     if (cudaMalloc(&c->ws, total) != cudaSuccess) {
@@ -302,12 +320,14 @@ int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
-                  const uint16_t *b13, void *stream) {
+                  const uint16_t *b13, const uint8_t *w2_scales, void *stream) {
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!aligned32(w13_codes) || !aligned16(w13_scales) || !aligned16(b13)) return MOE_ERR_ARG;
-    return gemm_launch(c, MODE_UP, T, top_k, w13_codes, w13_scales, b13, static_cast<cudaStream_t>(stream));
+    if (!aligned32(w13_codes) || !aligned16(w13_scales) || !aligned16(b13) || !aligned16(w2_scales))
+        return MOE_ERR_ARG;
+    return gemm_launch(c, MODE_UP, T, top_k, w13_codes, w13_scales, b13, w2_scales,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, const uint8_t *w2_scales,
@@ -316,7 +336,7 @@ int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, con
     if (rc) return rc;
     if (T == 0) return MOE_OK;
     if (!aligned32(w2_codes) || !aligned16(w2_scales) || !aligned16(b2)) return MOE_ERR_ARG;
-    return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, static_cast<cudaStream_t>(stream));
+    return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int moe_finalize(moe_ctx_t *c, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,
@@ -351,7 +371,7 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
     if (y == x) return MOE_ERR_ARG;
     if ((rc = moe_route(c, T, x, norm_scale, router_w, router_b, top_k, stream))) return rc;
     if ((rc = moe_group(c, T, top_k, stream))) return rc;
-    if ((rc = moe_expert_up(c, T, top_k, w13_codes, w13_scales, b13, stream))) return rc;
+    if ((rc = moe_expert_up(c, T, top_k, w13_codes, w13_scales, b13, w2_scales, stream))) return rc;
     if ((rc = moe_expert_down(c, T, top_k, w2_codes, w2_scales, b2, stream))) return rc;
     return moe_finalize(c, T, top_k, x, y, topk_idx_out, topk_w_out, stream);
 }

@@ -43,15 +43,15 @@
 // B (activations), 1 MMA issue, 2 TMEM allocation and (per-item scale factors)
 // the second MMA warp, 4-7 scale-factor warps (one per TMEM lane quarter),
 // 8-11 and 12-15 two epilogue groups taking 16-column chunks in turn.
-// Large blocks: the A producer decides each work item's pass count (one, or
-// two with the lo2 pass) from the item's weight scale bytes, which it stages
-// in shared memory one item ahead, and publishes it to the B producer, the
-// MMA warp and the scale-factor warps through a shared-memory word and an
-// mbarrier.
+// Large blocks: every role reads a work item's pass count (one, or two with the
+// lo2 pass) from a table that pass_plan_kernel writes from the weights' scale
+// bytes before the gate/up GEMM.
 // Producers and MMA run as whole converged warps, one elected lane issuing.
 // Every mbarrier wait is bounded (WaitCtl); when one runs out the CTA stops
 // issuing work, drains its copies and MMAs in flight, frees TMEM and returns
 // with the error latched.
+#include <cuda_bf16.h>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -99,6 +99,12 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n_slots, long lon
                                            unsigned long long limit_ns) {
     for (long long i = n_issued - 1; i >= 0 && i >= n_issued - n_slots; --i)
         mbar_wait_drain(&full[i % n_slots], (uint32_t)((i / n_slots) & 1), limit_ns);
+}
+
+// Passes over K of work item t: 2 (the hi and lo terms, then the lo2 term) where
+// the pass table says so, else 1.
+__device__ __forceinline__ int item_passes(const GemmParams &p, const Work &t) {
+    return p.item_pass ? (int)__ldg(p.item_pass + (size_t)t.e * p.item_pass_stride + t.mb) : 1;
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -154,11 +160,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *f_empty = f_full + 2;
     uint64_t *bw_full = f_empty + 2;        // the item's B scale words are staged (per-item mode)
     uint64_t *bw_empty = bw_full + 1;       // ... and have been read by all four scale-factor warps
-    uint64_t *info_full = bw_empty + 1;     // [2] the pass count of the item using scale buffer i is published
     uint32_t *bw_s = reinterpret_cast<uint32_t *>(smem + plan.bsf_off);   // [stage][4][32]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
-    volatile int *npass_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 8);   // [2] per scale buffer
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
     int *offsets_s = counts_s + (p.E + 1);
     int *tiles_s = offsets_s + (p.E + 1);
@@ -186,10 +190,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            // per-stage mode: the four scale-factor warps, and the B producer and the MMA
-            // warp once they have read the item's pass count
-            mbar_init(&s_empty[i], SFI ? 4 : 6);
-            mbar_init(&info_full[i], 1);
+            mbar_init(&s_empty[i], 4);
             mbar_init(&d_empty[i], 8);    // every epilogue warp
             mbar_init(&drain_bar[i], 1);
             mbar_init(&f_full[i], 4);     // the four scale-factor warps
@@ -235,10 +236,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // ------------------------------------------------- A producer (weights)
         // Per work item (per-stage mode) the 128 rows' E8M0 bytes (one or two
         // untiled bulk copies), issued one item ahead so the scale-factor warps
-        // can prepare an item while the MMAs work on the one before; from them the
-        // item's pass count (a lo2 pass when a byte reaches LO2_SCALE_MIN),
-        // published before the item starts.  Per stage one TMA box of E2M1 codes
-        // (128 rows x 128 K), the item's K stages once per pass.  The K tail (K not
+        // can prepare an item while the MMAs work on the one before.  Per stage one
+        // TMA box of E2M1 codes (128 rows x 128 K), the item's K stages once per
+        // pass.  The K tail (K not
         // a multiple of 128) is loaded at the start of the item, four rows per
         // lane, and written into its stage's slot here.
         if (lane == 0 && n_main > 0) tma_prefetch_desc(&p.map_a);
@@ -246,9 +246,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         uint32_t ph = 0, sph = 0;
         long long issued = 0, s_issued = 0;
         bool ok = true;
-        // scale-buffer index and phase parity of the item loaded last
-        int ld_buf = 0;
-        uint32_t ld_par = 0;
         auto load_scales = [&](const Work &t) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[sb], sph ^ 1, wc))) return false;
             uint8_t *sdst = scale_buf + sb * scale_bytes;
@@ -265,42 +262,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 bulk_load_w(sdst, p.scales + ((size_t)t.e * p.R + m0) * KB32, bytes, &s_full[sb]);
             }
             ++s_issued;
-            ld_buf = sb;
-            ld_par = sph;
             if (++sb == 2) { sb = 0; sph ^= 1; }
             return true;
         };
-        // The pass count of the item whose scale bytes sit in buffer `buf`: the largest
-        // E8M0 byte of its rows, then published for the other roles.  Returns the count
-        // (0 when a wait ran out).
-        auto publish_passes = [&](const Work &t, int buf, uint32_t par) -> int {
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], par, wc))) return 0;
-            const int rows = MODE == MODE_UP ? GEMM_BM : min(GEMM_BM, p.R - t.mb * GEMM_BM);
-            const int n16 = rows * KB32 / 16;
-            const uint4 *src = reinterpret_cast<const uint4 *>(scale_buf + buf * scale_bytes);
-            uint32_t m4 = 0;
-            for (int i = lane; i < n16; i += 32) {
-                const uint4 v = src[i];
-                m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
-            }
-            uint32_t mx = max(max(m4 & 0xFFu, (m4 >> 8) & 0xFFu), max((m4 >> 16) & 0xFFu, m4 >> 24));
-            mx = __reduce_max_sync(0xffffffffu, mx);
-            // (a stacked block's MMA already covers the lo2 rows)
-            const int np = !p.stacked && mx >= (uint32_t)LO2_SCALE_MIN ? 2 : 1;
-            if (lane == 0) npass_s[buf] = np;
-            __syncwarp();
-            mbar_arrive_w(&info_full[buf]);
-            return np;
-        };
         Work t;
-        int t_pass = 1;
         if (blockIdx.x < total) {
             work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            if constexpr (!SFI) {     // per-item mode: the scale-factor warps load the scales
-                ok = load_scales(t);
-                if (ok) t_pass = publish_passes(t, ld_buf, ld_par);
-                ok = ok && t_pass > 0;
-            }
+            if constexpr (!SFI) ok = load_scales(t);     // per-item mode: the scale-factor warps load them
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             uint4 tail[8];                   // the item's K tail codes (rows lane + 32j)
@@ -322,33 +290,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (n_st > n_main) load_tail();
             Work tn;
             const bool has_next = w + (int)gridDim.x < total;
-            int tn_buf = 0;
-            uint32_t tn_par = 0;
             if (has_next) {
                 work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
                 if constexpr (!SFI) {
                     if (!load_scales(tn)) { ok = false; break; }
-                    tn_buf = ld_buf;
-                    tn_par = ld_par;
                 }
             }
-            const int n_it = n_st * t_pass;
-            // the next item's pass count is published a few stages into this item (its
-            // scale bytes have landed by then, and the ring is full, so the wait costs
-            // nothing), well before the other roles reach the item
-            const int pub_st = min(n_it - 1, 2);
-            int next_pass = 1;
-            for (int st = 0; st < n_it; ++st) {
-                const int kst = st < n_st ? st : st - n_st;      // the K stage (the same in both passes)
-                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+            // one K stage of A into the next ring slot
+            auto issue_a = [&](int st) -> bool {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) return false;
                 uint8_t *adst = a_ring + slot * GEMM_A_STAGE;
-                if (kst < n_main) {
+                if (st < n_main) {
                     // the unpacked-type TMA counts the packed bytes: 128 rows x 64
                     mbar_arrive_expect_tx_w(&full[slot], 128u * 64u);
                     if (MODE == MODE_UP)
-                        tma_load_5d_w(adst, &p.map_a, &full[slot], kst * GEMM_KS, 0, 0, 4 * t.mb, t.e);
+                        tma_load_5d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, 0, 0, 4 * t.mb, t.e);
                     else
-                        tma_load_3d_w(adst, &p.map_a, &full[slot], kst * GEMM_KS, t.mb * GEMM_BM, t.e);
+                        tma_load_3d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, t.mb * GEMM_BM, t.e);
                 } else {
                     // K tail of rows lane + 32j: 2 x 16 code bytes -> the first four
                     // 16-byte units of the row (8 code bytes each, the rest zero),
@@ -370,15 +328,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 }
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
-                if constexpr (!SFI) {
-                    if (has_next && st == pub_st) {
-                        next_pass = publish_passes(tn, tn_buf, tn_par);
-                        if (next_pass == 0) { ok = false; break; }
+                return true;
+            };
+            for (int st = 0; st < n_st; ++st) {
+                if (!issue_a(st)) { ok = false; break; }
+            }
+            if constexpr (!SFI) {     // the lo2 pass: the item's K stages once more
+                if (ok && item_passes(p, t) > 1) {
+                    for (int st = 0; st < n_st; ++st) {
+                        if (!issue_a(st)) { ok = false; break; }
                     }
                 }
             }
             if (!ok) break;
-            t_pass = next_pass;
             t = tn;
         }
         if (!ok) {
@@ -394,29 +356,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         if constexpr (MODE == MODE_DOWN) pdl_wait();     // h comes from the gate/up GEMM
         int slot = 0;
         uint32_t ph = 0;
-        int ib = 0;                          // scale buffer (and pass-count word) of the item
-        uint32_t iph = 0;
         long long issued = 0;
         bool ok = true;
         const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            int npass = 1;
-            if constexpr (!SFI) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[ib], iph, wc))) { ok = false; break; }
-                npass = npass_s[ib];
-                __syncwarp();
-                mbar_arrive_w(&s_empty[ib]);
-                if (++ib == 2) { ib = 0; iph ^= 1; }
-            }
-            for (int st = 0; st < n_st * npass; ++st) {
-                const int kst = st < n_st ? st : st - n_st;
+            for (int st = 0; st < n_st; ++st) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                 mbar_arrive_expect_tx_w(&full[slot], b_bytes);
-                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], kst * GEMM_KS, t.p0, st < n_st ? 0 : 2);
+                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], st * GEMM_KS, t.p0, 0);
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
+            }
+            if constexpr (!SFI) {     // the lo2 pass: boxes from the lo2 plane
+                if (ok && item_passes(p, t) > 1) {
+                    for (int st = 0; st < n_st; ++st) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                        mbar_arrive_expect_tx_w(&full[slot], b_bytes);
+                        tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], st * GEMM_KS, t.p0, 2);
+                        ++issued;
+                        if (++slot == NS) { slot = 0; ph ^= 1; }
+                    }
+                }
             }
         }
         if (!ok) drain_ring(full, NS, issued, p.wait_limit_ns);
@@ -430,8 +392,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const int m = warp - 1;
         int db = 0, sb = 0;
         uint32_t dph = 0, sph = 0;
-        int ib = 0;
-        uint32_t iph = 0;
         bool ok = true, issued = false;
         // ring slot and phase parity of the current item's first stage
         int islot = 0;
@@ -444,15 +404,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            int npass = 1;
-            if constexpr (!SFI) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[ib], iph, wc))) { ok = false; break; }
-                npass = npass_s[ib];
-                __syncwarp();
-                mbar_arrive_w(&s_empty[ib]);
-                if (++ib == 2) { ib = 0; iph ^= 1; }
-            }
-            const int n_it = n_st * npass;
+            const int n_it = SFI ? n_st : n_st * item_passes(p, t);
             const uint32_t n = stacked ? (uint32_t)(3 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
             // E8M0 scales, M >> 4; K block kb of a stage takes scale byte kb (fields at 4 and 29)
@@ -469,9 +421,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             int slot = islot;
             uint32_t ph = iph_ring;
             advance(slot, ph, m);
-            for (int st = m; st < n_it; st += n_mma_warps) {
-                const bool lo2_pass = st >= n_st;
-                const int kst = lo2_pass ? st - n_st : st;
+            for (int st = m; st < n_st; st += n_mma_warps) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
                 tc_fence_after();
                 // descriptors of the slot's A and B; K block kb starts 32 bytes further
@@ -479,22 +429,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 const uint64_t ad = smem_desc_sw128(smem_addr(a_ring + slot * GEMM_A_STAGE));
                 const uint64_t bd = smem_desc_sw128(smem_addr(b_ring + slot * b_stage));
                 const uint64_t bd_lo = bd + (uint64_t)(NB * 128 >> 4);
-                const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * kst)
+                const uint32_t sf = SFI ? sf_item + (uint32_t)(GEMM_SFI_COLS * st)
                                         : tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
                 const uint32_t sfb = SFI ? sf + 4 : sf + 8;
-                // K blocks of this stage: 4, or 1..3 in the K tail
-                const int nkb = kst < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
-                if (lo2_pass) {
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb)
-                        if (kb < nkb) mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, 1u);
-                } else if (nkb == 4) {
+                if (st < n_main) {
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
                         mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sfb, (acc | kb) ? 1u : 0u);
                         if (!stacked) mma_mx_w(d_tmem, ad + 2 * kb, bd_lo + 2 * kb, idesc[kb], sf, sf + 16, 1u);
                     }
                 } else {
+                    const int nkb = (p.K - n_main * GEMM_KS) / 32;    // the K tail: 1..3 blocks
 #pragma unroll
                     for (int kb = 0; kb < 3; ++kb) {
                         if (kb >= nkb) break;
@@ -506,6 +451,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 issued = true;
                 mma_commit_w(&empty[slot]);
                 advance(slot, ph, n_mma_warps);
+            }
+            if constexpr (!SFI) {
+                // the lo2 pass (one MMA warp): per K block one MMA over the slot's first plane,
+                // the lo2 rows, with hi's scale column, into the same accumulator
+                if (ok && n_it > n_st) {
+                    for (int st = 0; st < n_st; ++st) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t ad = smem_desc_sw128(smem_addr(a_ring + slot * GEMM_A_STAGE));
+                        const uint64_t bd = smem_desc_sw128(smem_addr(b_ring + slot * b_stage));
+                        const uint32_t sf = tmem + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                        const int nkb = st < n_main ? 4 : (p.K - n_main * GEMM_KS) / 32;
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            if (kb < nkb) mma_mx_w(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc[kb], sf, sf + 8, 1u);
+                        mma_commit_w(&empty[slot]);
+                        advance(slot, ph, 1);
+                    }
+                }
             }
             if (!ok) break;
             advance(islot, iph_ring, n_it);
@@ -562,22 +526,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     }
                 }
         };
-        // per-stage mode: the item's stage st (counted over both passes) uses bw[st % SF_PD],
-        // loaded SF_PD stages ahead; an item with at least SF_PD stages loads the next item's
-        // first SF_PD stages into the slots its last stages free
+        // per-stage mode: stage st's B words sit in bw[st % SF_PD], loaded SF_PD stages
+        // ahead; the slots an item's last stages free take the next item's first stages
+        // (a lo2 pass loads its words as it goes)
         uint32_t bw[SF_PD][SF_WORDS];
-        bool bw_ready = false;               // bw holds the current item's first stages
         if constexpr (!SFI) {
             if constexpr (MODE == MODE_DOWN) pdl_wait();     // h's scales come from the gate/up GEMM
+            if (blockIdx.x < total) {
+                Work t0;
+                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t0);
+#pragma unroll
+                for (int i = 0; i < SF_PD; ++i)
+                    if (i < n_st) load_bsf(t0, i, bw[i]);
+            }
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            int npass = 1;
+            const int npass = item_passes(p, t);
             if constexpr (!SFI) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
-                if (!__all_sync(0xffffffffu, mbar_wait(&info_full[sb], sph, wc))) { ok = false; break; }
-                npass = npass_s[sb];
             }
             const uint8_t *sbase = scale_buf + (SFI ? 0 : sb * scale_bytes);
             const uint8_t *srow[4];
@@ -676,26 +644,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 mbar_arrive_w(&f_full[sb]);
                 bph ^= 1;
             } else {
-                const int n_it = n_st * npass;
-                if (!bw_ready) {
-#pragma unroll
-                    for (int i = 0; i < SF_PD; ++i) load_bsf(t, i % n_st, bw[i]);
-                }
                 Work tn;
                 const bool has_next = w + (int)gridDim.x < total;
                 if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
-                const bool pre_next = has_next && n_it >= SF_PD;
-                for (int st0 = 0; st0 < n_it && ok; st0 += SF_PD) {
+                for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
 #pragma unroll
                     for (int i = 0; i < SF_PD; ++i) {
                         const int st = st0 + i;
-                        if (st >= n_it) break;
-                        const int kst = st < n_st ? st : st - n_st;
+                        if (st >= n_st) break;
                         if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                         const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
                         {
                             uint32_t v[4];
-                            a_words(kst, v);
+                            a_words(st, v);
                             tmem_st4(sf, v);
                         }
                         // B: the hi (and lo) columns of the token block, one store per
@@ -712,19 +673,38 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                             tmem_st2v(sf + 20, b[10], b[11]);
                         }
                         tmem_wait_st();
-                        if (st + SF_PD < n_it) {
-                            const int kn = st + SF_PD;
-                            load_bsf(t, kn < n_st ? kn : kn - n_st, bw[i]);
-                        } else if (pre_next) {
-                            load_bsf(tn, i % n_st, bw[i]);
-                        }
+                        if (st + SF_PD < n_st) load_bsf(t, st + SF_PD, bw[i]);
+                        else if (has_next && i < n_st) load_bsf(tn, i, bw[i]);
                         tc_fence_before();
                         __syncwarp();
                         mbar_arrive_w(&full[slot]);
                         if (++slot == NS) { slot = 0; ph ^= 1; }
                     }
                 }
-                bw_ready = pre_next;
+                // the lo2 pass: each stage's A words and hi words again (the lo2 MMAs read
+                // hi's scale column), loaded as it goes
+                if (ok && npass > 1) {
+                    for (int st = 0; st < n_st; ++st) {
+                        uint32_t hw[SF_WORDS / 2];
+                        const uint32_t *bsf = p.b_sf + (size_t)st * 2 * p.P_max + t.p0;
+#pragma unroll
+                        for (int c = 0; c < SF_WORDS / 2; ++c) {
+                            const int j = 32 * c + lane;
+                            hw[c] = c < n_sfb && j < t.n_valid ? __ldg(bsf + j) : 0x7F7F7F7Fu;
+                        }
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
+                        const uint32_t sf = lane_base + sf_col0 + (uint32_t)(slot * GEMM_SF_COLS);
+                        uint32_t v[4];
+                        a_words(st, v);
+                        tmem_st4(sf, v);
+                        tmem_st8v(sf + 8, hw[0], hw[1], hw[2], hw[3], hw[4], hw[5], 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        mbar_arrive_w(&full[slot]);
+                        if (++slot == NS) { slot = 0; ph ^= 1; }
+                    }
+                }
             }
             if (!ok) break;
             if constexpr (!SFI) {
@@ -752,6 +732,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             const int wrow = tile_weight_row<MODE>(tl, t.mb, p.F);
             const bool row_valid = wrow < p.R;
+            // (up) h's lo2 plane: always for stacked blocks, else only where the down GEMM may read it
+            bool want_lo2 = MODE == MODE_UP && p.stacked;
+            if (MODE == MODE_UP && !p.stacked && p.down_pass) {
+                // the expert's row of the down pass table, one byte per lane (two loads)
+                const uint8_t *dp = p.down_pass + (size_t)t.e * DOWN_PASS_STRIDE;
+                const bool two = (lane < p.MB_down && __ldg(dp + lane) > 1) ||
+                                 (lane + 32 < p.MB_down && __ldg(dp + lane + 32) > 1);
+                want_lo2 = __any_sync(0xffffffffu, two);
+            }
             const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + wrow]) : 0.f;
             if (MODE == MODE_DOWN) {
                 for (int c = lane; c < t.n_valid; c += 32) mval[c] = p.row_w[t.p0 + c];
@@ -760,9 +749,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if (!__all_sync(0xffffffffu, mbar_wait(&d_full[db], dph, wc))) break;
             if (n_mma_warps == 2 && !__all_sync(0xffffffffu, mbar_wait(&d_full[2 + db], dph, wc))) break;
             tc_fence_after();
-            // The accumulator goes back to the MMA warps as soon as this warp has read its
-            // last chunk of it, before the chunk's SwiGLU / stores: with one buffer per MMA
-            // warp (per-item mode) the next item's MMAs then wait only for the TMEM reads.
+            // Per-item mode (one accumulator per MMA warp): the accumulator goes back to the
+            // MMA warps as soon as this warp has read its last chunk of it, before the
+            // chunk's SwiGLU / stores, so the next item's MMAs wait only for the TMEM reads.
+            // With two buffers the release comes after the stores (measured faster there).
             bool released = false;
             auto release = [&]() {
                 tc_fence_before();
@@ -770,7 +760,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 if (lane == 0) mbar_arrive(&d_empty[db]);
                 released = true;
             };
-            if (16 * eg >= t.n_mma) release();
+            if (SFI && 16 * eg >= t.n_mma) release();
             for (int c0 = 16 * eg; c0 < t.n_mma; c0 += 32) {
                 float acc[16];
 #pragma unroll
@@ -786,7 +776,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
                     }
                 }
-                if (c0 + 32 >= t.n_mma) release();
+                if (SFI && c0 + 32 >= t.n_mma) release();
                 if (MODE == MODE_UP) {
                     // SwiGLU: lanes < 16 hold gate rows, lanes >= 16 the linear rows of the
                     // same h rows; lanes < 16 finish columns 0..7, lanes >= 16 columns 8..15
@@ -844,13 +834,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                         const uint32_t qh = f32x2_to_e4m3x2(v * pow2f(-s_hi), 0.0f) & 0xFFu;
                         const float res = v - e4m3_to_f32(qh) * pow2f(s_hi);
                         const uint32_t ql = f32x2_to_e4m3x2(res * pow2f(-s_lo), 0.0f) & 0xFFu;
-                        const float res2 = res - e4m3_to_f32(ql) * pow2f(s_lo);
-                        const uint32_t ql2 = f32x2_to_e4m3x2(res2 * pow2f(-s_hi), 0.0f) & 0xFFu;
                         if (col < t.n_valid) {
                             const size_t prow = (size_t)(t.p0 + col);
                             p.h_q[prow * p.Kf + j] = (uint8_t)qh;
                             p.h_q[((size_t)p.P_max + prow) * p.Kf + j] = (uint8_t)ql;
-                            p.h_q[((size_t)2 * p.P_max + prow) * p.Kf + j] = (uint8_t)ql2;
+                            if (want_lo2) {
+                                const float res2 = res - e4m3_to_f32(ql) * pow2f(s_lo);
+                                const uint32_t ql2 = f32x2_to_e4m3x2(res2 * pow2f(-s_hi), 0.0f) & 0xFFu;
+                                p.h_q[((size_t)2 * p.P_max + prow) * p.Kf + j] = (uint8_t)ql2;
+                            }
                             if ((q & 1) == 0 && (lane & 15) == 0) {
                                 // one lane per (column, 32-block): the two scale bytes
                                 const size_t wi = (size_t)(fblk >> 2) * 2 * p.P_max;
@@ -887,6 +879,75 @@ template __global__ void expert_gemm_kernel<MODE_UP, false>(const __grid_constan
 template __global__ void expert_gemm_kernel<MODE_UP, true>(const __grid_constant__ GemmParams p);
 template __global__ void expert_gemm_kernel<MODE_DOWN, false>(const __grid_constant__ GemmParams p);
 template __global__ void expert_gemm_kernel<MODE_DOWN, true>(const __grid_constant__ GemmParams p);
+
+// The pass table of the large-block GEMMs: for every gate/up work-item weight
+// block (64 gate rows and their 64 linear rows of W13) and every down weight
+// block (128 rows of W2), 2 when a scale byte of its rows reaches LO2_SCALE_MIN
+// (a pass over the lo2 term), else 1.  One warp per block, all of a lane's
+// loads in flight together.  It reads weights only, so it runs at once; it
+// waits for the kernel before it only at its end, which keeps the stream's
+// order for the GEMM after it.
+__global__ void __launch_bounds__(256) pass_plan_kernel(const uint8_t *w13_scales, const uint8_t *w2_scales, int E,
+                                                        int d, int F, uint8_t *up_pass, uint8_t *down_pass) {
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int mb_up = F / 64, mb_dn = (d + GEMM_BM - 1) / GEMM_BM;
+    const long long n_up = (long long)E * mb_up, n_dn = (long long)E * mb_dn;
+    if (gw < n_up + n_dn) {
+        const uint4 *run[2];
+        int n16[2];
+        if (gw < n_up) {
+            const int e = (int)(gw / mb_up), mb = (int)(gw % mb_up);
+            const size_t kb = (size_t)d / 32;
+            run[0] = reinterpret_cast<const uint4 *>(w13_scales + ((size_t)e * 2 * F + (size_t)mb * 64) * kb);
+            run[1] = reinterpret_cast<const uint4 *>(w13_scales + ((size_t)e * 2 * F + F + (size_t)mb * 64) * kb);
+            n16[0] = n16[1] = (int)(64 * kb / 16);
+        } else {
+            const long long g = gw - n_up;
+            const int e = (int)(g / mb_dn), mb = (int)(g % mb_dn);
+            const size_t kb = (size_t)F / 32;
+            const int rows = min(GEMM_BM, d - mb * GEMM_BM);
+            run[0] = reinterpret_cast<const uint4 *>(w2_scales + ((size_t)e * d + (size_t)mb * GEMM_BM) * kb);
+            run[1] = run[0];
+            n16[0] = (int)(rows * kb / 16);
+            n16[1] = 0;
+        }
+        uint32_t m4 = 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            for (int i0 = lane; i0 < n16[r]; i0 += 32 * 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + 32 * u;
+                    v[u] = i < n16[r] ? __ldg(run[r] + i) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v[u].x, v[u].y), __vmaxu4(v[u].z, v[u].w)));
+            }
+        }
+        uint32_t m = max(max(m4 & 0xFFu, (m4 >> 8) & 0xFFu), max((m4 >> 16) & 0xFFu, m4 >> 24));
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) {
+            const uint8_t np = m >= (uint32_t)LO2_SCALE_MIN ? 2 : 1;
+            if (gw < n_up) {
+                up_pass[gw] = np;
+            } else {
+                const long long g = gw - n_up;
+                down_pass[(g / mb_dn) * DOWN_PASS_STRIDE + g % mb_dn] = np;
+            }
+        }
+    }
+    pdl_wait();
+}
+
+cudaError_t launch_pass_plan(const uint8_t *w13_scales, const uint8_t *w2_scales, int E, int d, int F,
+                             uint8_t *up_pass, uint8_t *down_pass, cudaStream_t s) {
+    const long long warps = (long long)E * (F / 64) + (long long)E * ((d + GEMM_BM - 1) / GEMM_BM);
+    return launch_pdl(pass_plan_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, w13_scales, w2_scales, E,
+                      d, F, up_pass, down_pass);
+}
 
 template <int MODE, bool SFI>
 static cudaError_t launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t s) {

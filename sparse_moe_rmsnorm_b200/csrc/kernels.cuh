@@ -115,6 +115,15 @@ struct GemmParams {
     uint8_t *h_q;
     uint8_t *h_sf;              // bytes of [Kf/128][2][P_max] words
     int Kf;                     // F rounded up to 128
+    // Large blocks: the pass count of each work item's weight block, u8 [E][MB]: 1, or 2 with a
+    // pass over the lo2 term (weights reaching LO2_SCALE_MIN); NULL: one pass.  Stacked blocks
+    // carry all three terms in one pass.
+    const uint8_t *item_pass;
+    int item_pass_stride;       // bytes per expert in item_pass
+    // UP, large blocks: the down GEMM's pass counts u8 [E][DOWN_PASS_STRIDE]; h gets its lo2
+    // plane for the experts with a two-pass down item (stacked blocks always write it)
+    const uint8_t *down_pass;
+    int MB_down;
     // DOWN output: fp32 weighted rows [P][d]
     float *out_rows;
     unsigned int *err;
@@ -134,6 +143,9 @@ constexpr int GEMM_SF_COLS = 24;      // TMEM columns per scale-factor slot: A a
 // its tolerance; above it the pre-activations grow large enough that two-term
 // rounding of the activations moves the clamped SwiGLU's output.
 constexpr int LO2_SCALE_MIN = 126;
+// Row stride (bytes) of the down GEMM's pass table: at least its weight blocks per expert
+// (ceil(d_model / 128) <= 48), so that a warp reads an expert's row in one load.
+constexpr int DOWN_PASS_STRIDE = 64;
 constexpr int GEMM_SMEM_LIMIT = 227 * 1024;
 
 // Shared-memory plan of the GEMM kernel (all offsets from a 1024-aligned base).
@@ -151,8 +163,7 @@ __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a *
 __host__ __device__ inline int gemm_num_barriers(int n_stages) {
     // stage full/empty [NS], A-scale full/empty [2], D full [2 MMA warps][2], D empty [2],
     // drain [2], epilogue exchange [2][2], item scale factors full/empty [2], staged B words full/empty,
-    // item pass count published [2]
-    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2 + 2;
+    return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2;
 }
 
 // B ring slot: the token block's hi, lo and lo2 rows (stacked) or two planes (hi and lo, or lo2
@@ -175,8 +186,7 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
     s.bsf_off = s.meta_off + align_up(8 * nb_rows * 4, 16);        // per epilogue warp: one value per column
     s.bar_off = s.bsf_off + (sf_item ? GEMM_SFI_BSF_BYTES : 0);
     s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_stages) * 8, 16);
-    // misc: tmem base, abort flag, the lo2 pass flags of the two scale buffers, then
-    // counts/offsets/tiles caches
+    // misc: tmem base, abort flag, then counts/offsets/tiles caches
     s.total = s.misc_off + 16 + 3 * (E + 1) * 4;
     s.total = align_up(s.total, 128) + 1024;  // slack for aligning the base
     return s;

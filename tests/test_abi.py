@@ -63,7 +63,7 @@ def test_strings_and_shape_validation_without_gpu(lib):
 
 def test_stage_calls_reject_null_context(lib):
     assert lib.moe_group(None, 4, 4, None) == moe.MOE_ERR_ARG
-    assert lib.moe_expert_up(None, 4, 4, None, None, None, None) == moe.MOE_ERR_ARG
+    assert lib.moe_expert_up(None, 4, 4, None, None, None, None, None) == moe.MOE_ERR_ARG
     assert lib.moe_copy_workspace(None, 0, None, 0, None) == moe.MOE_ERR_ARG
 
 

@@ -341,15 +341,15 @@ def _np_swiglu(gate, lin):
                                          (24, 256, 320, 32, 4)])
 def test_up_stage_h_encoding(T, d, F, E, k):
     """The gate/up GEMM + SwiGLU epilogue against float64 on the same (decoded) operands: h, read back
-    from its three E4M3 terms, within the encoding's rounding of the float64 value (2^-12 of the
-    32-block maximum, plus the fp32 accumulation)."""
+    from its E4M3 terms, within the encoding's rounding of the float64 value (2^-12 of the 32-block
+    maximum with three terms, 2^-9 with two, plus the fp32 accumulation)."""
     inp = custom_layer(T=T, d=d, F=F, E=E, k=k, seed=T + d)
     w = moe.MoEWeights.from_numpy(inp)
     x = _bf16_dev(inp["x"])
     m = moe.MoE(T, d, F, E, k)
     moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
     moe.moe_group(m.ctx, T, k)
-    moe.moe_expert_up(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13)
+    moe.moe_expert_up(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13, w.w2_scales)
     torch.cuda.synchronize()
     assert m.sync_status() == moe.MOE_OK
     P = T * k
@@ -365,7 +365,9 @@ def test_up_stage_h_encoding(T, d, F, E, k):
     nt = 3 if T <= 64 else 2
     xb = decode_terms([xq[i, :P, :d] for i in range(nt)], scale_bytes_from_words(xsf, 0, rows, d // 32),
                       scale_bytes_from_words(xsf, 1, rows, d // 32))
-    h = decode_terms([hq[i, :P, :F] for i in range(3)], scale_bytes_from_words(hsf, 0, rows, F // 32),
+    # h is written with three terms in decode-sized batches; larger ones write the third only for
+    # experts whose W2 scale bytes reach 126 (none here)
+    h = decode_terms([hq[i, :P, :F] for i in range(nt)], scale_bytes_from_words(hsf, 0, rows, F // 32),
                      scale_bytes_from_words(hsf, 1, rows, F // 32))
     W13 = oracle.decode_matrix(inp["w13_codes"].reshape(-1, d // 2), inp["w13_scales"].reshape(-1, d // 32))
     W13 = W13.reshape(E, 2 * F, d)
@@ -377,8 +379,8 @@ def test_up_stage_h_encoding(T, d, F, E, k):
         want[r] = _np_swiglu(z[:, :F], z[:, F:])
     blk_max = np.abs(want).reshape(P, F // 32, 32).max(axis=2, keepdims=True)
     err = np.abs(h - want).reshape(P, F // 32, 32)
-    # three terms keep h to 2^-12 of its block maximum (plus the fp32 accumulation of z)
-    bound = 2.0 ** -11 * blk_max + 1e-5 * np.abs(want).max()
+    # three terms keep h to 2^-12 of its block maximum, two to 2^-9 (plus the fp32 accumulation of z)
+    bound = (2.0 ** -11 if nt == 3 else 2.0 ** -8) * blk_max + 1e-5 * np.abs(want).max()
     print("h max err / block max", float(np.max(err / np.maximum(blk_max, 1e-30))))
     assert np.all(err <= bound)
     m.close()
