@@ -32,10 +32,12 @@ sys.path.insert(0, ROOT)
 from moe_inputs import CONFIGS, make_config_inputs, make_tokens  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
-# kernels of one moe_forward: route, group + permute, gate/up GEMM, down GEMM, combine; large
-# batches add the scan of the W2 scale bytes before the gate/up GEMM
-def kernels_per_layer(T: int) -> int:
-    return 5 if T <= 64 else 6
+# kernels of one moe_forward: route, group + permute, gate/up GEMM, down GEMM, combine; batches over
+# 64 tokens add the pass plan before the gate/up GEMM, and over 2048 pairs the grouping and the
+# tokens' encoding are two kernels
+def kernels_per_layer(T: int, k: int = 4) -> int:
+    n = 5 if T <= 64 else 6
+    return n + 1 if T * k > 2048 else n
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / bf16 tensor roofline"
 DESCRIPTIONS = {
     "tiny": "tiny MoE layer: T=16, d_model=d_ff=128, E=8, top-4",
@@ -506,7 +508,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "gemm_ms_live": {k_: round(v, 4) for k_, v in gemm_ms.items()},
             "experts_touched": cnt["touched"], "clocks": clocks.summary(), "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": kernels_per_layer(T) * layers * args.steps}
+            "gpu_launches": kernels_per_layer(T, cfg.k) * layers * args.steps}
 
 
 EXTRA_WORKLOADS = ("prefill20b", "decode120b", "stack20b")

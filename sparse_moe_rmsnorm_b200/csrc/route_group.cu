@@ -701,8 +701,10 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RoutePara
 // a row, one per lane.
 constexpr int GROUP_ROWS_MAX = 1024;   // expert-sorted rows per CTA, at most
 
-// Blocks b0 + lane (lane < 32) of expert-sorted row r, token tok.
-__device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int tok, int b0, int lane) {
+// Blocks b0 + lane (lane < 32) of token tok's encoding, written to the n_rows
+// expert-sorted rows rows[0..n_rows) (the token's rows; n_rows <= 8).
+__device__ __forceinline__ void quant_rows_part(const GroupParams &p, const int (&rows)[8], int n_rows, int tok, int b0,
+                                                int lane) {
     const float4 *src = reinterpret_cast<const float4 *>(p.xn + (size_t)tok * p.d);
     const int nblk = p.d / 32, nblk_pad = p.Kd / 32;
     {
@@ -744,15 +746,20 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
             s_lo = (uint32_t)(e_lo + 127);
         }
         if (b < nblk_pad) {
-            uint4 *dh = reinterpret_cast<uint4 *>(p.xq + (size_t)r * p.Kd + 32 * b);
-            uint4 *dl = reinterpret_cast<uint4 *>(p.xq + ((size_t)p.P_max + r) * p.Kd + 32 * b);
-            uint4 *dl2 = reinterpret_cast<uint4 *>(p.xq + ((size_t)2 * p.P_max + r) * p.Kd + 32 * b);
-            dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
-            dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
-            dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
-            dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
-            dl2[0] = make_uint4(ql2[0], ql2[1], ql2[2], ql2[3]);
-            dl2[1] = make_uint4(ql2[4], ql2[5], ql2[6], ql2[7]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (q >= n_rows) break;
+                const int r = rows[q];
+                uint4 *dh = reinterpret_cast<uint4 *>(p.xq + (size_t)r * p.Kd + 32 * b);
+                uint4 *dl = reinterpret_cast<uint4 *>(p.xq + ((size_t)p.P_max + r) * p.Kd + 32 * b);
+                uint4 *dl2 = reinterpret_cast<uint4 *>(p.xq + ((size_t)2 * p.P_max + r) * p.Kd + 32 * b);
+                dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
+                dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
+                dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
+                dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
+                dl2[0] = make_uint4(ql2[0], ql2[1], ql2[2], ql2[3]);
+                dl2[1] = make_uint4(ql2[4], ql2[5], ql2[6], ql2[7]);
+            }
         }
         // the scale bytes of four consecutive blocks (lanes 4m..4m+3) as one word
         uint32_t wh = s_hi, wl = s_lo;
@@ -763,12 +770,17 @@ __device__ __forceinline__ void quant_row_part(const GroupParams &p, int r, int 
         }
         if ((lane & 3) == 0 && b < nblk_pad) {
             const size_t g = (size_t)(b >> 2);
-            p.xsf[(g * 2) * p.P_max + r] = wh;
-            p.xsf[(g * 2 + 1) * p.P_max + r] = wl;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (q >= n_rows) break;
+                p.xsf[(g * 2) * p.P_max + rows[q]] = wh;
+                p.xsf[(g * 2 + 1) * p.P_max + rows[q]] = wl;
+            }
         }
     }
 }
 
+template <bool QUANT>
 __global__ void __launch_bounds__(1024) group_permute_kernel(const GroupParams p) {
     __shared__ int wcnt[32][257];
     __shared__ int off_s[257];
@@ -893,15 +905,37 @@ __global__ void __launch_bounds__(1024) group_permute_kernel(const GroupParams p
             __syncwarp();
         }
     }
-    __syncthreads();
+    if constexpr (QUANT) {
+        __syncthreads();
+        // this CTA's rows of the B operand: one warp per (row, 32 blocks of 32 elements), so
+        // that a row's loads are spread over warps rather than chained in one
+        const int parts = (p.Kd / 32 + 31) / 32;
+        for (int u = warp; u < (r1 - r0) * parts; u += 32) {
+            const int rr = u / parts;
+            const int rows[8] = {r0 + rr, 0, 0, 0, 0, 0, 0, 0};
+            quant_rows_part(p, rows, 1, tok_s[rr], (u - rr * parts) * 32, lane);
+        }
+    }
+}
 
-    // this CTA's rows of the B operand, one warp per row
-    // this CTA's rows of the B operand: one warp per (row, 32 blocks of 32 elements), so
-    // that a row's loads are spread over warps rather than chained in one
+// Large batches: the B operand token by token, after the grouping kernel.  A
+// warp takes (token, 32 blocks of 32 elements): it reads the token's normalised
+// row once, encodes it once and writes it to the token's k expert-sorted rows
+// (pair_row), so every token is read once rather than k times.
+__global__ void __launch_bounds__(256) encode_tokens_kernel(const GroupParams p, int T) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
     const int parts = (p.Kd / 32 + 31) / 32;
-    for (int u = warp; u < (r1 - r0) * parts; u += 32) {
-        const int rr = u / parts;
-        quant_row_part(p, r0 + rr, tok_s[rr], (u - rr * parts) * 32, lane);
+    const long long n_tasks = (long long)T * parts;
+    const long long n_warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n_tasks; u += n_warps) {
+        const int tok = (int)(u / parts), part = (int)(u % parts);
+        const int mine = lane < p.k ? __ldg(p.pair_row + (size_t)tok * p.k + lane) : 0;
+        int rows[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rows[q] = __shfl_sync(0xffffffffu, mine, q);
+        quant_rows_part(p, rows, p.k, tok, part * 32, lane);
     }
 }
 
@@ -1047,14 +1081,27 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
     return launch_route_cfg<4, 32, 8, 4>(p, s);
 }
 
+// Pairs above which the grouping and the token-major encoding run as two kernels.
+constexpr int GROUP_SPLIT_PAIRS = 2048;
+
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s) {
     if (p.P <= 0) return cudaSuccess;
-    // CTAs: one per 8 rows for small batches, one per SM for large ones, and at
-    // most GROUP_ROWS_MAX rows each
-    int grid = (p.P + 7) / 8;
-    if (grid > 148) grid = 148;
-    if ((p.P + grid - 1) / grid > GROUP_ROWS_MAX) grid = (p.P + GROUP_ROWS_MAX - 1) / GROUP_ROWS_MAX;
-    return launch_pdl(group_permute_kernel, dim3(grid), dim3(1024), 0, s, p);
+    if (p.P <= GROUP_SPLIT_PAIRS) {
+        // one kernel: a CTA per 8 rows, each encoding its own rows
+        int grid = (p.P + 7) / 8;
+        if (grid > 148) grid = 148;
+        if ((p.P + grid - 1) / grid > GROUP_ROWS_MAX) grid = (p.P + GROUP_ROWS_MAX - 1) / GROUP_ROWS_MAX;
+        return launch_pdl(group_permute_kernel<true>, dim3(grid), dim3(1024), 0, s, p);
+    }
+    // the grouping with up to GROUP_ROWS_MAX rows per CTA, then the tokens' encoding
+    const int grid = (p.P + GROUP_ROWS_MAX - 1) / GROUP_ROWS_MAX;
+    cudaError_t e = launch_pdl(group_permute_kernel<false>, dim3(grid), dim3(1024), 0, s, p);
+    if (e != cudaSuccess) return e;
+    const int T = p.P / p.k;
+    const int parts = (p.Kd / 32 + 31) / 32;
+    long long ctas = ((long long)T * parts + 7) / 8;
+    if (ctas > 148 * 8) ctas = 148 * 8;
+    return launch_pdl(encode_tokens_kernel, dim3((unsigned)ctas), dim3(256), 0, s, p, T);
 }
 
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
