@@ -85,10 +85,12 @@ inline bool encode_bq(CUtensorMap *m, const void *base, int rows, int Kpad, int 
 inline int round_up_128(int v) { return (v + 127) / 128 * 128; }
 
 // Token rows per GEMM work item.  Decode-sized batches (T <= 64) use blocks of
-// 16 rows: experts then rarely hold more than one block and the accumulator
-// stays small; an expert with more tokens takes extra blocks whose weight
-// re-reads hit L2.  Larger batches use the smallest multiple of 16 that holds
-// every token (an expert receives each token at most once), capped at
+// 16 rows: their three terms stack into one MMA of N = 48; experts then rarely
+// hold more than one block, and an expert with more tokens takes extra blocks
+// whose weight re-reads hit L2.  (Blocks of 8 -- an MMA of N = 32 over 24 rows
+// and 8 zero rows, a 4 KB slot and one more ring stage -- measured slower on
+// both decode shapes.)  Larger batches use the smallest multiple of 16 that
+// holds every token (an expert receives each token at most once), capped at
 // GEMM_NB_MAX.
 inline int token_block_rows(int T) {
     if (T <= 64) return 16;
@@ -102,7 +104,7 @@ inline int token_block_rows(int T) {
 inline int plan_gemm(GemmParams &p, int mode, int T, int top_k, int d, int F, int E, int P_max, int num_sms,
                      int *grid, int *smem) {
     p.nb_rows = token_block_rows(T);
-    // small token blocks: one MMA over the hi, lo and lo2 rows together (N = 3 nb_rows <= 192)
+    // small token blocks: one MMA over the hi, lo and lo2 rows together (N = 3 nb_rows, rounded up to 16)
     p.stacked = p.nb_rows <= 64 ? 1 : 0;
     if (mode == MODE_UP) {
         p.K = d;

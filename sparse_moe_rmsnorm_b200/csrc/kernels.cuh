@@ -33,8 +33,7 @@ enum : unsigned int {
     ERR_WAIT_UP = 1u,      // a bounded wait ran out in the gate/up GEMM
     ERR_WAIT_DOWN = 2u,    // ... in the down GEMM
     ERR_WAIT_SELFTEST = 4u,
-    ERR_ROUTING = 8u,      // an expert index out of range reached the grouping
-    ERR_WAIT_ROUTE = 16u   // a bounded wait ran out in the tensor-core router
+    ERR_ROUTING = 8u       // an expert index out of range reached the grouping
 };
 
 struct RouteParams {
@@ -49,8 +48,6 @@ struct RouteParams {
     float *topk_w;              // [T, k]
     float *logits;              // fp32 [T, E] (decode-sized path: the CTAs' share of each token's logits)
     unsigned int *tok_done;     // [T] CTAs finished per token (decode-sized path); zero between calls
-    unsigned int *err;          // device error word (bounded waits of the tensor-core router)
-    unsigned long long wait_limit_ns;
 };
 
 struct GroupParams {
@@ -102,7 +99,8 @@ struct GemmParams {
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= GEMM_NB_MAX)
-    int stacked;                // 1: one MMA covers the hi, lo and lo2 rows (N = 3 nb_rows); 0: one MMA per term
+    int stacked;                // 1: one MMA covers the hi, lo and lo2 rows (N = 3 nb_rows rounded up to 16);
+                                //    0: one MMA per term
     int n_stages;               // shared-memory ring depth (and TMEM scale-factor ring depth when !sf_item)
     int sf_item;                // 1: a work item's scale factors are written to TMEM once, before its first
                                 //    stage, and two MMA warps take alternate stages (decode-sized blocks);
@@ -154,9 +152,13 @@ struct GemmSmem {
 };
 
 // Per-item mode: the B scale words of one work item, staged in shared memory
-// for the scale-factor warps ([stage][4 columns][32 lanes] words).
+// for the scale-factor warps ([stage][B columns][32 lanes] words; a stacked
+// block's rows take one column per 32, at most 4).
 constexpr int GEMM_SFI_STAGES_MAX = 24;
-constexpr int GEMM_SFI_BSF_BYTES = GEMM_SFI_STAGES_MAX * 4 * 32 * 4;
+__host__ __device__ inline int gemm_sfi_b_cols(int nb_rows) { return (3 * nb_rows + 31) / 32; }
+__host__ __device__ inline int gemm_sfi_bsf_bytes(int nb_rows) {
+    return GEMM_SFI_STAGES_MAX * gemm_sfi_b_cols(nb_rows) * 32 * 4;
+}
 
 __host__ __device__ inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
@@ -166,11 +168,16 @@ __host__ __device__ inline int gemm_num_barriers(int n_stages) {
     return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2;
 }
 
-// B ring slot: the token block's hi, lo and lo2 rows (stacked) or two planes (hi and lo, or lo2
-// and an empty plane in a lo2 pass)
+// MMA width of a stacked block: its hi, lo and lo2 rows (3 nb_rows), rounded up to the
+// tensor core's N granularity of 16; the rows past 3 nb_rows are zeros
+__host__ __device__ inline int gemm_stacked_n(int nb_rows) { return (3 * nb_rows + 15) / 16 * 16; }
+// Planes one B copy brings: hi, lo and lo2 (stacked); hi and lo, or lo2 and an empty plane
+// in a lo2 pass
 __host__ __device__ inline int gemm_b_planes(int stacked) { return stacked ? 3 : 2; }
+// B ring slot: the token block's hi, lo and lo2 rows and the zero rows after them (stacked),
+// or two planes (hi and lo, or lo2 and an empty plane in a lo2 pass)
 __host__ __device__ inline int gemm_b_stage_bytes(int nb_rows, int stacked) {
-    return gemm_b_planes(stacked) * nb_rows * 128;
+    return (stacked ? gemm_stacked_n(nb_rows) : 2 * nb_rows) * 128;
 }
 
 __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int stacked, int n_stages,
@@ -184,7 +191,7 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
     s.amax_off = s.scale_off + (sf_item ? 1 : 2) * scale_bytes;
     s.meta_off = s.amax_off + 2 * 2 * 4 * 16 * 4;                 // [2 groups][2 parities][4 warps][16 columns] fp32
     s.bsf_off = s.meta_off + align_up(8 * nb_rows * 4, 16);        // per epilogue warp: one value per column
-    s.bar_off = s.bsf_off + (sf_item ? GEMM_SFI_BSF_BYTES : 0);
+    s.bar_off = s.bsf_off + (sf_item ? gemm_sfi_bsf_bytes(nb_rows) : 0);
     s.misc_off = s.bar_off + align_up(gemm_num_barriers(n_stages) * 8, 16);
     // misc: tmem base, abort flag, then counts/offsets/tiles caches
     s.total = s.misc_off + 16 + 3 * (E + 1) * 4;
@@ -196,7 +203,9 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
 // ring of scale-factor slots.  Per-item mode: accumulators [2 MMA warps] (one
 // buffer each), then two item regions of 8 columns per stage (A at +0, B at +4).
 constexpr int GEMM_SFI_COLS = 8;
-__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 3 * nb_rows : nb_rows; }
+__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) {
+    return stacked ? gemm_stacked_n(nb_rows) : nb_rows;
+}
 __host__ __device__ inline int gemm_tmem_cols(int nb_rows, int stacked, int n_stages) {
     return 2 * gemm_d_cols(nb_rows, stacked) + GEMM_SF_COLS * n_stages;
 }

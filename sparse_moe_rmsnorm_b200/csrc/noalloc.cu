@@ -188,8 +188,6 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     rp.topk_w = topk_w;
     rp.logits = logits;
     rp.tok_done = tok_done;
-    rp.err = err;
-    rp.wait_limit_ns = 2000000000ull;
     if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     GroupParams gp;

@@ -209,18 +209,6 @@ __device__ __forceinline__ void tma_load_5d_w(void *dst, const void *map, uint64
         : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (both operands bf16 or both
-// f16, per the instruction descriptor), one CTA, issued by an elected lane of
-// a converged warp.
-__device__ __forceinline__ void mma_f16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // D[tmem] (+)= A[smem] * B[smem]^T with E8M0 block scales (one per 32 K
 // elements) read from TMEM: kind::mxf8f6f4, one CTA.  The scale addresses must
 // be 4-column aligned (a misaligned one faults); the byte within each 32-bit
@@ -273,16 +261,6 @@ __device__ __forceinline__ void tmem_st8v(uint32_t taddr, uint32_t a, uint32_t b
                  "r"(b), "r"(c), "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
                  : "memory");
 }
-
-// 16-byte asynchronous copy global -> shared (L2 only); src_bytes 0 fills zeros
-// and reads nothing.  Completion is tracked per thread by commit groups.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to later
 // async-proxy reads (TMA, tcgen05.mma operands).

@@ -1,7 +1,7 @@
 // Routing side of the MoE block on sm_100a:
-//   route_kernel     RMSNorm + router logits + top-k + softmax over the chosen,
-//                    plus the fp16 normalised tokens for the experts;
-//   route_tc_kernel  the same for large batches, the router on tensor cores;
+//   route_fma_kernel RMSNorm + router logits + top-k + softmax over the chosen,
+//                    plus the fp32 normalised tokens for the experts; eight
+//                    tokens per CTA, the router on CUDA cores;
 //   route_small_kernel  the same for decode-sized batches, a CTA per (token,
 //                    16 experts);
 //   group_permute_kernel  expert histogram, exclusive scan and a stable
@@ -25,12 +25,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -41,39 +35,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
 }
 
 // ----------------------------------------------------------------- route
-//
-// One CTA per TB tokens, NW warps; NW / TB warps share each token.
-//   xn = x / sqrt(mean(x^2) + eps) * scale in fp32 ("gpt-oss-20B" hub page,
-//   section 3.2), kept in shared memory for the router and stored (fp32) for
-//   the experts.
-// Router: logit_e = W_r[e] . xn + b_e in fp32 ("gpt-oss-20B" page, 3.4).
-//   Warp w owns experts w, w+NW, ... (at most EPW); the loop runs over
-//   VEC-element chunks of d, holding the TB tokens' chunk in registers while
-//   it is applied to every expert of the warp.
-// Top-k: k rounds of a warp arg-max on (logit desc, index asc) -- ties go to
-//   the lower expert index; a NaN logit ranks below every number, so the k
-//   chosen indices are always distinct and in range.  Softmax over the chosen
-//   (pnsm.cn overview, section 2.2).
-template <int VEC>
-__device__ __forceinline__ void load_bf16_vec(const uint16_t *p, float (&f)[VEC]) {
-    if (VEC == 8) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(p);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-    } else {
-        const uint2 v = *reinterpret_cast<const uint2 *>(p);
-        const uint32_t w[2] = {v.x, v.y};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-    }
-}
 
 // Top-k of one token's E logits (E <= 256) by one warp, then the softmax over
 // the chosen (pnsm.cn overview, section 2.2): k rounds of a warp arg-max on
@@ -139,110 +100,165 @@ __device__ __forceinline__ void topk_softmax_warp(const float *lg, int E, int k,
     }
 }
 
-template <int TB, int NW, int EPW, int VEC>
-__global__ void __launch_bounds__(NW * 32) route_kernel(const RouteParams p) {
-    extern __shared__ float rsm[];
-    constexpr int WPT = NW / TB;            // warps per token
+// ------------------------------------------- route, eight tokens per CTA
+//
+// One CTA per RF_TOK = 8 tokens, 8 warps.  Warp w normalises token w: the
+// row's bf16 elements (8 per lane and load, up to RF_CHUNKS loads of a lane in
+// flight), the sum of squares, 1/rms = 1/sqrt(mean(x^2) + eps) ("gpt-oss-20B"
+// hub page, section 3.2); x_j scale_j -- exact in fp32, a product of two bf16
+// numbers -- goes to shared memory, and xn_j = (x_j scale_j) (1/rms), rounded
+// once, to global memory for the experts.  Router (same page, 3.4):
+// logit_e = (1/rms) sum_j (x_j scale_j) W_r[e, j] + b_e, every product exact
+// and the sum in fp32.  Warp w takes the tile of 4 tokens (4 (w / 4) ..) and
+// 8 experts (groups w % 4, w % 4 + 4, ...); lane l the 4-element K chunks l,
+// l + 32, ... of the row; packed fp32x2 FMAs sum each (token, expert) pair's
+// even and odd elements in the two halves of one register pair.  A
+// transposing warp reduction leaves the total of tile entry 8t + e in lane
+// 8t + e.  Then the top-k and the softmax over the chosen, one warp per token.
+constexpr int RF_TOK = 8;
+constexpr int RF_THREADS = 256;
+constexpr int RF_CHUNKS = 12;           // 8-element chunks of a row per lane and batch
+
+__device__ __forceinline__ unsigned long long f32x2_pack(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(unsigned long long v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// two independent fp32 FMAs, each rounded once: (a.lo b.lo + c.lo, a.hi b.hi + c.hi)
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// bf16 pair (element j in the low half) -> fp32 pair
+__device__ __forceinline__ unsigned long long bf16x2_to_f32x2(uint32_t w) {
+    return f32x2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+__global__ void __launch_bounds__(RF_THREADS, 2) route_fma_kernel(const RouteParams p) {
+    extern __shared__ float rf_sm[];
     const int d = p.d, E = p.E;
-    float *xs = rsm;                        // [TB][d]
-    float *lg = rsm + TB * d;               // [TB][E]
-    float *red = lg + TB * E;               // [NW] partial sums / maxima
-    const int t0 = blockIdx.x * TB;
-    const int ntok = min(TB, p.T - t0);
+    float *xs = rf_sm;                       // [RF_TOK][d] x * scale
+    float *lg = xs + RF_TOK * d;             // [RF_TOK][E] logits
+    float *rinv = lg + RF_TOK * E;           // [RF_TOK] 1/rms
+    const int t0 = blockIdx.x * RF_TOK;
+    const int ntok = min(RF_TOK, p.T - t0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
     pdl_trigger();
 
-    // ---- RMSNorm
-    const int ti = warp / WPT;              // token of this warp
-    const int u = (warp % WPT) * 32 + lane; // thread index within the token's warps
-    const bool has_tok = ti < ntok;
-    const int t = t0 + ti;
-    float *xsr = xs + ti * d;
-    float ss = 0.f;
-    if (has_tok) {
-        const uint16_t *xr = p.x + (size_t)t * d;
-        for (int j = u * 8; j < d; j += WPT * 256) {
-            float f[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xr + j), f);
+    // ---- RMSNorm: warp w, token t0 + w
+    {
+        float *xr = xs + warp * d;
+        const int nch = d / 8;
+        if (warp < ntok) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + warp) * d);
+            const uint4 *scp = reinterpret_cast<const uint4 *>(p.norm_scale);
+            float ss = 0.f;
+            for (int c0 = 0; c0 < nch; c0 += 32 * RF_CHUNKS) {
+                uint4 xv[RF_CHUNKS];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                ss += f[c] * f[c];
-                xsr[j + c] = f[c];
+                for (int i = 0; i < RF_CHUNKS; ++i) {
+                    const int c = c0 + lane + 32 * i;
+                    xv[i] = c < nch ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < RF_CHUNKS; ++i) {
+                    const int c = c0 + lane + 32 * i;
+                    if (c < nch) {
+                        float f[8], sc[8];
+                        bf16x8_to_f32(xv[i], f);
+                        bf16x8_to_f32(__ldg(scp + c), sc);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
+                        float4 *o = reinterpret_cast<float4 *>(xr + 8 * c);
+                        o[0] = make_float4(f[0] * sc[0], f[1] * sc[1], f[2] * sc[2], f[3] * sc[3]);
+                        o[1] = make_float4(f[4] * sc[4], f[5] * sc[5], f[6] * sc[6], f[7] * sc[7]);
+                    }
+                }
             }
-        }
-    }
-    ss = warp_sum(ss);
-    if (lane == 0) red[warp] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int i = 0; i < WPT; ++i) tot += red[ti * WPT + i];
-    const float inv_rms = 1.0f / sqrtf(tot / (float)d + p.eps);
-    if (has_tok) {
-        float *xo = p.xn + (size_t)t * d;
-        for (int j = u * 8; j < d; j += WPT * 256) {
-            float sc[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p.norm_scale + j), sc);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) xsr[j + c] = xsr[j + c] * inv_rms * sc[c];
-            reinterpret_cast<float4 *>(xo + j)[0] = make_float4(xsr[j], xsr[j + 1], xsr[j + 2], xsr[j + 3]);
-            reinterpret_cast<float4 *>(xo + j)[1] = make_float4(xsr[j + 4], xsr[j + 5], xsr[j + 6], xsr[j + 7]);
+            ss = warp_sum(ss);
+            const float r = 1.0f / sqrtf(ss / (float)d + p.eps);
+            if (lane == 0) rinv[warp] = r;
+            __syncwarp();
+            float4 *xo = reinterpret_cast<float4 *>(p.xn + (size_t)(t0 + warp) * d);
+            const float4 *xi = reinterpret_cast<const float4 *>(xr);
+            for (int c = lane; c < d / 4; c += 32) {
+                const float4 v = xi[c];
+                xo[c] = make_float4(v.x * r, v.y * r, v.z * r, v.w * r);
+            }
+        } else {
+            for (int c = lane; c < d / 4; c += 32) reinterpret_cast<float4 *>(xr)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane == 0) rinv[warp] = 0.f;
         }
     }
     __syncthreads();
 
-    // ---- router logits
+    // ---- router logits: tile of 4 tokens x 8 experts per warp
     {
-        float acc[EPW][TB];
+        const int tg = warp >> 2;
+        const int n_eg = (E + 7) / 8;
+        const float *xt = xs + (4 * tg) * d;
+        for (int eg = warp & 3; eg < n_eg; eg += 4) {
+            const int e0 = 8 * eg;
+            unsigned long long acc[4][8];
 #pragma unroll
-        for (int a = 0; a < EPW; ++a)
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int i = 0; i < TB; ++i) acc[a][i] = 0.f;
-        const int n_mine = (E - warp + NW - 1) / NW;   // experts of this warp
-#pragma unroll 2
-        for (int j = lane * VEC; j < d; j += 32 * VEC) {
-            float xv[TB][VEC];
+                for (int e = 0; e < 8; ++e) acc[t][e] = 0ull;
+            // the router rows' chunk j of this group (zeros past the last expert)
+            const uint2 *wbase = reinterpret_cast<const uint2 *>(p.router_w + (size_t)e0 * d);
+            const int wstride = d / 4;              // uint2 per router row
+            const int n_e = min(8, E - e0);
+            for (int j = 4 * lane; j < d; j += 128) {
+                uint2 wv[8];
 #pragma unroll
-            for (int i = 0; i < TB; ++i)
+                for (int e = 0; e < 8; ++e) wv[e] = e < n_e ? __ldg(wbase + e * wstride + (j >> 2)) : make_uint2(0, 0);
+                ulonglong2 xv[4];
 #pragma unroll
-                for (int c = 0; c < VEC; c += 4) {
-                    const float4 a4 = (i < ntok) ? *reinterpret_cast<const float4 *>(xs + i * d + j + c)
-                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-                    xv[i][c] = a4.x;
-                    xv[i][c + 1] = a4.y;
-                    xv[i][c + 2] = a4.z;
-                    xv[i][c + 3] = a4.w;
-                }
+                for (int t = 0; t < 4; ++t) xv[t] = *reinterpret_cast<const ulonglong2 *>(xt + t * d + j);
 #pragma unroll
-            for (int a = 0; a < EPW; ++a) {
-                if (a < n_mine) {
-                    float wf[VEC];
-                    load_bf16_vec<VEC>(p.router_w + (size_t)(warp + a * NW) * d + j, wf);
+                for (int e = 0; e < 8; ++e) {
+                    const unsigned long long w01 = bf16x2_to_f32x2(wv[e].x);
+                    const unsigned long long w23 = bf16x2_to_f32x2(wv[e].y);
 #pragma unroll
-                    for (int i = 0; i < TB; ++i)
-#pragma unroll
-                        for (int c = 0; c < VEC; ++c) acc[a][i] = fmaf(xv[i][c], wf[c], acc[a][i]);
-                }
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < EPW; ++a) {
-            if (a < n_mine) {
-                const int e = warp + a * NW;
-                const float b = p.router_b[e];
-#pragma unroll
-                for (int i = 0; i < TB; ++i) {
-                    const float v = warp_sum(acc[a][i]);
-                    if (lane == 0 && i < ntok) lg[i * E + e] = v + b;
+                    for (int t = 0; t < 4; ++t) {
+                        acc[t][e] = ffma2(xv[t].x, w01, acc[t][e]);
+                        acc[t][e] = ffma2(xv[t].y, w23, acc[t][e]);
+                    }
                 }
             }
+            // entry 8t + e: the even and odd partial sums, then the sum over the lanes
+            float v[32];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float a, b;
+                    f32x2_unpack(acc[t][e], a, b);
+                    v[8 * t + e] = a + b;
+                }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const bool upper = (lane & o) != 0;
+#pragma unroll
+                for (int i = 0; i < o; ++i) {
+                    const float send = upper ? v[i] : v[i + o];
+                    const float keep = upper ? v[i + o] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+            const int tok = 4 * tg + (lane >> 3), e = e0 + (lane & 7);
+            if (tok < ntok && e < E) lg[tok * E + e] = v[0] * rinv[tok] + p.router_b[e];
         }
     }
     __syncthreads();
 
     // ---- top-k and softmax, one warp per token
-    for (int i = warp; i < ntok; i += NW) topk_softmax_warp(lg + i * E, E, p.k, t0 + i, p.topk_idx, p.topk_w, lane);
+    if (warp < ntok) topk_softmax_warp(lg + warp * E, E, p.k, t0 + warp, p.topk_idx, p.topk_w, lane);
 }
 
 // ------------------------------------------------------ route, decode-sized
@@ -366,314 +382,6 @@ __global__ void __launch_bounds__(512) route_small_kernel(const RouteParams p) {
         __syncwarp();
         topk_softmax_warp(lgs, E, p.k, t, p.topk_idx, p.topk_w, lane);
         if (lane == 0) p.tok_done[t] = 0;
-    }
-}
-
-// ---------------------------------------- route, large batches (tensor cores)
-//
-// A CTA takes 128 tokens (the MMA's M) and all E experts (N = E padded to a
-// multiple of 16).  Per token, logit_e = (1/rms) * sum_j (x_j scale_j) W_r[e, j]
-// + b_e: xn . W_r[e] + b_e ("gpt-oss-20B" hub page, sections 3.2 and 3.4) with
-// the factor 1/rms taken out of the sum.  x_j scale_j, the product of two bf16
-// numbers, has at most 16 significant bits and is split exactly into bf16
-// hi + lo; two kind::f16 MMAs (hi . W, lo . W) per K step sum the exact
-// products in fp32 in the tensor core.  Eight producer warps copy 64-wide K
-// chunks of x and W_r ahead (cp.async), stage them (A hi, A lo, B = W_r rows;
-// 128-byte swizzled K-major) in a ring and
-// accumulate each token's sum of squares and max |x_j scale_j|; one warp
-// issues the MMAs; then four warps read the logits from TMEM (lane = token),
-// scale by 1/rms, add the bias and take the top-k (ties to the lower index,
-// NaN below every number) and the softmax in registers; last, xn
-// from a second read of the CTA's rows.
-constexpr int RT_TOK = 128;
-constexpr int RT_KC = 64;
-constexpr int RT_THREADS = 288;          // 8 producer warps + 1 MMA warp
-constexpr int RT_DEPTH = 4;              // K chunks of x and W_r in flight per producer thread
-
-__host__ __device__ inline int rt_npad(int E) { return E < 16 ? 16 : (E + 15) / 16 * 16; }
-__host__ __device__ inline int rt_stage_bytes(int npad) { return 2 * RT_TOK * 128 + npad * 128; }
-// The K chunks are spread over n_acc accumulators (contiguous groups), summed in
-// fp32 in the epilogue: the tensor core's accumulation over many MMAs is less
-// exact than fp32 additions, and a routing decision needs the logits to ~1e-5.
-__host__ __device__ inline int rt_n_acc(int npad) { return npad <= 64 ? 8 : 0; }
-__host__ __device__ inline int rt_tmem_cols(int npad) {
-    int c = 32;
-    while (c < rt_n_acc(npad) * npad) c <<= 1;
-    return c;
-}
-
-__global__ void __launch_bounds__(RT_THREADS, 1) route_tc_kernel(const RouteParams p, int npad, int nst) {
-    extern __shared__ uint8_t rt_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_raw) + 1023) & ~uintptr_t(1023));
-    const int stage_bytes = rt_stage_bytes(npad);
-    float *ss_s = reinterpret_cast<float *>(sm + nst * stage_bytes + RT_DEPTH * (RT_TOK + npad) * 128);   // [128]
-    float *mx_s = ss_s + RT_TOK;                                      // [128] max |x s|
-    uint64_t *full = reinterpret_cast<uint64_t *>(mx_s + RT_TOK);     // [nst]
-    uint64_t *empty = full + nst;                                     // [nst]
-    uint64_t *done = empty + nst;
-    uint32_t *tmem_s = reinterpret_cast<uint32_t *>(done + 1);
-    volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_s + 1);
-    // the RMSNorm scale row, bf16 [d], 16-byte aligned (it is read and written as uint4)
-    uint16_t *sc_s = reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(tmem_s + 2) + 15) & ~uintptr_t(15));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * RT_TOK;
-    const int ntok = min(RT_TOK, p.T - t0);
-    const int d = p.d, E = p.E, nk = d / RT_KC;
-    const int tcols = rt_tmem_cols(npad);
-    const int n_acc = min(rt_n_acc(npad), nk);       // accumulators in use
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < nst; ++i) {
-            mbar_init(&full[i], 8);       // the eight producer warps
-            mbar_init(&empty[i], 1);      // MMA commit
-        }
-        mbar_init(done, 1);
-        *abort_s = 0;
-        fence_barrier_init();
-    }
-    if (warp == 8) {
-        tmem_alloc(tmem_s, tcols);
-        tmem_relinquish();
-    }
-    for (int i = threadIdx.x; i < d / 8; i += RT_THREADS)
-        reinterpret_cast<uint4 *>(sc_s)[i] = __ldg(reinterpret_cast<const uint4 *>(p.norm_scale) + i);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_s;
-    const WaitCtl wc{abort_s, p.err, (unsigned)ERR_WAIT_ROUTE, p.wait_limit_ns};
-    // x may be the previous kernel's output
-    pdl_wait();
-    pdl_trigger();
-
-    if (warp < 8) {
-        // ------------------------------------------------------------- producers
-        // Thread: 16-byte chunk c of rows rb + 32q (q < 4) of x, and chunks tid + 256q of
-        // W_r.  Each thread copies its own chunks RT_DEPTH K chunks ahead into a raw
-        // staging ring (cp.async, zero fill past the rows / experts) and later converts
-        // exactly those, so no other thread's copies are waited for.
-        const int c = threadIdx.x & 7;
-        const int rb = threadIdx.x >> 3;
-        const int nbt = npad * 8;                    // 16-byte chunks of B per K chunk
-        float ss[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {0.f, 0.f, 0.f, 0.f};
-        uint8_t *raw0 = sm + nst * stage_bytes;      // RT_DEPTH raw slots: x [128][128 B], W [npad][128 B]
-        const int raw_bytes = (RT_TOK + npad) * 128;
-        auto issue = [&](int kc) {
-            if (kc < nk) {
-                uint8_t *raw = raw0 + (kc % RT_DEPTH) * raw_bytes;
-                const int k0 = kc * RT_KC;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = rb + 32 * q;
-                    cp_async16(raw + r * 128 + 16 * c, p.x + (size_t)(t0 + min(r, ntok - 1)) * d + k0 + 8 * c,
-                               r < ntok ? 16u : 0u);
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int task = threadIdx.x + 256 * q;
-                    if (task < nbt) {
-                        const int e = task >> 3, cc = task & 7;
-                        cp_async16(raw + (RT_TOK + e) * 128 + 16 * cc, p.router_w + (size_t)min(e, E - 1) * d + k0 + 8 * cc,
-                                   e < E ? 16u : 0u);
-                    }
-                }
-            }
-            cp_async_commit();                       // (an empty group past the last chunk)
-        };
-#pragma unroll
-        for (int i = 0; i < RT_DEPTH - 1; ++i) issue(i);
-        int slot = 0;
-        uint32_t ph = 0;
-        for (int kc = 0; kc < nk; ++kc) {
-            issue(kc + RT_DEPTH - 1);
-            cp_async_wait<RT_DEPTH - 1>();           // this thread's copies of chunk kc have landed
-            const uint8_t *raw = raw0 + (kc % RT_DEPTH) * raw_bytes;
-            const uint4 sr = *reinterpret_cast<const uint4 *>(sc_s + kc * RT_KC + 8 * c);
-            if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) break;
-            uint8_t *a_hi = sm + slot * stage_bytes;
-            uint8_t *a_lo = a_hi + RT_TOK * 128;
-            uint8_t *bs = a_lo + RT_TOK * 128;
-            float s8[8];
-            bf16x8_to_f32(sr, s8);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = rb + 32 * q;
-                float f[8];
-                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(raw + r * 128 + 16 * c), f);
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float p0 = f[2 * i] * s8[2 * i], p1 = f[2 * i + 1] * s8[2 * i + 1];
-                    ss[q] += f[2 * i] * f[2 * i] + f[2 * i + 1] * f[2 * i + 1];
-                    mx[q] = fmaxf(mx[q], fmaxf(fabsf(p0), fabsf(p1)));
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    const float2 hf = __bfloat1622float2(h2);
-                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-                    hw[i] = *reinterpret_cast<const uint32_t *>(&h2);
-                    lw[i] = *reinterpret_cast<const uint32_t *>(&l2);
-                }
-                const int off = r * 128 + ((c ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4 *>(a_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(a_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int task = threadIdx.x + 256 * q;
-                if (task < nbt) {
-                    const int e = task >> 3, cc = task & 7;
-                    *reinterpret_cast<uint4 *>(bs + e * 128 + ((cc ^ (e & 7)) << 4)) =
-                        *reinterpret_cast<const uint4 *>(raw + (RT_TOK + e) * 128 + 16 * cc);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            mbar_arrive_w(&full[slot]);
-            if (++slot == nst) { slot = 0; ph ^= 1; }
-        }
-        cp_async_wait<0>();
-        // the row statistics: the eight threads of a row are consecutive lanes
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float a = ss[q], m = mx[q];
-#pragma unroll
-            for (int o = 4; o > 0; o >>= 1) {
-                a += __shfl_xor_sync(0xffffffffu, a, o);
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            }
-            if (c == 0) {
-                ss_s[rb + 32 * q] = a;
-                mx_s[rb + 32 * q] = m;
-            }
-        }
-    } else {
-        // --------------------------------------------------------------- MMA issue
-        // kind::f16: D f32 (1 << 4), A bf16 (1 << 7), B bf16 (1 << 10), K-major, N >> 3, M >> 4
-        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(npad >> 3) << 17) |
-                               ((uint32_t)(RT_TOK >> 4) << 24);
-        int slot = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (int kc = 0; kc < nk; ++kc) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], ph, wc))) { ok = false; break; }
-            tc_fence_after();
-            uint8_t *a_hi = sm + slot * stage_bytes;
-            const uint64_t dh = smem_desc_sw128(smem_addr(a_hi));
-            const uint64_t dl = smem_desc_sw128(smem_addr(a_hi + RT_TOK * 128));
-            const uint64_t db = smem_desc_sw128(smem_addr(a_hi + 2 * RT_TOK * 128));
-            // accumulator a takes chunks [a nk / n_acc, (a + 1) nk / n_acc)
-            const int a = kc * n_acc / nk;
-            const bool first = kc == 0 || (kc - 1) * n_acc / nk != a;
-            const uint32_t dacc = tmem + (uint32_t)(a * npad);
-#pragma unroll
-            for (int ks = 0; ks < RT_KC / 16; ++ks) {      // K = 16 per MMA: 32 bytes of a row
-                mma_f16_ss_w(dacc, dh + 2 * ks, db + 2 * ks, idesc, (first && ks == 0) ? 0u : 1u);
-                mma_f16_ss_w(dacc, dl + 2 * ks, db + 2 * ks, idesc, 1u);
-            }
-            mma_commit_w(&empty[slot]);
-            if (++slot == nst) { slot = 0; ph ^= 1; }
-        }
-        // arrives once every MMA issued above has completed (also on the abort path,
-        // where the epilogue sees the abort and skips the logits)
-        mma_commit_w(done);
-        if (!ok) {
-            const uint64_t start = globaltimer_ns();
-            while (!mbar_try_wait(done, 0) && globaltimer_ns() - start < p.wait_limit_ns) {
-            }
-        }
-    }
-    __syncthreads();                               // row statistics in shared memory
-
-    if (warp < 4) {
-        // ---------------------------------------------------- logits, top-k, softmax
-        const int row = 32 * warp + lane;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, wc));
-        tc_fence_after();
-        if (ok) {
-            const float r = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);
-            float bl[8];
-            int be[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                bl[i] = -INFINITY;
-                be[i] = -1;                        // empty
-            }
-            const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-            for (int c0 = 0; c0 < npad; c0 += 16) {
-                float sum[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-                for (int a = 0; a < n_acc; ++a) {
-                    uint32_t v[16];
-                    tmem_ld16(lane_base + (uint32_t)(a * npad + c0), v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(v[i]);
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    int e = c0 + i;
-                    if (e < E) {
-                        float l = sum[i] * r + p.router_b[e];
-                        if (l != l) l = -INFINITY;
-                        // sorted insertion: a later (higher) index never passes an equal logit
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            if (j < p.k && e >= 0 && (be[j] < 0 || l > bl[j])) {
-                                const float tl = bl[j];
-                                const int te = be[j];
-                                bl[j] = l;
-                                be[j] = e;
-                                l = tl;
-                                e = te;
-                            }
-                        }
-                    }
-                }
-            }
-            if (row < ntok) {
-                const int t = t0 + row;
-                float wsum = 0.f, wv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (j < p.k) {
-                        wv[j] = expf(bl[j] - bl[0]);
-                        wsum += wv[j];
-                    }
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (j < p.k) {
-                        p.topk_idx[(size_t)t * p.k + j] = be[j];
-                        p.topk_w[(size_t)t * p.k + j] = wv[j] / wsum;
-                    }
-            }
-        }
-    }
-    // xn = x * (1/rms) * scale in fp32: the per-row factors first, then every (row,
-    // 8-element chunk) with loads in flight
-    if (threadIdx.x < RT_TOK) {
-        const int row = threadIdx.x;
-        ss_s[row] = 1.0f / sqrtf(ss_s[row] / (float)d + p.eps);   // reused: 1/rms
-    }
-    __syncthreads();
-    {
-        const int nch = d / 8;
-        const int total = ntok * nch;
-#pragma unroll 2
-        for (int i = threadIdx.x; i < total; i += RT_THREADS) {
-            const int row = i / nch, cc = i - row * nch;
-            const float r = ss_s[row];
-            float f[8], sc[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + row) * d) + cc), f);
-            bf16x8_to_f32(reinterpret_cast<const uint4 *>(sc_s)[cc], sc);
-            float4 *xo = reinterpret_cast<float4 *>(p.xn + (size_t)(t0 + row) * d + 8 * cc);
-            xo[0] = make_float4(f[0] * r * sc[0], f[1] * r * sc[1], f[2] * r * sc[2], f[3] * r * sc[3]);
-            xo[1] = make_float4(f[4] * r * sc[4], f[5] * r * sc[5], f[6] * r * sc[6], f[7] * r * sc[7]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 8) {
-        tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)tcols);
     }
 }
 
@@ -1042,43 +750,18 @@ __global__ void selftest_wait_kernel(unsigned int *err, unsigned long long limit
 
 // --------------------------------------------------------------- launchers
 
-template <int TB, int NW, int EPW, int VEC>
-static cudaError_t launch_route_cfg(const RouteParams &p, cudaStream_t s) {
-    const size_t smem = ((size_t)TB * (p.d + p.E) + NW) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<TB, NW, EPW, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(route_kernel<TB, NW, EPW, VEC>, dim3((p.T + TB - 1) / TB), dim3(NW * 32), smem, s, p);
-}
-
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
     if (p.T <= 0) return cudaSuccess;
     // decode-sized batches: a CTA per (token, 16 experts), router rows held in registers
     if (p.T <= 512 && p.d <= ROUTE_SMALL_CHUNKS * 256 && p.logits && p.tok_done) {
         return launch_pdl(route_small_kernel, dim3(p.T, (p.E + 15) / 16), dim3(512), 0, s, p);
     }
-    // large batches: the tensor-core router, 128 tokens per CTA (from 4096 tokens,
-    // where its grid covers enough SMs to beat the CUDA-core router below)
-    if (p.T >= 4096 && p.err && rt_n_acc(rt_npad(p.E)) > 0) {
-        const int npad = rt_npad(p.E);
-        const int sb = rt_stage_bytes(npad);
-        const int fixed = RT_DEPTH * (RT_TOK + npad) * 128 + 2 * RT_TOK * 4 + 16 * 8 + 64 + 2 * p.d + 1024;
-        // (raw ring, statistics, barriers, the scale row, alignment slack)
-        int nst = (220 * 1024 - fixed) / sb;
-        if (nst > 4) nst = 4;
-        if (nst >= 2) {
-            const int smem = nst * sb + fixed;
-            cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            return launch_pdl(route_tc_kernel, dim3((p.T + RT_TOK - 1) / RT_TOK), dim3(RT_THREADS), (size_t)smem, s,
-                              p, npad, nst);
-        }
-    }
-    // otherwise: one token per CTA, 32 warps (few tokens); the router weights
-    // reused across 8 (or 4) tokens of a CTA (many tokens)
-    if (p.T <= 512 || (size_t)8 * (p.d + p.E) * 4 > 200 * 1024) return launch_route_cfg<1, 32, 8, 8>(p, s);
-    if (p.E <= 128) return launch_route_cfg<8, 16, 8, 4>(p, s);
-    return launch_route_cfg<4, 32, 8, 4>(p, s);
+    // otherwise eight tokens per CTA, the router on CUDA cores (packed fp32x2 FMAs); at most
+    // 8 (6144 + 256) + 8 floats = 200 KB of shared memory
+    const size_t smem = ((size_t)RF_TOK * (p.d + p.E) + RF_TOK) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(route_fma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(route_fma_kernel, dim3((p.T + RF_TOK - 1) / RF_TOK), dim3(RF_THREADS), smem, s, p);
 }
 
 // Pairs above which the grouping and the token-major encoding run as two kernels.

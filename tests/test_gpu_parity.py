@@ -151,9 +151,11 @@ def _assert_same_e4m3(got, want, what):
     assert same.all(), what
 
 
-# decode-sized (a CTA per token and 16 experts), the CUDA-core router (T 513..4095) and the
-# tensor-core router (T >= 4096), including E not a multiple of 16 and a ragged last token block
+# decode-sized (a CTA per token and 16 experts) and the router of 8 tokens per CTA (T > 512, and smaller
+# batches with d_model > 3072), including E not a multiple of 8 or 16, the largest d_model and E, and a
+# ragged last token block
 @pytest.mark.parametrize("T,d,E,k", [(16, 128, 8, 4), (37, 2880, 32, 4), (600, 2880, 128, 4), (2100, 256, 64, 8),
+                                     (2048, 2880, 32, 4), (700, 64, 3, 3), (100, 6144, 256, 8),
                                      (4200, 256, 40, 8), (4096, 2880, 32, 4)])
 def test_route_stage(T, d, E, k):
     inp = custom_layer(T=T, d=d, F=64, E=E, k=k, seed=T)
