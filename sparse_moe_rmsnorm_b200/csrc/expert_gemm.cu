@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     uint64_t *f_empty = f_full + 2;
     uint64_t *bw_full = f_empty + 2;        // the item's B scale words are staged (per-item mode)
     uint64_t *bw_empty = bw_full + 1;       // ... and have been read by all four scale-factor warps
-    uint32_t *bw_s = reinterpret_cast<uint32_t *>(smem + plan.bsf_off);   // [stage][B columns][32]
+    uint32_t *bw_s = reinterpret_cast<uint32_t *>(smem + plan.bsf_off);   // [stage][4][32]
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + plan.misc_off);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + plan.misc_off + 4);
     int *counts_s = reinterpret_cast<int *>(smem + plan.misc_off + 16);
@@ -625,8 +625,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     const int st = q + 4 * i;
                     if (st < n_st) {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            if (c < n_sfb) bw_s[(st * n_sfb + c) * 32 + lane] = bwr[i][c];
+                        for (int c = 0; c < 4; ++c) bw_s[(st * 4 + c) * 32 + lane] = bwr[i][c];
                     }
                 }
 #pragma unroll
@@ -644,7 +643,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     uint32_t v[8];
                     a_words(st, v);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) v[4 + c] = c < n_sfb ? bw_s[(st * n_sfb + c) * 32 + lane] : 0x7F7F7F7Fu;
+                    for (int c = 0; c < 4; ++c) v[4 + c] = bw_s[(st * 4 + c) * 32 + lane];
                     tmem_st8(region + (uint32_t)(GEMM_SFI_COLS * st), v);
                 }
                 __syncwarp();
