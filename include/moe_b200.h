@@ -215,8 +215,9 @@ MOE_API int moe_debug_plan(int mode, int T, int top_k, int d_model, int d_ff, in
  * Scratch memory comes from one fixed 8 MiB __device__ array inside the
  * library, held on every GPU that loads it until process exit; no context is
  * needed.  Limits: T <= MOE_NOALLOC_MAX_TOKENS and the workspace for the shape
- * (about T*(2d + 4E) + T*k*(7d + 3F) bytes, e.g. 7.6 MiB for 64 tokens of the
- * d_model = d_ff = 2880, top-4, 128-expert layer) must fit in the array; larger requests
+ * (about T*(4d + 4E) + T*k*(7d + 3F) bytes, d and F rounded up to 128, e.g.
+ * 7.96 MiB for 64 tokens of the d_model = d_ff = 2880, top-4, 128-expert
+ * layer) must fit in the array; larger requests
  * return MOE_ERR_ARG.  Shape limits otherwise as in moe_init.
  *
  * The first call on a device looks up the array's device address

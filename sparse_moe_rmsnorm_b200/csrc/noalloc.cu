@@ -38,7 +38,7 @@ using namespace moe;
 namespace {
 
 // 8 MiB of scratch: enough for decode-sized batches of the gpt-oss layers
-// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 7.8 MiB with 128
+// (up to 64 tokens, top-4, d_model = d_ff = 2880 needs about 7.96 MiB with 128
 // experts).
 constexpr size_t kScratchBytes = 8u << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
