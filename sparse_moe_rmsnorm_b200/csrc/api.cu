@@ -62,10 +62,10 @@ struct moe_ctx {
     uint8_t *down_pass;     // [E][DOWN_PASS_STRIDE] ... of each down weight block
     unsigned int *err;
     unsigned long long wait_limit_ns;
-    // B tensor maps, one per token-block height (8 * (i + 1) rows), made on first use
-    CUtensorMap map_xq[GEMM_NB_MAX / 8];
-    CUtensorMap map_hq[GEMM_NB_MAX / 8];
-    bool have_xq[GEMM_NB_MAX / 8], have_hq[GEMM_NB_MAX / 8];
+    // B tensor maps, one per token-block height (16 * (i + 1) rows), made on first use
+    CUtensorMap map_xq[GEMM_NB_MAX / 16];
+    CUtensorMap map_hq[GEMM_NB_MAX / 16];
+    bool have_xq[GEMM_NB_MAX / 16], have_hq[GEMM_NB_MAX / 16];
     const void *w13_ptr;
     CUtensorMap map_w13;
     const void *w2_ptr;
@@ -121,8 +121,8 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     int rc = plan_gemm(p, mode, T, top_k, d, F, E, P_max, c->num_sms, &grid, &smem);
     if (rc) return rc;
     // the cached B maps of this token-block height
-    if (p.nb_rows < 8 || p.nb_rows > GEMM_NB_MAX || p.nb_rows % 8) return MOE_ERR_ARG;
-    const int bi = p.nb_rows / 8 - 1;
+    if (p.nb_rows < 16 || p.nb_rows > GEMM_NB_MAX || p.nb_rows % 16) return MOE_ERR_ARG;
+    const int bi = p.nb_rows / 16 - 1;
     if (mode == MODE_UP) {
         if (codes != c->w13_ptr) {
             if (p.K_main >= 128 && !encode_a_up(&c->map_w13, codes, E, F, d, p.K_main)) return MOE_ERR_CUDA;

@@ -209,15 +209,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         tmem_alloc(tmem_base_s, 512);
         tmem_relinquish();
     }
-    if (p.stacked) {
-        // the zero rows of the stacked B slots (past 3 NB, up to the MMA width), which no copy writes
-        const int z0 = 3 * NB * 128, z_bytes = b_stage - z0;
-        for (int i = threadIdx.x; i < NS * (z_bytes / 16); i += blockDim.x) {
-            const int sl = i / (z_bytes / 16), o = i - sl * (z_bytes / 16);
-            *reinterpret_cast<uint4 *>(b_ring + sl * b_stage + z0 + 16 * o) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-    }
     // The routing arrays come from the group kernel and the B operand from the
     // kernel before this one.  The gate/up GEMM follows the group kernel and
     // waits for it here.  The down GEMM follows the gate/up GEMM, which starts
@@ -367,8 +358,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         uint32_t ph = 0;
         long long issued = 0;
         bool ok = true;
-        // bytes one copy brings: the block's rows of its planes (a stacked slot's zero rows are not copied)
-        const uint32_t b_bytes = (uint32_t)(gemm_b_planes(p.stacked) * NB * 128);
+        const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
@@ -415,7 +405,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             Work t;
             work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
             const int n_it = SFI ? n_st : n_st * item_passes(p, t);
-            const uint32_t n = stacked ? (uint32_t)gemm_stacked_n(NB) : (uint32_t)t.n_mma;
+            const uint32_t n = stacked ? (uint32_t)(3 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
             // E8M0 scales, M >> 4; K block kb of a stage takes scale byte kb (fields at 4 and 29)
             const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
@@ -778,27 +768,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 // the sum over the MMA warps' accumulators and, stacked, their hi, lo and lo2 thirds
                 for (int mw = 0; mw < n_mma_warps; ++mw) {
                     const uint32_t d_tmem = lane_base + (uint32_t)((mw * n_dbuf + db) * d_cols);
-                    if (p.stacked && NB == 8) {
-                        // columns hi 0..7 | lo 8..15 | lo2 16..23 | zeros: two 16-column loads at
-                        // 16-aligned columns (c0 is 0: a block of 8 is one chunk)
-                        uint32_t v0[16], v1[16];
-                        tmem_ld16(d_tmem, v0);
-                        tmem_ld16(d_tmem + 16u, v1);
+                    for (int half = 0; half < (p.stacked ? 3 : 1); ++half) {
+                        uint32_t v[16];
+                        tmem_ld16(d_tmem + (uint32_t)(half * NB + c0), v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            acc[i] += __uint_as_float(v0[i]);
-                            acc[i] += __uint_as_float(v0[8 + i]);
-                            acc[i] += __uint_as_float(v1[i]);
-                        }
-                    } else {
-                        for (int half = 0; half < (p.stacked ? 3 : 1); ++half) {
-                            uint32_t v[16];
-                            tmem_ld16(d_tmem + (uint32_t)(half * NB + c0), v);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
-                        }
+                        for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
                     }
                 }
                 if (SFI && c0 + 32 >= t.n_mma) release();

@@ -87,11 +87,9 @@ inline int round_up_128(int v) { return (v + 127) / 128 * 128; }
 // Token rows per GEMM work item.  Decode-sized batches (T <= 64) use blocks of
 // 16 rows: their three terms stack into one MMA of N = 48; experts then rarely
 // hold more than one block, and an expert with more tokens takes extra blocks
-// whose weight re-reads hit L2.  (Blocks of 8 -- an MMA of N = 32 over 24 rows
-// and 8 zero rows, a 4 KB slot and one more ring stage -- measured slower on
-// both decode shapes.)  Larger batches use the smallest multiple of 16 that
-// holds every token (an expert receives each token at most once), capped at
-// GEMM_NB_MAX.
+// whose weight re-reads hit L2.  Larger batches use the smallest multiple of 16
+// that holds every token (an expert receives each token at most once), capped
+// at GEMM_NB_MAX.
 inline int token_block_rows(int T) {
     if (T <= 64) return 16;
     int nb = ((T > 0 ? T : 1) + 15) / 16 * 16;

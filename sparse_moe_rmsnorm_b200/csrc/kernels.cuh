@@ -99,8 +99,7 @@ struct GemmParams {
     int E;
     int MB;                     // weight blocks per expert: F/64 (UP) or ceil(d/128) (DOWN)
     int nb_rows;                // token rows per work item (multiple of 16, <= GEMM_NB_MAX)
-    int stacked;                // 1: one MMA covers the hi, lo and lo2 rows (N = 3 nb_rows rounded up to 16);
-                                //    0: one MMA per term
+    int stacked;                // 1: one MMA covers the hi, lo and lo2 rows (N = 3 nb_rows); 0: one MMA per term
     int n_stages;               // shared-memory ring depth (and TMEM scale-factor ring depth when !sf_item)
     int sf_item;                // 1: a work item's scale factors are written to TMEM once, before its first
                                 //    stage, and two MMA warps take alternate stages (decode-sized blocks);
@@ -166,16 +165,11 @@ __host__ __device__ inline int gemm_num_barriers(int n_stages) {
     return 2 * n_stages + 4 + 4 + 2 + 2 + 4 + 4 + 2;
 }
 
-// MMA width of a stacked block: its hi, lo and lo2 rows (3 nb_rows), rounded up to the
-// tensor core's N granularity of 16; the rows past 3 nb_rows are zeros
-__host__ __device__ inline int gemm_stacked_n(int nb_rows) { return (3 * nb_rows + 15) / 16 * 16; }
-// Planes one B copy brings: hi, lo and lo2 (stacked); hi and lo, or lo2 and an empty plane
-// in a lo2 pass
+// B ring slot: the token block's hi, lo and lo2 rows (stacked) or two planes (hi and lo, or lo2
+// and an empty plane in a lo2 pass)
 __host__ __device__ inline int gemm_b_planes(int stacked) { return stacked ? 3 : 2; }
-// B ring slot: the token block's hi, lo and lo2 rows and the zero rows after them (stacked),
-// or two planes (hi and lo, or lo2 and an empty plane in a lo2 pass)
 __host__ __device__ inline int gemm_b_stage_bytes(int nb_rows, int stacked) {
-    return (stacked ? gemm_stacked_n(nb_rows) : 2 * nb_rows) * 128;
+    return gemm_b_planes(stacked) * nb_rows * 128;
 }
 
 __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, int stacked, int n_stages,
@@ -201,9 +195,7 @@ __host__ __device__ inline GemmSmem gemm_smem_plan(int K, int E, int nb_rows, in
 // ring of scale-factor slots.  Per-item mode: accumulators [2 MMA warps] (one
 // buffer each), then two item regions of 8 columns per stage (A at +0, B at +4).
 constexpr int GEMM_SFI_COLS = 8;
-__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) {
-    return stacked ? gemm_stacked_n(nb_rows) : nb_rows;
-}
+__host__ __device__ inline int gemm_d_cols(int nb_rows, int stacked) { return stacked ? 3 * nb_rows : nb_rows; }
 __host__ __device__ inline int gemm_tmem_cols(int nb_rows, int stacked, int n_stages) {
     return 2 * gemm_d_cols(nb_rows, stacked) + GEMM_SF_COLS * n_stages;
 }
