@@ -16,6 +16,9 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+bool route_group_small_fits(const RouteParams &p);
+cudaError_t launch_route_group_small(const RouteParams &rp, const GroupParams &gp, unsigned int *bar,
+                                     unsigned long long wait_limit_ns, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
@@ -179,6 +182,55 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     return cuda_status(launch_expert_gemm(mode, p, grid, smem, stream));
 }
 
+
+RouteParams route_params(moe_ctx *c, int T, const uint16_t *x, const uint16_t *norm_scale, const uint16_t *router_w,
+                         const float *router_b, int top_k) {
+    RouteParams p;
+    p.x = x;
+    p.norm_scale = norm_scale;
+    p.router_w = router_w;
+    p.router_b = router_b;
+    p.T = T;
+    p.d = c->shape.d_model;
+    p.E = c->shape.n_experts;
+    p.k = top_k;
+    p.eps = c->shape.eps;
+    p.xn = c->xn;
+    p.topk_idx = c->topk_idx;
+    p.topk_w = c->topk_w;
+    p.logits = c->logits;
+    p.tok_done = c->tok_done;
+    return p;
+}
+
+GroupParams group_params(moe_ctx *c, int T, int top_k) {
+    GroupParams p;
+    p.topk_idx = c->topk_idx;
+    p.topk_w = c->topk_w;
+    p.P = T * top_k;
+    p.k = top_k;
+    p.E = c->shape.n_experts;
+    p.nb_rows = token_block_rows(T);
+    p.counts = c->counts;
+    p.offsets = c->offsets;
+    p.tiles = c->tiles;
+    p.row_token = c->row_token;
+    p.row_w = c->row_w;
+    p.pair_row = c->pair_row;
+    p.err = c->err;
+    p.xn = c->xn;
+    p.xq = c->xq;
+    p.xsf = c->xsf;
+    p.P_max = c->shape.T_max * c->shape.top_k;
+    p.d = c->shape.d_model;
+    p.Kd = c->Kd;
+    return p;
+}
+
+// the grid barrier words of the decode-sized route + group launch: [count, generation], in the
+// error word's slot (zero at creation; moe_sync_status clears the slot after an error)
+unsigned int *route_group_barrier(moe_ctx *c) { return c->err + 8; }
+
 }  // namespace
 
 extern "C" {
@@ -274,49 +326,15 @@ int moe_route(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *norm_scale
     if (rc) return rc;
     if (T == 0) return MOE_OK;
     if (!aligned16(x) || !aligned16(norm_scale) || !aligned16(router_w) || !aligned16(router_b)) return MOE_ERR_ARG;
-    RouteParams p;
-    p.x = x;
-    p.norm_scale = norm_scale;
-    p.router_w = router_w;
-    p.router_b = router_b;
-    p.T = T;
-    p.d = c->shape.d_model;
-    p.E = c->shape.n_experts;
-    p.k = top_k;
-    p.eps = c->shape.eps;
-    p.xn = c->xn;
-    p.topk_idx = c->topk_idx;
-    p.topk_w = c->topk_w;
-    p.logits = c->logits;
-    p.tok_done = c->tok_done;
-    return cuda_status(launch_route(p, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_route(route_params(c, T, x, norm_scale, router_w, router_b, top_k),
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 int moe_group(moe_ctx_t *c, int T, int top_k, void *stream) {
     int rc = check_call(c, T, top_k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    GroupParams p;
-    p.topk_idx = c->topk_idx;
-    p.topk_w = c->topk_w;
-    p.P = T * top_k;
-    p.k = top_k;
-    p.E = c->shape.n_experts;
-    p.nb_rows = token_block_rows(T);
-    p.counts = c->counts;
-    p.offsets = c->offsets;
-    p.tiles = c->tiles;
-    p.row_token = c->row_token;
-    p.row_w = c->row_w;
-    p.pair_row = c->pair_row;
-    p.err = c->err;
-    p.xn = c->xn;
-    p.xq = c->xq;
-    p.xsf = c->xsf;
-    p.P_max = c->shape.T_max * c->shape.top_k;
-    p.d = c->shape.d_model;
-    p.Kd = c->Kd;
-    return cuda_status(launch_group(p, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_group(group_params(c, T, top_k), static_cast<cudaStream_t>(stream)));
 }
 
 int moe_expert_up(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
@@ -369,8 +387,16 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
         !aligned16(b2) || !aligned16(norm_scale) || !aligned16(y))
         return MOE_ERR_ARG;
     if (y == x) return MOE_ERR_ARG;
-    if ((rc = moe_route(c, T, x, norm_scale, router_w, router_b, top_k, stream))) return rc;
-    if ((rc = moe_group(c, T, top_k, stream))) return rc;
+    const RouteParams rp = route_params(c, T, x, norm_scale, router_w, router_b, top_k);
+    if (route_group_small_fits(rp)) {
+        // decode-sized batches: route and group in one launch (the same outputs as the two stages)
+        if (launch_route_group_small(rp, group_params(c, T, top_k), route_group_barrier(c), c->wait_limit_ns,
+                                     static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        if ((rc = moe_route(c, T, x, norm_scale, router_w, router_b, top_k, stream))) return rc;
+        if ((rc = moe_group(c, T, top_k, stream))) return rc;
+    }
     if ((rc = moe_expert_up(c, T, top_k, w13_codes, w13_scales, b13, w2_scales, stream))) return rc;
     if ((rc = moe_expert_down(c, T, top_k, w2_codes, w2_scales, b2, stream))) return rc;
     return moe_finalize(c, T, top_k, x, y, topk_idx_out, topk_w_out, stream);
@@ -391,7 +417,8 @@ int moe_sync_status(moe_ctx_t *c, void *stream) {
     if (cudaMemcpyAsync(&err, c->err, sizeof err, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
     if (err) {
-        if (cudaMemsetAsync(c->err, 0, sizeof err, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        // the error word and the grid barrier words beside it (a barrier that ran out is left mid-count)
+        if (cudaMemsetAsync(c->err, 0, 64, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
             return MOE_ERR_CUDA;
         return MOE_ERR_TIMEOUT;
     }

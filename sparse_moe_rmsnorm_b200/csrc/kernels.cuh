@@ -33,7 +33,8 @@ enum : unsigned int {
     ERR_WAIT_UP = 1u,      // a bounded wait ran out in the gate/up GEMM
     ERR_WAIT_DOWN = 2u,    // ... in the down GEMM
     ERR_WAIT_SELFTEST = 4u,
-    ERR_ROUTING = 8u       // an expert index out of range reached the grouping
+    ERR_ROUTING = 8u,      // an expert index out of range reached the grouping
+    ERR_WAIT_ROUTE = 16u   // the grid barrier of the decode-sized route + group launch ran out
 };
 
 struct RouteParams {

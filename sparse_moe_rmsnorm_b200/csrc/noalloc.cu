@@ -28,6 +28,9 @@
 namespace moe {
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+bool route_group_small_fits(const RouteParams &p);
+cudaError_t launch_route_group_small(const RouteParams &rp, const GroupParams &gp, unsigned int *bar,
+                                     unsigned long long wait_limit_ns, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pair_row, uint16_t *y, int T, int d, int k,
                            cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
@@ -168,9 +171,10 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     CUtensorMap map_xq, map_hq;
     if (!encode_bq(&map_xq, xq, (int)P, Kd, nb, planes) || !encode_bq(&map_hq, hq, (int)P, Kf, nb, planes))
         return MOE_ERR_CUDA;
-    // the error word and the route kernel's per-token counters must start at zero
-    // on every call (the array keeps whatever the previous call, of any shape, left)
-    if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    // the error word with the grid barrier words beside it, and the route kernel's per-token
+    // counters, must start at zero on every call (the array keeps whatever the previous call,
+    // of any shape, left)
+    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemsetAsync(tok_done, 0, (size_t)T * sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
 
     RouteParams rp;
@@ -188,7 +192,6 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     rp.topk_w = topk_w;
     rp.logits = logits;
     rp.tok_done = tok_done;
-    if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     GroupParams gp;
     gp.topk_idx = topk_idx;
@@ -210,7 +213,13 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.P_max = (int)P;
     gp.d = d;
     gp.Kd = Kd;
-    if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (route_group_small_fits(rp)) {
+        // route and group in one launch; its grid barrier words sit after the error word
+        if (launch_route_group_small(rp, gp, err + 8, 2000000000ull, s) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_group(gp, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
 
     rc = launch_gemm_stage(MODE_UP, T, k, d, F, E, num_sms, w13_codes, w13_scales, b13, &map_xq, xsf, counts,
                            offsets, tiles, row_token, row_w, hq, hsf, orows, err, s);

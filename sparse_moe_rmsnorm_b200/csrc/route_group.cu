@@ -647,6 +647,227 @@ __global__ void __launch_bounds__(256) encode_tokens_kernel(const GroupParams p,
     }
 }
 
+// ------------------------------- route and group, decode-sized, one launch
+//
+// T <= RGS_MAX_T tokens: a CTA per token, 16 warps.  The token's RMSNorm and its
+// E logits take route_small_kernel's arithmetic (the same values), warp w taking
+// experts w, w + 16, ...; then the top-k and the softmax over the chosen, and xn
+// to global memory.  A grid-wide barrier follows: a counter the last CTA to
+// arrive resets and a generation word it then advances, with a bounded wait (a
+// CTA per token fits the GPU in one wave, so every CTA is resident before any
+// waits for long).  After it every CTA computes the grouping of all T k pairs in
+// shared memory, in group_permute_kernel's stable order (by expert, then pair):
+// per-warp match counts, a scan over warps, a scan over experts.  CTA 0 writes
+// counts, offsets and tiles; each CTA writes its own token's k pairs -- their
+// row_token, row_w and pair_row entries -- and the three E4M3 planes of its xn
+// into those k rows (quant_rows_part).  The outputs equal those of
+// route_small_kernel followed by group_permute_kernel, bit for bit.
+constexpr int RGS_MAX_T = 64;
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(512) route_group_small_kernel(const RouteParams rp, const GroupParams gp,
+                                                                unsigned int *bar, unsigned long long wait_limit_ns) {
+    __shared__ float xs[ROUTE_SMALL_CHUNKS * 256];
+    __shared__ float red[16];
+    __shared__ float lg[256];
+    __shared__ int wcnt[16][257];
+    __shared__ int off_s[257];
+    __shared__ int pos_s[8];
+    __shared__ int go_s;
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d = rp.d, E = rp.E, k = rp.k;
+    const int nch = d / 8;
+    for (int i = threadIdx.x; i < 16 * 257; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    if (threadIdx.x < 8) pos_s[threadIdx.x] = -1;
+    pdl_wait();
+    pdl_trigger();
+
+    // ---- RMSNorm of token t (route_small_kernel's arithmetic): thread u owns chunks u and u + 512
+    float f[2][8], sc[2][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c = threadIdx.x + 512 * h;
+        if (c < nch) {
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(rp.x + (size_t)t * d) + c), f[h]);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(rp.norm_scale) + c), sc[h]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ss += f[h][q] * f[h][q];
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tot += red[i];
+    const float inv_rms = 1.0f / sqrtf(tot / (float)d + rp.eps);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c = threadIdx.x + 512 * h;
+        if (c < nch) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float v = f[h][q] * inv_rms * sc[h][q];
+                f[h][q] = v;
+                xs[8 * c + q] = v;
+            }
+            float4 *xo = reinterpret_cast<float4 *>(rp.xn + (size_t)t * d + 8 * c);
+            xo[0] = make_float4(f[h][0], f[h][1], f[h][2], f[h][3]);
+            xo[1] = make_float4(f[h][4], f[h][5], f[h][6], f[h][7]);
+        }
+    }
+    __syncthreads();
+
+    // ---- logits of experts warp, warp + 16, ... (route_small_kernel's per-warp sum)
+    for (int e = warp; e < E; e += 16) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < ROUTE_SMALL_CHUNKS; ++i) {
+            const int c = lane + 32 * i;
+            if (c < nch) {
+                float w8[8];
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(rp.router_w + (size_t)e * d) + c), w8);
+                const float4 a = *reinterpret_cast<const float4 *>(xs + 8 * c);
+                const float4 b = *reinterpret_cast<const float4 *>(xs + 8 * c + 4);
+                acc = fmaf(a.x, w8[0], acc);
+                acc = fmaf(a.y, w8[1], acc);
+                acc = fmaf(a.z, w8[2], acc);
+                acc = fmaf(a.w, w8[3], acc);
+                acc = fmaf(b.x, w8[4], acc);
+                acc = fmaf(b.y, w8[5], acc);
+                acc = fmaf(b.z, w8[6], acc);
+                acc = fmaf(b.w, w8[7], acc);
+            }
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) lg[e] = acc + rp.router_b[e];
+    }
+    __syncthreads();
+    if (warp == 0) topk_softmax_warp(lg, E, k, t, rp.topk_idx, rp.topk_w, lane);
+
+    // ---- grid-wide barrier: every token's top-k (and xn) written
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned int gen = ld_acquire_gpu(bar + 1);    // before arriving: the last arrival advances it
+        const unsigned int n = atomicAdd(bar, 1u);
+        int ok = 1;
+        if (n == gridDim.x - 1) {
+            atomicExch(bar, 0u);
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            const uint64_t start = globaltimer_ns();
+            while (ld_acquire_gpu(bar + 1) == gen) {
+                if (globaltimer_ns() - start > wait_limit_ns) {
+                    atomicOr(gp.err, ERR_WAIT_ROUTE);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        go_s = ok;
+    }
+    __syncthreads();
+    if (!go_s) return;
+
+    // ---- the grouping of all P pairs (pair i = token i / k, slot i % k), one pair per thread
+    const int P = gp.P;
+    const int i = threadIdx.x;
+    int e_i = -1;
+    if (i < P) {
+        e_i = __ldcg(gp.topk_idx + i);
+        if (e_i < 0 || e_i >= E) {
+            if (t == 0) atomicOr(gp.err, ERR_ROUTING);
+            e_i = -1;
+        }
+    }
+    const unsigned m = __match_any_sync(0xffffffffu, e_i);
+    if (e_i >= 0 && lane == __ffs(m) - 1) wcnt[warp][e_i] = __popc(m);
+    __syncthreads();
+    if ((int)threadIdx.x < E) {
+        const int e = threadIdx.x;
+        int s = 0;
+        for (int w = 0; w < 16; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = s;
+            s += c;
+        }
+        if (t == 0) gp.counts[e] = s;
+        off_s[e] = s;   // total for now
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // exclusive scans of counts and of token blocks; lane owns 8 experts
+        int cnt[8], blk[8];
+        int cs = 0, bs = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane * 8 + c;
+            cnt[c] = e < E ? off_s[e] : 0;
+            blk[c] = (cnt[c] + gp.nb_rows - 1) / gp.nb_rows;
+            cs += cnt[c];
+            bs += blk[c];
+        }
+        int ci = cs, bi = bs;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, ci, o);
+            const int b = __shfl_up_sync(0xffffffffu, bi, o);
+            if (lane >= o) {
+                ci += a;
+                bi += b;
+            }
+        }
+        int co = ci - cs, bo = bi - bs;   // exclusive
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int e = lane * 8 + c;
+            if (e < E) {
+                off_s[e] = co;
+                if (t == 0) {
+                    gp.offsets[e] = co;
+                    gp.tiles[e] = bo;
+                }
+            }
+            co += cnt[c];
+            bo += blk[c];
+        }
+        if (lane == 31 && t == 0) {
+            gp.offsets[E] = ci;
+            gp.tiles[E] = bi;
+        }
+    }
+    __syncthreads();
+    // this token's pairs: their rows and permutation entries
+    if (e_i >= 0 && i >= t * k && i < t * k + k) {
+        const int pos = off_s[e_i] + wcnt[warp][e_i] + __popc(m & ((1u << lane) - 1u));
+        pos_s[i - t * k] = pos;
+        gp.row_token[pos] = t;
+        gp.row_w[pos] = __ldcg(gp.topk_w + i);
+        gp.pair_row[i] = pos;
+    }
+    __syncthreads();
+    // the token's three E4M3 planes into its k rows, a warp per 32 blocks of 32 elements
+    const int parts = (gp.Kd / 32 + 31) / 32;
+    if (warp < parts) {
+        int rows[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int n_rows = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q < k && pos_s[q] >= 0) rows[n_rows++] = pos_s[q];
+        quant_rows_part(gp, rows, n_rows, t, warp * 32, lane);
+    }
+}
+
 // --------------------------------------------------------------- combine
 //
 // y[t] = bf16(x[t] + sum_i o[pair_row[t*k + i]]) in fp32, the k weighted
@@ -762,6 +983,17 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(route_fma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(route_fma_kernel, dim3((p.T + RF_TOK - 1) / RF_TOK), dim3(RF_THREADS), smem, s, p);
+}
+
+// Route and group of a decode-sized batch in one launch; false when the batch is
+// not one (the caller then launches the two stages).
+bool route_group_small_fits(const RouteParams &p) {
+    return p.T >= 1 && p.T <= RGS_MAX_T && p.d <= ROUTE_SMALL_CHUNKS * 256 && p.E <= 256 && p.k <= 8;
+}
+
+cudaError_t launch_route_group_small(const RouteParams &rp, const GroupParams &gp, unsigned int *bar,
+                                     unsigned long long wait_limit_ns, cudaStream_t s) {
+    return launch_pdl(route_group_small_kernel, dim3(rp.T), dim3(512), 0, s, rp, gp, bar, wait_limit_ns);
 }
 
 // Pairs above which the grouping and the token-major encoding run as two kernels.

@@ -388,6 +388,48 @@ def test_up_stage_h_encoding(T, d, F, E, k):
     m.close()
 
 
+# moe_forward routes and groups a decode-sized batch (T <= 64, d_model <= 3072) in one launch with a
+# grid-wide barrier; the stage calls run the two kernels.  Same inputs, same outputs, bit for bit:
+# routing, the grouping arrays, the E4M3 operand rows and y.
+@pytest.mark.parametrize("T,d,F,E,k", [(1, 128, 128, 8, 4), (17, 192, 320, 5, 2), (32, 2880, 2880, 32, 4),
+                                       (64, 512, 256, 128, 4), (40, 512, 256, 16, 8), (64, 3072, 128, 256, 8),
+                                       (9, 64, 64, 1, 1)])
+def test_decode_route_group_launch_equals_the_stages(T, d, F, E, k):
+    inp = custom_layer(T=T, d=d, F=F, E=E, k=k, seed=7 * T + E)
+    w = moe.MoEWeights.from_numpy(inp)
+    x = _bf16_dev(inp["x"])
+    m = moe.MoE(T, d, F, E, k)
+    names = ("topk_idx", "topk_w", "counts", "offsets", "tiles", "row_token", "row_w", "pair_row", "xn",
+             "xperm", "xsf")
+    P = T * k
+    y_fused = torch.empty_like(x)
+    m.forward(x, w, y=y_fused)
+    fused = {n: m.workspace(n, T).cpu().numpy() for n in names}
+    y_stages = torch.empty_like(x)
+    moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
+    moe.moe_group(m.ctx, T, k)
+    moe.moe_expert_up(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13, w.w2_scales)
+    moe.moe_expert_down(m.ctx, T, k, w.w2_codes, w.w2_scales, w.b2)
+    moe.moe_finalize(m.ctx, T, k, x, y_stages)
+    staged = {n: m.workspace(n, T).cpu().numpy() for n in names}
+    assert m.sync_status() == moe.MOE_OK
+    for n in names:
+        a, b = fused[n], staged[n]
+        if n == "xperm":
+            a, b = a[:, :P], b[:, :P]
+        elif n == "xsf":
+            a, b = a[:, :, :P], b[:, :, :P]
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8)), n
+    assert torch.equal(y_fused.view(torch.int16), y_stages.view(torch.int16))
+    # and the block against the oracle
+    ref = oracle.moe_forward(inp, k, 1e-5)
+    yf = y_fused.float().cpu().numpy().astype(np.float64)
+    idx = fused["topk_idx"]
+    res = compare_block(yf, idx, fused["topk_w"], ref, k, E)
+    assert res["ok"], res
+    m.close()
+
+
 def test_decode_blocks_several_per_expert():
     """Decode-sized token blocks when the router sends most tokens to a few experts: those experts
     take several blocks each, the last one ragged."""
