@@ -35,12 +35,13 @@ L2_BYTES = 126 * 2 ** 20
 # kernels of one moe_forward: route, group + permute, gate/up GEMM, down GEMM, combine; batches over
 # 64 tokens add the pass plan before the gate/up GEMM, and over 2048 pairs the grouping and the
 # tokens' encoding are two kernels
-def kernels_per_layer(T: int, k: int = 4, d: int = 2880) -> int:
+def kernels_per_layer(T: int, k: int = 4, d: int = 2880, F: int = 2880) -> int:
     """The library's launches per layer step of moe_forward: route + group (one launch for
     decode-sized batches), the pass plan (above 64 tokens), the token encoder (above 2048
-    pairs), the two GEMMs and the combine."""
+    pairs), the two GEMMs (one launch for decode-sized batches with d_model == d_ff) and the
+    combine."""
     if T <= 64 and d <= 3072:
-        return 4
+        return 3 if d == F else 4
     n = 5 if T <= 64 else 6
     return n + 1 if T * k > 2048 else n
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / bf16 tensor roofline"
@@ -513,7 +514,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "gemm_ms_live": {k_: round(v, 4) for k_, v in gemm_ms.items()},
             "experts_touched": cnt["touched"], "clocks": clocks.summary(), "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": kernels_per_layer(T, cfg.k, cfg.d) * layers * args.steps}
+            "gpu_launches": kernels_per_layer(T, cfg.k, cfg.d, cfg.F) * layers * args.steps}
 
 
 EXTRA_WORKLOADS = ("prefill20b", "decode120b", "stack20b")

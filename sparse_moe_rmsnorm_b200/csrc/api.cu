@@ -24,6 +24,7 @@ cudaError_t launch_combine(const uint16_t *x, const float *orows, const int *pai
 cudaError_t launch_decode(const uint8_t *codes, const uint8_t *scales, int R, int K, float *out, cudaStream_t s);
 cudaError_t launch_selftest_wait(unsigned int *err, unsigned long long limit_ns, cudaStream_t s);
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s);
+cudaError_t launch_expert_ffn(const GemmParams &pu, const GemmParams &pd, int grid, int smem, cudaStream_t s);
 cudaError_t launch_pass_plan(const uint8_t *w13_scales, const uint8_t *w2_scales, int E, int d, int F,
                              uint8_t *up_pass, uint8_t *down_pass, cudaStream_t s);
 }  // namespace moe
@@ -63,6 +64,7 @@ struct moe_ctx {
     float *orows;           // weighted expert output per expert-sorted row
     uint8_t *up_pass;       // [E][F/64] passes over K of each gate/up weight block (large batches)
     uint8_t *down_pass;     // [E][DOWN_PASS_STRIDE] ... of each down weight block
+    unsigned int *h_ready;  // [E + P_max/16 + 1] the fused decode GEMM's per-token-block counters
     unsigned int *err;
     unsigned long long wait_limit_ns;
     // B tensor maps, one per token-block height (16 * (i + 1) rows), made on first use
@@ -113,10 +115,12 @@ int check_call(moe_ctx *c, int T, int top_k) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
-                const uint16_t *bias, const uint8_t *w2_scales, cudaStream_t stream) {
+// The parameters, grid and shared memory of one grouped GEMM launch (and, for the
+// gate/up GEMM of large batches, the launch of the pass plan both GEMMs read).
+int gemm_prepare(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
+                 const uint16_t *bias, const uint8_t *w2_scales, cudaStream_t stream, GemmParams &p, int &grid_out,
+                 int &smem_out) {
     const moe_shape_t &s = c->shape;
-    GemmParams p;
     memset(&p, 0, sizeof p);
     const int E = s.n_experts, d = s.d_model, F = s.d_ff;
     const int P_max = s.T_max * s.top_k;
@@ -179,7 +183,37 @@ int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, co
     p.row_w = c->row_w;
     p.err = c->err;
     p.wait_limit_ns = c->wait_limit_ns;
+    grid_out = grid;
+    smem_out = smem;
+    return MOE_OK;
+}
+
+int gemm_launch(moe_ctx *c, int mode, int T, int top_k, const uint8_t *codes, const uint8_t *scales,
+                const uint16_t *bias, const uint8_t *w2_scales, cudaStream_t stream) {
+    GemmParams p;
+    int grid = 0, smem = 0;
+    const int rc = gemm_prepare(c, mode, T, top_k, codes, scales, bias, w2_scales, stream, p, grid, smem);
+    if (rc) return rc;
     return cuda_status(launch_expert_gemm(mode, p, grid, smem, stream));
+}
+
+// Both GEMMs of a decode-sized batch in one launch, when both use per-item scale factors and
+// d_model == d_ff; MOE_ERR_UNSUPPORTED when they do not (the caller launches them apart).
+int ffn_launch(moe_ctx *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
+               const uint16_t *b13, const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+               cudaStream_t stream) {
+    if (c->shape.d_model != c->shape.d_ff) return MOE_ERR_UNSUPPORTED;
+    GemmParams pu, pd;
+    int grid_u = 0, smem_u = 0, grid_d = 0, smem_d = 0;
+    int rc = gemm_prepare(c, MODE_UP, T, top_k, w13_codes, w13_scales, b13, w2_scales, stream, pu, grid_u, smem_u);
+    if (rc) return rc;
+    rc = gemm_prepare(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, nullptr, stream, pd, grid_d, smem_d);
+    if (rc) return rc;
+    if (!pu.sf_item || !pd.sf_item || pu.n_stages != pd.n_stages || smem_u != smem_d) return MOE_ERR_UNSUPPORTED;
+    pu.h_ready = pd.h_ready = c->h_ready;
+    pu.h_target = pd.h_target = 8u * (unsigned)pu.MB;     // every epilogue warp of every gate/up weight block
+    const int grid = grid_u + grid_d < c->num_sms ? grid_u + grid_d : c->num_sms;
+    return cuda_status(launch_expert_ffn(pu, pd, grid, smem_u, stream));
 }
 
 
@@ -224,6 +258,8 @@ GroupParams group_params(moe_ctx *c, int T, int top_k) {
     p.P_max = c->shape.T_max * c->shape.top_k;
     p.d = c->shape.d_model;
     p.Kd = c->Kd;
+    p.h_ready = c->h_ready;
+    p.n_h_ready = c->shape.n_experts + p.P_max / 16 + 1;
     return p;
 }
 
@@ -284,12 +320,13 @@ int moe_init(const moe_shape_t *shape, moe_ctx_t **out) {
                             3 * P * c->Kd, (size_t)(c->Kd / 128) * 2 * P * 4,
                             3 * P * c->Kf, (size_t)(c->Kf / 128) * 2 * P * 4,
                             P * s.d_model * 4, 64, T * E * 4, T * 4, E * (size_t)(s.d_ff / 64),
-                            E * (size_t)DOWN_PASS_STRIDE};
+                            E * (size_t)DOWN_PASS_STRIDE, (E + P / 16 + 1) * 4};
     void **slots[] = {(void **)&c->xn, (void **)&c->topk_idx, (void **)&c->topk_w,
                       (void **)&c->counts, (void **)&c->offsets, (void **)&c->tiles, (void **)&c->row_token,
                       (void **)&c->row_w, (void **)&c->pair_row, (void **)&c->xq, (void **)&c->xsf,
                       (void **)&c->hq, (void **)&c->hsf, (void **)&c->orows, (void **)&c->err,
-                      (void **)&c->logits, (void **)&c->tok_done, (void **)&c->up_pass, (void **)&c->down_pass};
+                      (void **)&c->logits, (void **)&c->tok_done, (void **)&c->up_pass, (void **)&c->down_pass,
+                      (void **)&c->h_ready};
     size_t total = 0;
     for (size_t v : sizes) total += round256(v);
     if (cudaMalloc(&c->ws, total) != cudaSuccess) {
@@ -389,10 +426,15 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
     if (y == x) return MOE_ERR_ARG;
     const RouteParams rp = route_params(c, T, x, norm_scale, router_w, router_b, top_k);
     if (route_group_small_fits(rp)) {
-        // decode-sized batches: route and group in one launch (the same outputs as the two stages)
+        // decode-sized batches: route and group in one launch, then both GEMMs in one launch (the
+        // same outputs as the stages; the route + group launch zeroes the GEMM launch's counters)
         if (launch_route_group_small(rp, group_params(c, T, top_k), route_group_barrier(c), c->wait_limit_ns,
                                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
             return MOE_ERR_CUDA;
+        rc = ffn_launch(c, T, top_k, w13_codes, w13_scales, b13, w2_codes, w2_scales, b2,
+                        static_cast<cudaStream_t>(stream));
+        if (rc == MOE_OK) return moe_finalize(c, T, top_k, x, y, topk_idx_out, topk_w_out, stream);
+        if (rc != MOE_ERR_UNSUPPORTED) return rc;
     } else {
         if ((rc = moe_route(c, T, x, norm_scale, router_w, router_b, top_k, stream))) return rc;
         if ((rc = moe_group(c, T, top_k, stream))) return rc;

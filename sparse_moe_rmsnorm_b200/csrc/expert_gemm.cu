@@ -62,6 +62,8 @@ constexpr int SF_WORDS = 12;    // B scale words per lane and stage, at most (6 
 
 struct Work {
     int e, mb, p0, n_valid, n_mma;
+    int blk;        // the token block's index over all experts (tiles[e] + block)
+    bool up;        // a gate/up item (always in MODE_UP launches, never in MODE_DOWN ones)
 };
 
 __device__ __forceinline__ void work_of(int w, const int *tiles_s, const int *counts_s, const int *offsets_s, int E,
@@ -78,6 +80,7 @@ __device__ __forceinline__ void work_of(int w, const int *tiles_s, const int *co
     t.e = e;
     t.mb = local / nblk;
     const int nb = local - t.mb * nblk;
+    t.blk = tiles_s[e] + nb;
     t.p0 = offsets_s[e] + nb * nb_rows;
     t.n_valid = min(nb_rows, counts_s[e] - nb * nb_rows);
     // never past the row buffers, even for routing arrays that do not match (the down
@@ -110,30 +113,48 @@ __device__ __forceinline__ int item_passes(const GemmParams &p, const Work &t) {
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 // Source row (0..127) in the work item's scale buffer of tile row r (the A
-// row in shared memory and TMEM lane r).  UP: the buffer holds the 64 gate rows
-// then the 64 linear rows; tile row 32q + l is gate row 16q + l (l < 16) or
+// row in shared memory and TMEM lane r).  Gate/up: the buffer holds the 64 gate
+// rows then the 64 linear rows; tile row 32q + l is gate row 16q + l (l < 16) or
 // linear row 16q + l - 16.
-template <int MODE>
-__device__ __forceinline__ int tile_scale_row(int r) {
-    if (MODE == MODE_UP) {
+__device__ __forceinline__ int tile_scale_row(bool up, int r) {
+    if (up) {
         const int q = r >> 5, l = r & 31;
         return l < 16 ? 16 * q + l : 64 + 16 * q + (l - 16);
     }
     return r;
 }
 
-// Weight row of tile row r in the expert's row space (UP: [0, 2F); DOWN: [0, d)).
-template <int MODE>
-__device__ __forceinline__ int tile_weight_row(int r, int mb, int F) {
-    if (MODE == MODE_UP) {
+// Weight row of tile row r in the expert's row space (gate/up: [0, 2F); down: [0, d)).
+__device__ __forceinline__ int tile_weight_row(bool up, int r, int mb, int F) {
+    if (up) {
         const int q = r >> 5, l = r & 31;
         return l < 16 ? mb * 64 + 16 * q + l : F + mb * 64 + 16 * q + (l - 16);
     }
     return mb * GEMM_BM + r;
 }
 
+// Bounded wait until a counter another CTA releases reaches `target` (as mbar_wait:
+// false when the CTA has aborted or the wait ran out, which aborts the CTA).
+__device__ __forceinline__ bool wait_count(const unsigned int *ctr, unsigned int target, const WaitCtl &w) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        __nanosleep(128);
+        if (ld_acquire_gpu(ctr) >= target) return true;
+        if (*w.abort) return false;
+        if (globaltimer_ns() - start > w.limit_ns) {
+            *w.abort = 1;
+            atomicOr(w.err, w.err_bit);
+            return false;
+        }
+    }
+}
+
+// p: the launch's GEMM (MODE_UP, MODE_DOWN) or, in MODE_FFN, the gate/up GEMM; p2: the down
+// GEMM in MODE_FFN (the same as p otherwise).  MODE_FFN needs d_model == d_ff (one K for both).
 template <int MODE, bool SFI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __grid_constant__ GemmParams p,
+                                                                      const __grid_constant__ GemmParams p2) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NS = p.n_stages;
@@ -217,7 +238,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     // B producer and the loads of B scale words wait for the gate/up GEMM.
     // Its weight copies and weight scales start while the gate/up GEMM's last
     // CTAs finish.
-    if constexpr (MODE == MODE_UP) pdl_wait();
+    if constexpr (MODE == MODE_UP || MODE == MODE_FFN) pdl_wait();
     pdl_trigger();
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
         counts_s[i] = i < p.E ? __ldcg(p.counts + i) : 0;
@@ -228,8 +249,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
-    const int total = p.MB * tiles_s[p.E];
-    const WaitCtl wc{abort_s, p.err, MODE == MODE_UP ? (unsigned)ERR_WAIT_UP : (unsigned)ERR_WAIT_DOWN,
+    // work items: MODE_FFN runs the gate/up items [0, W_up), then the down items
+    const GemmParams &pd = MODE == MODE_FFN ? p2 : p;    // the down items' GEMM
+    const int W_up = p.MB * tiles_s[p.E];
+    const int total = MODE == MODE_FFN ? W_up + pd.MB * tiles_s[p.E] : W_up;
+    auto item_of = [&](int w, Work &t) {
+        const bool up = MODE == MODE_FFN ? w < W_up : MODE == MODE_UP;
+        const int wl = MODE == MODE_FFN && !up ? w - W_up : w;
+        work_of(wl, tiles_s, counts_s, offsets_s, p.E, up ? p.MB : pd.MB, NB, p.P_max, t);
+        t.up = up;
+    };
+    auto gp_of = [&](const Work &t) -> const GemmParams & { return t.up ? p : pd; };
+    const WaitCtl wc{abort_s, p.err, MODE == MODE_DOWN ? (unsigned)ERR_WAIT_DOWN : (unsigned)ERR_WAIT_UP,
                      p.wait_limit_ns};
 
     if (warp == 0) {
@@ -241,7 +272,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // pass.  The K tail (K not
         // a multiple of 128) is loaded at the start of the item, four rows per
         // lane, and written into its stage's slot here.
-        if (lane == 0 && n_main > 0) tma_prefetch_desc(&p.map_a);
+        if (lane == 0 && n_main > 0) {
+            tma_prefetch_desc(&p.map_a);
+            if (MODE == MODE_FFN) tma_prefetch_desc(&p2.map_a);
+        }
         int slot = 0, sb = 0;
         uint32_t ph = 0, sph = 0;
         long long issued = 0, s_issued = 0;
@@ -267,19 +301,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         };
         Work t;
         if (blockIdx.x < total) {
-            work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
+            item_of(blockIdx.x, t);
             if constexpr (!SFI) ok = load_scales(t);     // per-item mode: the scale-factor warps load them
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             uint4 tail[8];                   // the item's K tail codes (rows lane + 32j)
             auto load_tail = [&]() {
+                const GemmParams &q = gp_of(t);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int wrow = tile_weight_row<MODE>(lane + 32 * j, t.mb, p.F);
+                    const int wrow = tile_weight_row(t.up, lane + 32 * j, t.mb, p.F);
                     tail[2 * j] = tail[2 * j + 1] = make_uint4(0, 0, 0, 0);
-                    if (wrow < p.R) {
+                    if (wrow < q.R) {
                         const uint4 *src = reinterpret_cast<const uint4 *>(
-                            p.codes + ((size_t)t.e * p.R + wrow) * (p.K / 2) + p.K_main / 2);
+                            q.codes + ((size_t)t.e * q.R + wrow) * (p.K / 2) + p.K_main / 2);
                         tail[2 * j] = __ldg(src);
                         tail[2 * j + 1] = __ldg(src + 1);
                     }
@@ -291,7 +326,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             Work tn;
             const bool has_next = w + (int)gridDim.x < total;
             if (has_next) {
-                work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
+                item_of(w + gridDim.x, tn);
                 if constexpr (!SFI) {
                     if (!load_scales(tn)) { ok = false; break; }
                 }
@@ -303,10 +338,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 if (st < n_main) {
                     // the unpacked-type TMA counts the packed bytes: 128 rows x 64
                     mbar_arrive_expect_tx_w(&full[slot], 128u * 64u);
-                    if (MODE == MODE_UP)
+                    if (t.up)
                         tma_load_5d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, 0, 0, 4 * t.mb, t.e);
                     else
-                        tma_load_3d_w(adst, &p.map_a, &full[slot], st * GEMM_KS, t.mb * GEMM_BM, t.e);
+                        tma_load_3d_w(adst, &pd.map_a, &full[slot], st * GEMM_KS, t.mb * GEMM_BM, t.e);
                 } else {
                     // K tail of rows lane + 32j: 2 x 16 code bytes -> the first four
                     // 16-byte units of the row (8 code bytes each, the rest zero),
@@ -352,7 +387,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         // Per stage one TMA box: the token block's rows of two planes (hi, lo) or,
         // stacked, of all three (hi, lo, lo2); in a lo2 pass the box starts at the
         // lo2 plane (the plane after it lies outside the map and reads as zeros).
-        if (lane == 0) tma_prefetch_desc(&p.map_b);
+        if (lane == 0) {
+            tma_prefetch_desc(&p.map_b);
+            if (MODE == MODE_FFN) tma_prefetch_desc(&p2.map_b);
+        }
         if constexpr (MODE == MODE_DOWN) pdl_wait();     // h comes from the gate/up GEMM
         int slot = 0;
         uint32_t ph = 0;
@@ -361,11 +399,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const uint32_t b_bytes = (uint32_t)b_stage;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
+            item_of(w, t);
+            if (MODE == MODE_FFN && !t.up) {
+                // a down item: its token block's h rows, written by the gate/up items' epilogues
+                // (generic-proxy stores, released per warp), before TMA reads them
+                if (!__all_sync(0xffffffffu, wait_count(p.h_ready + t.blk, p.h_target, wc))) { ok = false; break; }
+                fence_proxy_async_global();
+            }
+            const CUtensorMap *map_b = &gp_of(t).map_b;
             for (int st = 0; st < n_st; ++st) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ph ^ 1, wc))) { ok = false; break; }
                 mbar_arrive_expect_tx_w(&full[slot], b_bytes);
-                tma_load_3d_w(b_ring + slot * b_stage, &p.map_b, &full[slot], st * GEMM_KS, t.p0, 0);
+                tma_load_3d_w(b_ring + slot * b_stage, map_b, &full[slot], st * GEMM_KS, t.p0, 0);
                 ++issued;
                 if (++slot == NS) { slot = 0; ph ^= 1; }
             }
@@ -403,7 +448,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         const bool stacked = SFI || p.stacked;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
+            item_of(w, t);
             const int n_it = SFI ? n_st : n_st * item_passes(p, t);
             const uint32_t n = stacked ? (uint32_t)(3 * NB) : (uint32_t)t.n_mma;
             // kind::mxf8f6f4 descriptor: A E2M1 (5), B E4M3 (0), both K-major, N >> 3,
@@ -534,7 +579,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             if constexpr (MODE == MODE_DOWN) pdl_wait();     // h's scales come from the gate/up GEMM
             if (blockIdx.x < total) {
                 Work t0;
-                work_of(blockIdx.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t0);
+                item_of(blockIdx.x, t0);
 #pragma unroll
                 for (int i = 0; i < SF_PD; ++i)
                     if (i < n_st) load_bsf(t0, i, bw[i]);
@@ -542,7 +587,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         }
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
+            item_of(w, t);
             const int npass = item_passes(p, t);
             if constexpr (!SFI) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], sph, wc))) { ok = false; break; }
@@ -552,8 +597,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             bool row_ok[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                srow[c] = sbase + tile_scale_row<MODE>(32 * c + lane) * KB32;
-                row_ok[c] = MODE == MODE_UP || t.mb * GEMM_BM + 32 * c + lane < p.R;
+                srow[c] = sbase + tile_scale_row(t.up, 32 * c + lane) * KB32;
+                row_ok[c] = t.up || t.mb * GEMM_BM + 32 * c + lane < gp_of(t).R;
             }
             // A words of K stage kst: column c
             auto a_words = [&](int kst, uint32_t *v) {
@@ -577,12 +622,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                 // stage them in shared memory for each other; then each warp writes one
                 // 8-column group (A, B) per stage of its lane quarter and waits once.
                 const int sf_tid = 32 * q + lane;
-                const int run_bytes = MODE == MODE_UP ? 64 * KB32 : min(GEMM_BM, p.R - t.mb * GEMM_BM) * KB32;
+                const GemmParams &gq = gp_of(t);
+                const int run_bytes = t.up ? 64 * KB32 : min(GEMM_BM, gq.R - t.mb * GEMM_BM) * KB32;
                 const int n16 = run_bytes / 16;
-                const int n_words = MODE == MODE_UP ? 2 * n16 : n16;
+                const int n_words = t.up ? 2 * n16 : n16;
                 const uint4 *run0 = reinterpret_cast<const uint4 *>(
-                    p.scales + ((size_t)t.e * p.R + (MODE == MODE_UP ? t.mb * 64 : t.mb * GEMM_BM)) * KB32);
-                const uint4 *run1 = reinterpret_cast<const uint4 *>(p.scales + ((size_t)t.e * p.R + p.F + t.mb * 64) * KB32);
+                    gq.scales + ((size_t)t.e * gq.R + (t.up ? t.mb * 64 : t.mb * GEMM_BM)) * KB32);
+                const uint4 *run1 = reinterpret_cast<const uint4 *>(gq.scales + ((size_t)t.e * gq.R + p.F + t.mb * 64) * KB32);
                 constexpr int SW = (GEMM_SFI_STAGES_MAX * 4 * GEMM_BM / 16 + 127) / 128;   // words per thread, at most
                 uint4 sreg[SW];
 #pragma unroll
@@ -590,22 +636,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     const int wi = sf_tid + 128 * i;
                     sreg[i] = make_uint4(0, 0, 0, 0);
                     if (wi < n16) sreg[i] = __ldg(run0 + wi);
-                    else if (MODE == MODE_UP && wi < n_words) sreg[i] = __ldg(run1 + (wi - n16));
+                    else if (t.up && wi < n_words) sreg[i] = __ldg(run1 + (wi - n16));
                 }
                 if constexpr (MODE == MODE_DOWN) pdl_wait();   // h's scales come from the gate/up GEMM
+                if (MODE == MODE_FFN && !t.up) {
+                    // h's scale words come from this launch's gate/up items of the token block
+                    if (!__all_sync(0xffffffffu, wait_count(p.h_ready + t.blk, p.h_target, wc))) { ok = false; break; }
+                }
                 uint32_t bwr[GEMM_SFI_STAGES_MAX / 4][4];
 #pragma unroll
                 for (int i = 0; i < GEMM_SFI_STAGES_MAX / 4; ++i) {
                     const int st = q + 4 * i;
                     // stacked block: B column c is row 32c + lane of [hi rows | lo rows | lo2 rows]
-                    const uint32_t *bsf = p.b_sf + (size_t)min(st, n_st - 1) * 2 * p.P_max + t.p0;
+                    const uint32_t *bsf = gq.b_sf + (size_t)min(st, n_st - 1) * 2 * p.P_max + t.p0;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int r = 32 * c + lane;
                         const int plane = r / NB;
                         const int j = r - plane * NB;
+                        // (in MODE_FFN h's words were written during this launch: a coherent load)
+                        const uint32_t *src = bsf + (plane == 1 ? (size_t)p.P_max : 0) + j;
                         bwr[i][c] = st < n_st && c < n_sfb && r < 3 * NB && j < t.n_valid
-                                        ? __ldg(bsf + (plane == 1 ? (size_t)p.P_max : 0) + j) : 0x7F7F7F7Fu;
+                                        ? (MODE == MODE_FFN ? __ldcg(src) : __ldg(src)) : 0x7F7F7F7Fu;
                     }
                 }
                 // the staging buffer is free once all four warps have read the last item's words
@@ -646,7 +698,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
             } else {
                 Work tn;
                 const bool has_next = w + (int)gridDim.x < total;
-                if (has_next) work_of(w + gridDim.x, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, tn);
+                if (has_next) item_of(w + gridDim.x, tn);
                 for (int st0 = 0; st0 < n_st && ok; st0 += SF_PD) {
 #pragma unroll
                     for (int i = 0; i < SF_PD; ++i) {
@@ -729,20 +781,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
         uint32_t ex_ph = 0;                  // bit i: phase parity of exchange buffer i
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Work t;
-            work_of(w, tiles_s, counts_s, offsets_s, p.E, p.MB, NB, p.P_max, t);
-            const int wrow = tile_weight_row<MODE>(tl, t.mb, p.F);
-            const bool row_valid = wrow < p.R;
+            item_of(w, t);
+            const GemmParams &gq = gp_of(t);
+            const int wrow = tile_weight_row(t.up, tl, t.mb, p.F);
+            const bool row_valid = wrow < gq.R;
             // (up) h's lo2 plane: always for stacked blocks, else only where the down GEMM may read it
-            bool want_lo2 = MODE == MODE_UP && p.stacked;
-            if (MODE == MODE_UP && !p.stacked && p.down_pass) {
+            bool want_lo2 = t.up && p.stacked;
+            if (t.up && !p.stacked && p.down_pass) {
                 // the expert's row of the down pass table, one byte per lane (two loads)
                 const uint8_t *dp = p.down_pass + (size_t)t.e * DOWN_PASS_STRIDE;
                 const bool two = (lane < p.MB_down && __ldg(dp + lane) > 1) ||
                                  (lane + 32 < p.MB_down && __ldg(dp + lane + 32) > 1);
                 want_lo2 = __any_sync(0xffffffffu, two);
             }
-            const float bias = row_valid ? bf16_to_f32(p.bias[(size_t)t.e * p.R + wrow]) : 0.f;
-            if (MODE == MODE_DOWN) {
+            const float bias = row_valid ? bf16_to_f32(gq.bias[(size_t)t.e * gq.R + wrow]) : 0.f;
+            if (!t.up) {
                 for (int c = lane; c < t.n_valid; c += 32) mval[c] = p.row_w[t.p0 + c];
                 __syncwarp();
             }
@@ -777,7 +830,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
                     }
                 }
                 if (SFI && c0 + 32 >= t.n_mma) release();
-                if (MODE == MODE_UP) {
+                if (t.up) {
                     // SwiGLU: lanes < 16 hold gate rows, lanes >= 16 the linear rows of the
                     // same h rows; lanes < 16 finish columns 0..7, lanes >= 16 columns 8..15
                     const int half = lane >> 4;
@@ -857,11 +910,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             if (c0 + i < t.n_valid)
-                                p.out_rows[(size_t)(t.p0 + c0 + i) * p.R + wrow] = (acc[i] + bias) * mval[c0 + i];
+                                gq.out_rows[(size_t)(t.p0 + c0 + i) * gq.R + wrow] = (acc[i] + bias) * mval[c0 + i];
                     }
                 }
             }
             if (!ok) break;
+            if (MODE == MODE_FFN && t.up) {
+                // this warp's h rows of the token block are written: release them to the down
+                // items (each lane's stores fenced, then one count per warp)
+                fence_proxy_async_global();
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(p.h_ready + t.blk, 1u);
+            }
             if (!released) release();
             if (++db == n_dbuf) { db = 0; dph ^= 1; }
         }
@@ -875,10 +936,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) expert_gemm_kernel(const __gr
     }
 }
 
-template __global__ void expert_gemm_kernel<MODE_UP, false>(const __grid_constant__ GemmParams p);
-template __global__ void expert_gemm_kernel<MODE_UP, true>(const __grid_constant__ GemmParams p);
-template __global__ void expert_gemm_kernel<MODE_DOWN, false>(const __grid_constant__ GemmParams p);
-template __global__ void expert_gemm_kernel<MODE_DOWN, true>(const __grid_constant__ GemmParams p);
+template __global__ void expert_gemm_kernel<MODE_UP, false>(const __grid_constant__ GemmParams p,
+                                                              const __grid_constant__ GemmParams p2);
+template __global__ void expert_gemm_kernel<MODE_UP, true>(const __grid_constant__ GemmParams p,
+                                                             const __grid_constant__ GemmParams p2);
+template __global__ void expert_gemm_kernel<MODE_DOWN, false>(const __grid_constant__ GemmParams p,
+                                                                const __grid_constant__ GemmParams p2);
+template __global__ void expert_gemm_kernel<MODE_DOWN, true>(const __grid_constant__ GemmParams p,
+                                                               const __grid_constant__ GemmParams p2);
+template __global__ void expert_gemm_kernel<MODE_FFN, true>(const __grid_constant__ GemmParams p,
+                                                              const __grid_constant__ GemmParams p2);
 
 // The pass table of the large-block GEMMs: for every gate/up work-item weight
 // block (64 gate rows and their 64 linear rows of W13) and every down weight
@@ -950,16 +1017,25 @@ cudaError_t launch_pass_plan(const uint8_t *w13_scales, const uint8_t *w2_scales
 }
 
 template <int MODE, bool SFI>
-static cudaError_t launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t s) {
+static cudaError_t launch_gemm_t(const GemmParams &p, const GemmParams &p2, int grid, int smem, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, SFI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(expert_gemm_kernel<MODE, SFI>, dim3(grid), dim3(GEMM_THREADS), (size_t)smem, s, p);
+    return launch_pdl(expert_gemm_kernel<MODE, SFI>, dim3(grid), dim3(GEMM_THREADS), (size_t)smem, s, p, p2);
 }
 
 cudaError_t launch_expert_gemm(int mode, const GemmParams &p, int grid, int smem, cudaStream_t s) {
     if (mode == MODE_UP)
-        return p.sf_item ? launch_gemm_t<MODE_UP, true>(p, grid, smem, s) : launch_gemm_t<MODE_UP, false>(p, grid, smem, s);
-    return p.sf_item ? launch_gemm_t<MODE_DOWN, true>(p, grid, smem, s) : launch_gemm_t<MODE_DOWN, false>(p, grid, smem, s);
+        return p.sf_item ? launch_gemm_t<MODE_UP, true>(p, p, grid, smem, s)
+                         : launch_gemm_t<MODE_UP, false>(p, p, grid, smem, s);
+    return p.sf_item ? launch_gemm_t<MODE_DOWN, true>(p, p, grid, smem, s)
+                     : launch_gemm_t<MODE_DOWN, false>(p, p, grid, smem, s);
+}
+
+// Both GEMMs of a decode-sized batch in one launch (per-item scale factors, d_model == d_ff):
+// pu the gate/up GEMM with h_ready / h_target set, pd the down GEMM.
+cudaError_t launch_expert_ffn(const GemmParams &pu, const GemmParams &pd, int grid, int smem, cudaStream_t s) {
+    if (!pu.sf_item || !pd.sf_item || pu.K != pd.K || !pu.h_ready) return cudaErrorInvalidValue;
+    return launch_gemm_t<MODE_FFN, true>(pu, pd, grid, smem, s);
 }
 
 }  // namespace moe

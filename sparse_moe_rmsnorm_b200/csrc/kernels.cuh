@@ -65,6 +65,8 @@ struct GroupParams {
     // the expert-sorted E4M3 terms of the normalised tokens (gate/up B operand)
     const float *xn;            // fp32 [T, d]
     uint8_t *xq;                // [3][P_max][Kd]: hi, lo, lo2 planes
+    unsigned int *h_ready;      // the fused decode GEMM's per-token-block counters, zeroed by the
+    int n_h_ready;              //   decode-sized route + group launch (NULL: none)
     uint32_t *xsf;              // [Kd/128][2][P_max]: scales of the hi (also lo2) and lo planes
     int P_max, d, Kd;
 };
@@ -82,7 +84,10 @@ struct GroupParams {
 // MODE_UP: rows are the gate/linear pairs of W13, epilogue is the clamped
 // SwiGLU, written as the down GEMM's B.  MODE_DOWN: rows are W2's, epilogue
 // writes the routing-weighted expert output rows.
-enum { MODE_UP = 0, MODE_DOWN = 1 };
+// MODE_FFN: both GEMMs of a decode-sized batch in one persistent launch -- the
+// gate/up items, then the down items; a down item waits until every gate/up
+// item of its token block has written its h rows (a counter per token block).
+enum { MODE_UP = 0, MODE_DOWN = 1, MODE_FFN = 2 };
 
 struct GemmParams {
     CUtensorMap map_a;          // E2M1 codes, 16 x 4-bit per 16 bytes in shared memory (unpacked TMA type);
@@ -126,6 +131,10 @@ struct GemmParams {
     float *out_rows;
     unsigned int *err;
     unsigned long long wait_limit_ns;
+    // MODE_FFN: per token block (index tiles[e] + block), the gate/up epilogue warps that have
+    // written their h rows; a down item of the block starts at h_target (8 x gate/up weight blocks)
+    unsigned int *h_ready;
+    unsigned int h_target;
 };
 
 constexpr int GEMM_THREADS = 512;     // 16 warps

@@ -213,6 +213,8 @@ MOE_API int moe_forward_noalloc(int T, int d_model, int d_ff, int n_experts, int
     gp.P_max = (int)P;
     gp.d = d;
     gp.Kd = Kd;
+    gp.h_ready = nullptr;
+    gp.n_h_ready = 0;
     if (route_group_small_fits(rp)) {
         // route and group in one launch; its grid barrier words sit after the error word
         if (launch_route_group_small(rp, gp, err + 8, 2000000000ull, s) != cudaSuccess) return MOE_ERR_CUDA;

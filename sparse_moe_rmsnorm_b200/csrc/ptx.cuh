@@ -262,6 +262,19 @@ __device__ __forceinline__ void tmem_st8v(uint32_t taddr, uint32_t a, uint32_t b
                  : "memory");
 }
 
+// Load with acquire semantics at GPU scope (a flag or counter another CTA releases).
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Order this thread's generic-proxy global-memory accesses with its async-proxy ones
+// (TMA copies of data other CTAs wrote, after acquiring their flag).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to later
 // async-proxy reads (TMA, tcgen05.mma operands).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -664,12 +664,6 @@ __global__ void __launch_bounds__(256) encode_tokens_kernel(const GroupParams p,
 // route_small_kernel followed by group_permute_kernel, bit for bit.
 constexpr int RGS_MAX_T = 64;
 
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __global__ void __launch_bounds__(512) route_group_small_kernel(const RouteParams rp, const GroupParams gp,
                                                                 unsigned int *bar, unsigned long long wait_limit_ns) {
     __shared__ float xs[ROUTE_SMALL_CHUNKS * 256];
@@ -687,6 +681,10 @@ __global__ void __launch_bounds__(512) route_group_small_kernel(const RouteParam
     if (threadIdx.x < 8) pos_s[threadIdx.x] = -1;
     pdl_wait();
     pdl_trigger();
+    // the fused decode GEMM's per-token-block counters start at zero (it runs after this
+    // launch; the wait above orders this after the previous layer step's GEMM)
+    if (t == 0 && gp.h_ready)
+        for (int i = threadIdx.x; i < gp.n_h_ready; i += blockDim.x) gp.h_ready[i] = 0u;
 
     // ---- RMSNorm of token t (route_small_kernel's arithmetic): thread u owns chunks u and u + 512
     float f[2][8], sc[2][8];

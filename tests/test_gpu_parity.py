@@ -389,18 +389,20 @@ def test_up_stage_h_encoding(T, d, F, E, k):
 
 
 # moe_forward routes and groups a decode-sized batch (T <= 64, d_model <= 3072) in one launch with a
-# grid-wide barrier; the stage calls run the two kernels.  Same inputs, same outputs, bit for bit:
-# routing, the grouping arrays, the E4M3 operand rows and y.
+# grid-wide barrier, and (d_model == d_ff) runs both GEMMs in one launch whose down items wait on
+# per-token-block counters; the stage calls run four kernels.  Same inputs, same outputs, bit for
+# bit: routing, the grouping arrays, the E4M3 operand rows, h, the weighted rows and y.
 @pytest.mark.parametrize("T,d,F,E,k", [(1, 128, 128, 8, 4), (17, 192, 320, 5, 2), (32, 2880, 2880, 32, 4),
                                        (64, 512, 256, 128, 4), (40, 512, 256, 16, 8), (64, 3072, 128, 256, 8),
-                                       (9, 64, 64, 1, 1)])
+                                       (9, 64, 64, 1, 1), (64, 2880, 2880, 128, 4), (48, 256, 256, 4, 4),
+                                       (33, 2880, 2880, 32, 4)])
 def test_decode_route_group_launch_equals_the_stages(T, d, F, E, k):
     inp = custom_layer(T=T, d=d, F=F, E=E, k=k, seed=7 * T + E)
     w = moe.MoEWeights.from_numpy(inp)
     x = _bf16_dev(inp["x"])
     m = moe.MoE(T, d, F, E, k)
     names = ("topk_idx", "topk_w", "counts", "offsets", "tiles", "row_token", "row_w", "pair_row", "xn",
-             "xperm", "xsf")
+             "xperm", "xsf", "h", "hsf", "out_rows")
     P = T * k
     y_fused = torch.empty_like(x)
     m.forward(x, w, y=y_fused)
@@ -415,9 +417,9 @@ def test_decode_route_group_launch_equals_the_stages(T, d, F, E, k):
     assert m.sync_status() == moe.MOE_OK
     for n in names:
         a, b = fused[n], staged[n]
-        if n == "xperm":
+        if n in ("xperm", "h"):
             a, b = a[:, :P], b[:, :P]
-        elif n == "xsf":
+        elif n in ("xsf", "hsf"):
             a, b = a[:, :, :P], b[:, :, :P]
         assert np.array_equal(a.view(np.uint8), b.view(np.uint8)), n
     assert torch.equal(y_fused.view(torch.int16), y_stages.view(torch.int16))
