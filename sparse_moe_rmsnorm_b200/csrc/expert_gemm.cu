@@ -38,6 +38,15 @@
 // Down epilogue: o = w_token * (D + b2) written to the pair's expert-sorted
 //   row; the combine kernel adds a token's rows to its residual (weighted
 //   combine, "gpt-oss-20B" page section 3.4; pnsm.cn overview 2.2).
+// MODE_FFN (decode-sized batches, d_model == d_ff): one launch walks the
+//   gate/up items, then the down items, with the same per-item code as the two
+//   separate launches.  A gate/up item's eight epilogue warps each count their
+//   h stores into the token block's counter once they are fenced; a down item's
+//   B producer and scale-factor warps wait (bounded) until the counter reaches
+//   eight per gate/up weight block, and the B producer then orders its TMA reads
+//   of h after that acquire (a proxy fence).  Every CTA takes its gate/up items
+//   before its down items and only down items wait, on gate/up items, so every
+//   wait ends once the grid is resident.
 //
 // Warp roles (512 threads): 0 TMA producer of A (weights), 3 TMA producer of
 // B (activations), 1 MMA issue, 2 TMEM allocation and (per-item scale factors)
