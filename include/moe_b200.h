@@ -83,7 +83,7 @@ typedef struct {
 typedef struct moe_ctx moe_ctx_t;
 
 /* Create a context for `shape` on the current CUDA device.  Allocates the
- * device workspace sized for shape->T_max (routing arrays, the fp16 normalised
+ * device workspace sized for shape->T_max (routing arrays, the fp32 normalised
  * activations, the expert-sorted activations and the SwiGLU output h in the
  * E4M3 terms the block-scaled expert GEMMs read, and the fp32
  * weighted expert rows [T_max*k, d]).  The context owns the workspace; free it with
@@ -98,8 +98,11 @@ MOE_API int moe_destroy(moe_ctx_t *ctx);
 /* The whole block for T tokens (0 <= T <= T_max, 1 <= top_k <= shape.top_k):
  * route (RMSNorm, router, top-k, softmax), group the (token, expert) pairs by
  * expert, gate/up grouped GEMM with the SwiGLU epilogue, down grouped GEMM
- * with the routing-weight scatter-add, and the bf16 output cast.  y must not
- * alias x or any weight.  topk_idx_out / topk_w_out may be NULL; when given
+ * with each row scaled by its routing weight, and y = x + the token's rows in
+ * a fixed order, cast to bf16.  It is the stage calls below, except that a
+ * decode-sized batch (T <= 64, d_model <= 3072) routes and groups in one
+ * launch and, when d_model == d_ff, runs both GEMMs as moe_expert_ffn: the
+ * outputs equal the stages' bit for bit.  y must not alias x or any weight.  topk_idx_out / topk_w_out may be NULL; when given
  * they receive the chosen experts (in descending logit order) and their
  * softmax weights. */
 MOE_API int moe_forward(moe_ctx_t *ctx, int T,
@@ -112,7 +115,7 @@ MOE_API int moe_forward(moe_ctx_t *ctx, int T,
                 void *stream);
 
 /* The five stages of moe_forward, callable one by one on the same context
- * and stream, in this order (moe_forward is exactly these five calls):
+ * and stream, in this order:
  *   moe_route        RMSNorm, router logits, top-k and softmax;
  *   moe_group        expert histogram, prefix sum and the stable permutation
  *                    of (token, expert) pairs into expert-contiguous rows,
@@ -131,7 +134,16 @@ MOE_API int moe_forward(moe_ctx_t *ctx, int T,
  * for batches over 64 tokens, moe_expert_up's pass plan) before it waits for
  * the kernel before it: call it right after moe_expert_up (a call
  * in another order computes nothing useful, but every row index it uses stays
- * inside the workspace). */
+ * inside the workspace).
+ *
+ * moe_expert_ffn runs moe_expert_up and moe_expert_down as one persistent
+ * launch, for decode-sized batches (T <= 64, top_k * T <= 512) of a context with
+ * d_model == d_ff: a down work item starts once every gate/up item of its token
+ * block has written its h rows (per-token-block counters in the workspace,
+ * zeroed by moe_group and by moe_forward's route + group launch, so a moe_group
+ * must come before every moe_expert_ffn).  Same outputs as the two calls, bit for
+ * bit.  Returns MOE_ERR_UNSUPPORTED (and launches nothing) for other batches and
+ * shapes: call the two stages then. */
 MOE_API int moe_route(moe_ctx_t *ctx, int T, const uint16_t *x, const uint16_t *norm_scale,
               const uint16_t *router_w, const float *router_b, int top_k, void *stream);
 MOE_API int moe_group(moe_ctx_t *ctx, int T, int top_k, void *stream);
@@ -139,6 +151,9 @@ MOE_API int moe_expert_up(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w13_c
                   const uint16_t *b13, const uint8_t *w2_scales, void *stream);
 MOE_API int moe_expert_down(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w2_codes, const uint8_t *w2_scales,
                     const uint16_t *b2, void *stream);
+MOE_API int moe_expert_ffn(moe_ctx_t *ctx, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
+                   const uint16_t *b13, const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+                   void *stream);
 MOE_API int moe_finalize(moe_ctx_t *ctx, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,
                  float *topk_w_out, void *stream);
 

@@ -21,7 +21,7 @@ __all__ = [
     "MOE_OK", "MOE_ERR_ARG", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT", "MOE_ERR_UNSUPPORTED", "MOE_ERR_NOMEM",
     "MoEError", "MoEShape", "MoEWeights", "MoE", "lib", "library_path",
     "moe_init", "moe_destroy", "moe_forward", "moe_route", "moe_group", "moe_expert_up", "moe_expert_down",
-    "moe_finalize", "moe_copy_workspace", "moe_sync_status", "moe_set_wait_limit_ns",
+    "moe_expert_ffn", "moe_finalize", "moe_copy_workspace", "moe_sync_status", "moe_set_wait_limit_ns",
     "moe_selftest_wait_timeout", "moe_debug_decode", "moe_debug_plan", "moe_strerror", "moe_version", "WS",
     "moe_forward_noalloc", "MOE_NOALLOC_MAX_TOKENS",
 ]
@@ -63,6 +63,7 @@ _SIGS = {
     "moe_group": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "moe_expert_up": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5),
     "moe_expert_down": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4),
+    "moe_expert_ffn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 7),
     "moe_finalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5),
     "moe_copy_workspace": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                                           ctypes.c_void_p]),
@@ -162,6 +163,17 @@ def moe_expert_up(ctx, T, top_k, w13_codes, w13_scales, b13, w2_scales, stream=N
 def moe_expert_down(ctx, T, top_k, w2_codes, w2_scales, b2, stream=None) -> None:
     _check(lib().moe_expert_down(ctx, int(T), int(top_k), _ptr(w2_codes), _ptr(w2_scales), _ptr(b2),
                                  _stream(stream)), "moe_expert_down")
+
+
+def moe_expert_ffn(ctx, T, top_k, w13_codes, w13_scales, b13, w2_codes, w2_scales, b2, stream=None) -> bool:
+    """Both expert GEMMs in one launch; False (nothing launched) where the batch or shape does
+    not allow it, and the caller runs moe_expert_up and moe_expert_down."""
+    rc = lib().moe_expert_ffn(ctx, int(T), int(top_k), _ptr(w13_codes), _ptr(w13_scales), _ptr(b13),
+                              _ptr(w2_codes), _ptr(w2_scales), _ptr(b2), _stream(stream))
+    if rc == MOE_ERR_UNSUPPORTED:
+        return False
+    _check(rc, "moe_expert_ffn")
+    return True
 
 
 def moe_finalize(ctx, T, top_k, x, y, topk_idx_out=None, topk_w_out=None, stream=None) -> None:

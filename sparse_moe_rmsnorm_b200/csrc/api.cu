@@ -394,6 +394,20 @@ int moe_expert_down(moe_ctx_t *c, int T, int top_k, const uint8_t *w2_codes, con
     return gemm_launch(c, MODE_DOWN, T, top_k, w2_codes, w2_scales, b2, nullptr, static_cast<cudaStream_t>(stream));
 }
 
+int moe_expert_ffn(moe_ctx_t *c, int T, int top_k, const uint8_t *w13_codes, const uint8_t *w13_scales,
+                   const uint16_t *b13, const uint8_t *w2_codes, const uint8_t *w2_scales, const uint16_t *b2,
+                   void *stream) {
+    int rc = check_call(c, T, top_k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned32(w13_codes) || !aligned16(w13_scales) || !aligned16(b13) || !aligned32(w2_codes) ||
+        !aligned16(w2_scales) || !aligned16(b2))
+        return MOE_ERR_ARG;
+    if (T > 64 || T * top_k > 512) return MOE_ERR_UNSUPPORTED;
+    return ffn_launch(c, T, top_k, w13_codes, w13_scales, b13, w2_codes, w2_scales, b2,
+                      static_cast<cudaStream_t>(stream));
+}
+
 int moe_finalize(moe_ctx_t *c, int T, int top_k, const uint16_t *x, uint16_t *y, int32_t *topk_idx_out,
                  float *topk_w_out, void *stream) {
     int rc = check_call(c, T, top_k);
@@ -431,8 +445,7 @@ int moe_forward(moe_ctx_t *c, int T, const uint16_t *x, const uint16_t *router_w
         if (launch_route_group_small(rp, group_params(c, T, top_k), route_group_barrier(c), c->wait_limit_ns,
                                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        rc = ffn_launch(c, T, top_k, w13_codes, w13_scales, b13, w2_codes, w2_scales, b2,
-                        static_cast<cudaStream_t>(stream));
+        rc = moe_expert_ffn(c, T, top_k, w13_codes, w13_scales, b13, w2_codes, w2_scales, b2, stream);
         if (rc == MOE_OK) return moe_finalize(c, T, top_k, x, y, topk_idx_out, topk_w_out, stream);
         if (rc != MOE_ERR_UNSUPPORTED) return rc;
     } else {

@@ -500,6 +500,10 @@ __global__ void __launch_bounds__(1024) group_permute_kernel(const GroupParams p
     for (int i = threadIdx.x; i < 32 * 257; i += blockDim.x) (&wcnt[0][0])[i] = 0;
     pdl_wait();
     pdl_trigger();
+    // the fused decode GEMM's per-token-block counters start at zero (after the wait: the
+    // previous layer step's GEMM has finished with them)
+    if (blockIdx.x == 0 && p.h_ready)
+        for (int i = threadIdx.x; i < p.n_h_ready; i += blockDim.x) p.h_ready[i] = 0u;
     __syncthreads();
     const int seg = (P + 31) / 32;
     const int beg = warp * seg, end = min(P, beg + seg);

@@ -28,7 +28,8 @@ def lib():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for s in ["moe_init", "moe_forward", "moe_destroy", "moe_route", "moe_group", "moe_expert_up",
-              "moe_expert_down", "moe_finalize", "moe_sync_status", "moe_strerror", "moe_forward_noalloc"]:
+              "moe_expert_down", "moe_expert_ffn", "moe_finalize", "moe_sync_status", "moe_strerror",
+              "moe_forward_noalloc"]:
         assert s in syms
 
 
@@ -64,6 +65,7 @@ def test_strings_and_shape_validation_without_gpu(lib):
 def test_stage_calls_reject_null_context(lib):
     assert lib.moe_group(None, 4, 4, None) == moe.MOE_ERR_ARG
     assert lib.moe_expert_up(None, 4, 4, None, None, None, None, None) == moe.MOE_ERR_ARG
+    assert lib.moe_expert_ffn(None, 4, 4, *([None] * 7)) == moe.MOE_ERR_ARG
     assert lib.moe_copy_workspace(None, 0, None, 0, None) == moe.MOE_ERR_ARG
 
 

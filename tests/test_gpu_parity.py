@@ -415,6 +415,17 @@ def test_decode_route_group_launch_equals_the_stages(T, d, F, E, k):
     moe.moe_finalize(m.ctx, T, k, x, y_stages)
     staged = {n: m.workspace(n, T).cpu().numpy() for n in names}
     assert m.sync_status() == moe.MOE_OK
+    # the GEMM stages as one launch where the shape allows it (moe_expert_ffn), else the two
+    y_ffn = torch.empty_like(x)
+    moe.moe_route(m.ctx, T, x, w.norm_scale, w.router_w, w.router_b, k)
+    moe.moe_group(m.ctx, T, k)
+    if not moe.moe_expert_ffn(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13, w.w2_codes, w.w2_scales, w.b2):
+        assert d != F
+        moe.moe_expert_up(m.ctx, T, k, w.w13_codes, w.w13_scales, w.b13, w.w2_scales)
+        moe.moe_expert_down(m.ctx, T, k, w.w2_codes, w.w2_scales, w.b2)
+    moe.moe_finalize(m.ctx, T, k, x, y_ffn)
+    assert m.sync_status() == moe.MOE_OK
+    assert torch.equal(y_ffn.view(torch.int16), y_stages.view(torch.int16))
     for n in names:
         a, b = fused[n], staged[n]
         if n in ("xperm", "h"):
