@@ -347,8 +347,8 @@ def gemm_roofline(which, t_s, cnt, tensor_bound, peaks, peak_key, workload):
 
 
 def measure_workload(name, args, rank, world, local_rank, main):
-    """Time one workload: K steps of moe_forward (the value), then K steps of the five stage calls
-    with the two GEMMs bracketed by events, per-stage times, and (main line only) the end-to-end
+    """Time one workload: K steps of moe_forward (the value), then K steps of the stage calls
+    with the GEMM launches bracketed by events, per-stage times, and (main line only) the end-to-end
     number and the CPU oracle sample.  Returns the measurements (rank 0) or None."""
     import torch
     import sparse_moe_rmsnorm_b200 as moe
@@ -375,7 +375,7 @@ def measure_workload(name, args, rank, world, local_rank, main):
 
     def step(timed=False):
         """One step: the block on every layer.  timed=False: moe_forward (the public call);
-        timed=True: the five stage calls moe_forward is made of, with the two GEMMs bracketed
+        timed=True: the stage calls moe_forward is made of, with the GEMM launches bracketed
         by events on the launching stream."""
         cur = x
         for l, w in enumerate(weights):
