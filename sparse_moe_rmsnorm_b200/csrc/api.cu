@@ -1,5 +1,6 @@
 // C ABI of the B200 MoE block: context and workspace management, argument
-// validation, TMA descriptor encoding and the five stage launches.
+// validation, TMA descriptor encoding and the stage launches (moe_forward's
+// decode-sized path fuses route + group and the two GEMMs into one launch each).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
