@@ -254,6 +254,27 @@ def test_shapes(shape):
     check(custom_layer(**shape, k=k, seed=sum(shape.values())), k, label=str(shape))
 
 
+# d_model or d_ff above 3072, up to the largest the library accepts (6144): decode-sized batches
+# route in the 8-tokens-per-CTA kernel and run the GEMMs on stacked 16-row token blocks with
+# per-stage scale factors (an item's K stages no longer fit TMEM beside the accumulators); larger
+# batches run 192-row blocks with a ring of two stages.  The widest large-batch case is checked on
+# sampled rows, as the oracle's cost grows with d_model x d_ff.
+WIDE = [
+    dict(T=16, d=6144, F=6144, E=4, k=2, rows=None),
+    dict(T=48, d=4096, F=1024, E=8, k=4, rows=None),     # d_model != d_ff: the GEMMs in two launches
+    dict(T=300, d=6144, F=6144, E=4, k=2, rows=24),
+]
+
+
+@pytest.mark.parametrize("shape", WIDE, ids=lambda s: "T%d_d%d_F%d_E%d_k%d" % tuple(list(s.values())[:5]))
+def test_wide_model_dims(shape):
+    shape = dict(shape)
+    k, n_rows = shape.pop("k"), shape.pop("rows")
+    inp = custom_layer(**shape, k=k, seed=sum(shape.values()))
+    rows = None if n_rows is None else np.sort(np.random.default_rng(5).choice(shape["T"], n_rows, replace=False))
+    check(inp, k, rows=rows, label=str(shape))
+
+
 @pytest.mark.parametrize("T", [24, 200])
 def test_scale_extremes(T):
     """E8M0 exponents far from 127, outside the layers' distribution, at the block's stated
