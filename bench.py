@@ -462,34 +462,60 @@ def measure_workload(name, args, rank, world, local_rank, main):
     counts = m.workspace("counts", T).cpu().numpy()
     cnt = algorithmic_counts(cfg, counts)
 
-    # ---- end to end through the public API: pinned host x in, y out, every step
+    # ---- end to end through the public API: every step copies its tokens in from pinned host
+    # memory, runs the block on every layer (moe_forward) and copies the result back.  As a serving
+    # loop would, the copies run on two copy streams against double-buffered device tokens, so a
+    # step's copies overlap the compute of the steps around it; events order each buffer's reuse.
     e2e = None
     if main:
         x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
         y_host = torch.empty_like(x_host).pin_memory()
-        x_dev = torch.empty_like(x)
-        for _ in range(max(1, args.warmup)):
-            m.forward_host(x_host, w0, y_host, x_dev, bufs[0])
+        h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        xd = [torch.empty_like(x) for _ in range(2)]
+        yd = [torch.empty_like(x) for _ in range(2)]
+        ev = {k_: [torch.cuda.Event() for _ in range(2)] for k_ in ("h2d", "fwd", "d2h")}
+
+        def e2e_step(i):
+            b = i % 2
+            with torch.cuda.stream(h2d_s):
+                h2d_s.wait_event(ev["fwd"][b])          # the step before last has read xd[b]
+                xd[b].copy_(x_host, non_blocking=True)
+                ev["h2d"][b].record(h2d_s)
+            stream.wait_event(ev["h2d"][b])
+            stream.wait_event(ev["d2h"][b])             # ... and its result has left yd[b]
+            cur = xd[b]
+            for l, w in enumerate(weights):
+                out = yd[b] if l == layers - 1 else bufs[l % 2]
+                m.forward(cur, w, y=out, stream=stream)
+                cur = out
+            ev["fwd"][b].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev["fwd"][b])
+                y_host.copy_(yd[b], non_blocking=True)
+                ev["d2h"][b].record(d2h_s)
+            return b
+
+        for i in range(max(1, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize()
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            if layers == 1:
-                m.forward_host(x_host, w0, y_host, x_dev, bufs[0])
-            else:
-                x_dev.copy_(x_host, non_blocking=True)
-                cur = x_dev
-                for l, w in enumerate(weights):
-                    out = bufs[l % 2]
-                    m.forward(cur, w, y=out)
-                    cur = out
-                y_host.copy_(cur, non_blocking=True)
+        h2d_s.wait_event(e0)
+        d2h_s.wait_event(e0)
+        for i in range(args.steps):
+            last = e2e_step(i)
+        stream.wait_event(ev["d2h"][last])               # the last result is on the host
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        # the host result is the block's output on these tokens, bit for bit
+        y_ref = step()
+        torch.cuda.synchronize()
+        if not torch.equal(y_host, y_ref.cpu()):
+            raise RuntimeError("end-to-end result differs from moe_forward's (%s)" % name)
         e2e = {"value": job_tokens_per_s(e2e_ms, T, args.steps, world), "unit": "tokens/s",
                "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2}
     m.close()

@@ -319,10 +319,16 @@ class MoE:
 
     def forward_host(self, x_host, w: MoEWeights, y_host, x_dev, y_dev, top_k: Optional[int] = None,
                      stream=None):
-        """End-to-end call from pinned host memory: copy x in, run the block, copy y out."""
-        x_dev.copy_(x_host, non_blocking=True)
-        self.forward(x_dev, w, top_k=top_k, y=y_dev, stream=stream)
-        y_host.copy_(y_dev, non_blocking=True)
+        """End-to-end call from pinned host memory: copy x in, run the block, copy y out, all
+        three in order on `stream` (default: the current stream)."""
+        import torch
+        s = torch.cuda.current_stream() if stream is None else stream
+        if isinstance(s, int):
+            s = torch.cuda.ExternalStream(s)
+        with torch.cuda.stream(s):
+            x_dev.copy_(x_host, non_blocking=True)
+            self.forward(x_dev, w, top_k=top_k, y=y_dev, stream=s)
+            y_host.copy_(y_dev, non_blocking=True)
         return y_host
 
     def workspace(self, name: str, T: int, top_k: Optional[int] = None, stream=None):

@@ -512,6 +512,28 @@ def test_repeat_calls_and_smaller_T():
     m.close()
 
 
+def test_forward_host_on_a_side_stream():
+    """The end-to-end helper: pinned host tokens in, the host result out, the copies and the block
+    ordered on the stream given; the same bits as a device call."""
+    inp = custom_layer(T=32, d=256, F=256, E=8, k=4, seed=3)
+    w = moe.MoEWeights.from_numpy(inp)
+    m = moe.MoE(32, 256, 256, 8, 4)
+    x = _bf16_dev(inp["x"])
+    y_ref = m.forward(x, w)
+    torch.cuda.synchronize()
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev, y_dev = torch.empty_like(x), torch.empty_like(x)
+    s = torch.cuda.Stream()
+    for _ in range(3):
+        y_host.zero_()
+        m.forward_host(x_host, w, y_host, x_dev, y_dev, stream=s)
+        s.synchronize()
+        assert torch.equal(y_host, y_ref.cpu())
+    assert m.sync_status() == moe.MOE_OK
+    m.close()
+
+
 def test_empty_batch_is_a_no_op():
     inp = custom_layer(T=4, d=128, F=128, E=8, k=4, seed=1)
     w = moe.MoEWeights.from_numpy(inp)
