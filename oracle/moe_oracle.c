@@ -17,8 +17,9 @@
  *   3. Top-k (k = 4) of the logits, ties to the lower expert index
  *      (pnsm.cn overview section 2.2; config.json read-out on youleyou.com:
  *      experts_per_token 4).
- *   4. Softmax over the k chosen logits (pnsm.cn overview section 2.2:
- *      "选中专家做 softmax 加权"; "gpt-oss-20B" page section 3.4).
+ *   4. Softmax over the k chosen logits (pnsm.cn overview section 2.2: the
+ *      chosen experts' outputs are weighted by a softmax over them;
+ *      "gpt-oss-20B" page section 3.4).
  *   5. Per chosen expert, gated SwiGLU with the clamp at 7 and the "+1"
  *      ("gpt-oss-20B" page section 3.3 "SwiGLU：带有夹断和残差的门控激活"):
  *        z = W13 xn + b13 (2F values: rows [0,F) gate, [F,2F) linear)
